@@ -1,0 +1,104 @@
+"""8-bit Sage decode, following the pages' formula step by step (test infrastructure only).
+
+Source: "FlashInfer PrimTS, Sage Attention 도입으로 8비트 양자화 및 성능 최적화
+달성", section "코드 분석" item 1 (README "Sage attention"):
+
+    S[r][c] = sfQ[blkQ(r)] * sfK[blkK(c)] * (Q8 . K8^T)[r][c]
+    P       = softmax_row(S), quantized to E4M3 as 448 * p
+    O[r][d] = sfV[d] * (sum_c P8[r][c] * V8[c][d]) / (448 * l[r])  (+ v_mean[d])
+
+and item 4 of the same section: the Q and K scales enter before the row max
+and the exponential, P is E4M3 with the static factor 448, and the V scales
+are applied per channel in the epilogue.  The caller supplies the 8-bit
+tensors and all scales, which must be finite and positive and are not checked
+(same item 1).
+
+Layout (one decode token per request, DECODE mode):
+  q8      int8  [B, Hq, D]           sf_q  float32 [B, Hq]       (blkQ = one row)
+  k8 pool int8  [num_slots, Hkv, D]  sf_k  float32 [num_slots // k_block, Hkv]
+  v8 pool uint8 [num_slots, Hkv, D]  (E4M3 codes)
+  sf_v, v_mean float32 [Hkv, D]      (v_mean optional)
+
+Readings where the formula leaves a step open (listed in the design notes):
+* blkK(c) is the physical 64-key block of key c's slot, slot // k_block, so a
+  scale travels with its page.
+* softmax_row takes the maximum m over the request's whole row of keys; the
+  top key therefore quantises to exactly 448.
+* l[r] = sum_c exp(S[r][c] - m) of the unquantised probabilities.
+* E4M3 rounding is round-to-nearest-even with saturation.
+* The quantisation code is an integer decided by floating point, so it is
+  decided in the kernel's precision: S is formed in float32 as
+  fp32(fp32(sfQ * sfK) * fp32(dot)) (the integer dot is exact: |dot| <=
+  127 * 127 * 128 < 2**24), and m is the float32 row maximum.  Everything
+  after that (exp, 448 * p, the sums, the epilogue) is float64.
+* There is no extra 1/sqrt(d) factor: the formula has none, so a caller folds
+  any softmax scale into sfQ.
+* An empty row (L = 0) gives O = v_mean (zero if absent).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import gather_slots
+from .codecs import e4m3_to_f64, f64_to_e4m3
+
+
+def sage_scores_f32(q8_row: np.ndarray, k8_rows: np.ndarray, sf_q: float, sf_k_rows: np.ndarray) -> np.ndarray:
+    """S for one query row over keys: float32 (sfQ * sfK) * float32(exact int dot).
+
+    q8_row [D] int8, k8_rows [N, D] int8, sf_k_rows [N] float32 (the scale of
+    each key's block).  Returns float32 [N].
+    """
+    dot = k8_rows.astype(np.int64) @ q8_row.astype(np.int64)          # exact integers
+    scale = np.float32(sf_q) * sf_k_rows.astype(np.float32)           # fp32 product, rounded
+    return (scale * dot.astype(np.float32)).astype(np.float32)        # fp32 product, rounded
+
+
+def sage_row(q8_row, k8_rows, v8_rows, sf_q, sf_k_rows, sf_v, v_mean, quantize_p: bool = True):
+    """The Sage formula for one query row; returns O [D] float64.
+
+    v8_rows [N, D] uint8 E4M3 codes, sf_v and v_mean [D].  ``quantize_p=False``
+    replaces the E4M3 step on 448 * p by the identity (a switch used to tie
+    this function to plain softmax attention in the tests).
+    """
+    D = v8_rows.shape[1] if v8_rows.ndim == 2 else len(sf_v)
+    vm = np.zeros(D) if v_mean is None else np.asarray(v_mean, dtype=np.float64)
+    if k8_rows.shape[0] == 0:
+        return vm.copy()
+    S = sage_scores_f32(q8_row, k8_rows, sf_q, sf_k_rows)             # step 1: scores
+    m = np.float32(S.max())                                           # step 2: row max (fp32)
+    p = np.exp(S.astype(np.float64) - np.float64(m))                  # step 3: exp(S - m) in (0, 1]
+    l = p.sum()                                                       # unquantised row sum
+    if quantize_p:
+        P = e4m3_to_f64(f64_to_e4m3(448.0 * p))                       # step 4: E4M3(448 p)
+    else:
+        P = 448.0 * p
+    V = e4m3_to_f64(v8_rows)                                          # exact decode of V8
+    acc = P @ V                                                       # step 5: sum_c P8 V8
+    return np.asarray(sf_v, dtype=np.float64) * acc / (448.0 * l) + vm   # step 6: epilogue
+
+
+def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_lens,
+                page_size: int, k_block: int = 64, quantize_p: bool = True) -> np.ndarray:
+    """Sage DECODE over the paged cache; returns O [B, Hq, D] float64.
+
+    Keys are gathered through the page table exactly as in the bf16 path
+    (``oracle.attention.gather_slots``); key c's K scale is
+    sf_k[slot(c) // k_block][h_kv]; query head h reads KV head h // (Hq // Hkv).
+    """
+    B, Hq, D = q8.shape
+    Hkv = k8_pool.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    for r in range(B):
+        L = int(seq_lens[r])
+        slots = gather_slots(page_table, L, page_size, r)
+        blocks = slots // k_block
+        for hk in range(Hkv):
+            k8 = k8_pool[slots, hk, :]
+            v8 = v8_pool[slots, hk, :]
+            sfk = sf_k[blocks, hk]
+            vm = None if v_mean is None else v_mean[hk]
+            for h in range(hk * G, (hk + 1) * G):
+                out[r, h] = sage_row(q8[r, h], k8, v8, sf_q[r, h], sfk, sf_v[hk], vm, quantize_p)
+    return out

@@ -1,0 +1,113 @@
+"""Pins for the oracle's integer plan.
+
+Hand-derived golden cases (tests/golden/plan_cases.json) and invariants that
+any correct split-KV plan has: the splits of a request cover [0, L) exactly
+once, in order, on tile boundaries; items run longest first; the item count
+stays within the host-side bound used to size the grid; and the plan depends
+only on the lengths.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import plan as op
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "plan_cases.json")))
+
+
+@pytest.mark.parametrize("case", GOLDEN["cases"], ids=[c["name"] for c in GOLDEN["cases"]])
+def test_hand_derived_plans(case):
+    got = op.plan(case["mode"], case["seq_lens"], case.get("cu_seqlens_q"), hkv=case["hkv"],
+                  page_size=case["page_size"], num_sms=case["num_sms"], max_splits=case["max_splits"],
+                  max_q_tokens=(case.get("cu_seqlens_q") or [0])[-1])
+    e = case["expect"]
+    assert got["tile"] == e["tile"]
+    assert got["chunk_tiles"] == e["chunk_tiles"]
+    assert got["req_splits"] == e["req_splits"]
+    assert got["req_base"] == e["req_base"]
+    assert [list(x) for x in got["items"]] == e["items"]
+
+
+def _check_decode_invariants(lens, hkv, P, num_sms, max_splits):
+    pl = op.plan(op.MODE_DECODE, lens, hkv=hkv, page_size=P, num_sms=num_sms, max_splits=max_splits)
+    T = pl["tile"]
+    assert T == max(64, P)
+    assert pl["num_items"] <= op.max_items(op.MODE_DECODE, len(lens), hkv, num_sms)
+    by_req = {}
+    for (r, s, a, b) in pl["items"]:
+        by_req.setdefault(r, []).append((s, a, b))
+    sizes = [b - a for (_, _, a, b) in pl["items"]]
+    assert sizes == sorted(sizes, reverse=True)
+    for r, L in enumerate(lens):
+        parts = sorted(by_req[r])
+        assert [s for s, _, _ in parts] == list(range(pl["req_splits"][r]))
+        assert len(parts) <= max(1, max_splits)
+        assert parts[0][1] == 0 and parts[-1][2] == L
+        for (s0, a0, b0), (s1, a1, b1) in zip(parts, parts[1:]):
+            assert b0 == a1
+        for (_, a, b) in parts:
+            assert a % T == 0 and a < b or L == 0
+    assert pl["req_base"][-1] == pl["num_items"]
+
+
+def test_decode_invariants_random():
+    rng = np.random.default_rng(30)
+    for _ in range(300):
+        B = int(rng.integers(1, 70))
+        lens = [int(x) for x in rng.integers(0, 20000, B)]
+        if rng.random() < 0.3:
+            lens[int(rng.integers(0, B))] = 0
+        hkv = int(rng.choice([1, 2, 4, 8]))
+        P = int(rng.choice([1, 16, 64, 128, 256]))
+        _check_decode_invariants(lens, hkv, P, int(rng.integers(1, 200)), int(rng.integers(1, 80)))
+
+
+def test_decode_plan_at_the_workload_shapes():
+    # Llama-3-8B decode shape and the 128k long-context shape on 148 SMs
+    rng = np.random.default_rng(31)
+    lens = [int(x) for x in rng.integers(512, 8193, 64)]
+    _check_decode_invariants(lens, 8, 1, 148, 64)
+    pl = op.plan(op.MODE_DECODE, [131072] * 8, hkv=8, page_size=64, num_sms=148, max_splits=64)
+    # total = 8 * 2048 * 8 tile-heads over 148 * 8 slots: chunk = ceil(131072 / 1184) = 111 tiles
+    assert pl["chunk_tiles"] == 111
+    assert pl["req_splits"] == [19] * 8
+    assert pl["num_items"] == 152 <= op.max_items(op.MODE_DECODE, 8, 8, 148)
+
+
+def test_plan_is_a_function_of_lengths_only():
+    rng = np.random.default_rng(32)
+    lens = [int(x) for x in rng.integers(1, 5000, 17)]
+    a = op.plan(op.MODE_DECODE, lens, hkv=4, page_size=16, num_sms=148, max_splits=16)
+    b = op.plan(op.MODE_DECODE, np.array(lens), hkv=4, page_size=16, num_sms=148, max_splits=16)
+    assert a == b
+
+
+def test_extend_invariants_random():
+    rng = np.random.default_rng(33)
+    for _ in range(200):
+        B = int(rng.integers(1, 12))
+        new = rng.integers(0, 700, B)
+        pre = rng.integers(0, 3000, B)
+        cu = np.concatenate([[0], np.cumsum(new)]).tolist()
+        lens = (new + pre).tolist()
+        pl = op.plan(op.MODE_EXTEND, lens, cu, hkv=8, page_size=16, num_sms=148, max_q_tokens=cu[-1])
+        assert pl["num_items"] <= op.max_items(op.MODE_EXTEND, B, 8, 148, cu[-1])
+        seen = {}
+        for (r, t, q0, q1) in pl["items"]:
+            seen.setdefault(r, []).append((t, q0, q1))
+        for r in range(B):
+            parts = sorted(seen.get(r, []))
+            assert sum(q1 - q0 for _, q0, q1 in parts) == new[r]
+            for (t, q0, q1) in parts:
+                assert q0 == 128 * t and 0 < q1 - q0 <= 128
+        keys = [-(-(lens[r] - new[r] + q1) // 128) for (r, t, q0, q1) in pl["items"]]
+        assert keys == sorted(keys, reverse=True)
+
+
+def test_rejects_negative_lengths():
+    with pytest.raises(ValueError):
+        op.plan(op.MODE_DECODE, [5, -1], hkv=1, page_size=1, num_sms=1)
+    with pytest.raises(ValueError):
+        op.plan(op.MODE_EXTEND, [5], [0, 6], hkv=1, page_size=1, num_sms=1)
