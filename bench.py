@@ -1,0 +1,401 @@
+"""Benchmark of the paged-KV attention library on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Default workload: DECODE at the Llama-3-8B attention shape (batch 64, KV
+lengths uniform in 512..8192, Hq 32, Hkv 8, D 128, bf16, page size 1 with
+shuffled slots in a 600k-slot pool).  One step = one attn_plan followed by 32
+layer calls of attn_decode_paged, each layer with its own pool (78.6 GB in
+total, so every step reads inputs far larger than L2).  The metric is the
+decode's algorithmic KV bandwidth: K and V rows read once, slot ids, Q and O,
+divided by the device time.  Other workloads (``--workload``):
+decode_long_llama3_70b, extend_prefix, sage_decode, decode_tiny.
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
+replica on its own GPU (no collective on the data path); the time is the max
+over ranks and the value the sum of all ranks' bytes over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode KV GB/s (% HBM peak); paged extend TFLOP/s (% bf16 peak)"
+
+
+# --------------------------------------------------------------------------- utilities
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "paged_kv_flashattention_split_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key: str, src_hash: str):
+    """ncu DRAM bytes per launch recorded under profiles/ for this exact kernel source, else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel_key)
+        if rec and rec.get("source_hash") == src_hash:
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- decode workload
+
+class DecodeWorkload:
+    """plan + L layer decode calls; layers rotate over `distinct_pools` pools."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        import paged_kv_flashattention_split_b200 as pa
+        self.pa, self.spec, self.dev = pa, spec, device
+        self.batch = wl.make_batch(spec, device)
+        n_pools = spec.distinct_pools or spec.layers
+        self.pools = [wl.make_bf16_pools(spec, self.batch, l, device) for l in range(n_pools)]
+        self.q = [wl.make_bf16_queries(spec, spec.batch, l, device) for l in range(spec.layers)]
+        self.out = [torch.empty_like(x) for x in self.q]
+        self.params = pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, spec.head_dim,
+                                     spec.page_size, max_kv_len=self.batch.page_table.shape[1] * spec.page_size)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        self.stream = torch.cuda.current_stream()
+        L = self.batch.seq_lens.cpu().tolist()
+        self.layer_bytes = wl.decode_kv_bytes(L, spec.hkv, spec.head_dim, 2, spec.page_size, spec.hq, 2, 2)
+        self.step_bytes = self.layer_bytes * spec.layers
+        self.launches_per_step = 1 + 2 * spec.layers
+
+    def pool(self, l):
+        return self.pools[l % len(self.pools)]
+
+    def layer(self, l):
+        k, v = self.pool(l)
+        self.pa.attn_decode_paged(self.params, self.ws, self.q[l], k, v, self.batch.page_table,
+                                  self.spec.sm_scale, self.out[l])
+
+    def step(self, layer_events=None):
+        self.pa.attn_plan(self.params, self.batch.seq_lens, None, self.ws)
+        for l in range(self.spec.layers):
+            if layer_events is not None:
+                layer_events[l][0].record()
+            self.layer(l)
+            if layer_events is not None:
+                layer_events[l][1].record()
+
+    # end to end: inputs from pinned host buffers, result read back, every step
+    def setup_e2e(self):
+        self.h_q = [x.cpu().pin_memory() for x in self.q]
+        self.h_lens = self.batch.seq_lens.cpu().pin_memory()
+        self.h_table = self.batch.page_table.cpu().pin_memory()
+        self.h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in self.out]
+        self.e2e_h2d = sum(x.numel() * 2 for x in self.h_q) + self.h_lens.numel() * 4 + self.h_table.numel() * 4
+        self.e2e_d2h = sum(x.numel() * 2 for x in self.h_out)
+
+    def step_e2e(self):
+        self.batch.seq_lens.copy_(self.h_lens, non_blocking=True)
+        self.batch.page_table.copy_(self.h_table, non_blocking=True)
+        self.pa.attn_plan(self.params, self.batch.seq_lens, None, self.ws)
+        for l in range(self.spec.layers):
+            self.q[l].copy_(self.h_q[l], non_blocking=True)
+            self.layer(l)
+            self.h_out[l].copy_(self.out[l], non_blocking=True)
+
+    # the oracle on a bounded sample of the same workload (host cores)
+    def oracle_sample(self, seconds=12.0):
+        from oracle import attention as oa
+        spec = self.spec
+        t0 = time.perf_counter()
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        k, v = self.pool(0)
+        kb = k.view(torch.int16).cpu().numpy().view(np.uint16)
+        vb = v.view(torch.int16).cpu().numpy().view(np.uint16)
+        qb = self.q[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        prep = time.perf_counter() - t0
+        done, nbytes, r = 0.0, 0.0, 0
+        t0 = time.perf_counter()
+        while r < spec.batch and (time.perf_counter() - t0) < seconds:
+            oa.decode(qb[r:r + 1], kb, vb, table[r:r + 1], lens[r:r + 1], spec.page_size, spec.sm_scale)
+            nbytes += wl.decode_kv_bytes([int(lens[r])], spec.hkv, spec.head_dim, 2, spec.page_size, spec.hq, 2, 2)
+            r += 1
+        done = time.perf_counter() - t0
+        return nbytes, done, f"oracle.attention.decode on requests 0..{r - 1} of layer 0 ({r} of {spec.batch} requests, {int(lens[:r].sum())} keys); host copy {prep:.1f}s untimed"
+
+
+WORKLOADS = {
+    "decode_llama3_8b": (2, DecodeWorkload),
+    "decode_long_llama3_70b": (4, DecodeWorkload),
+    "decode_tiny": (1, DecodeWorkload),
+}
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_llama3_8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+
+    cfg_id, cls = WORKLOADS[args.workload]
+    spec = wl.CONFIGS[cfg_id]
+    hbm_peak, bf16_peak, bf16_sus, peak_src = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            if dist is not None:
+                dist.destroy_process_group()
+            return
+        run_reference(args, spec, cls)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(dev)
+    work = cls(spec, dev)
+    torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        work.step()
+    torch.cuda.synchronize()
+
+    # timed region: events on the launching stream, per-layer events for the decode call
+    layer_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(spec.layers)]
+    layer_ms = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start.record()
+        for s in range(args.steps):
+            work.step(layer_events)
+            if s == args.steps - 1:
+                pass
+        end.record()
+        torch.cuda.synchronize()
+        # per-layer durations of the last step (the events are re-recorded every step)
+        layer_ms = [a.elapsed_time(b) for a, b in layer_events]
+    total_ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = total_ms / args.steps
+    value = work.step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    work.setup_e2e()
+    for _ in range(2):
+        work.step_e2e()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(args.steps, 5))
+    e_start.record()
+    for _ in range(e_steps):
+        work.step_e2e()
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = work.step_bytes * world / (e2e_ms * 1e-3) / 1e9
+
+    avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
+    achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("decode_" + args.workload, source_hash("decode.cu", "common.cuh"))
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload,
+            "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
+            "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
+            "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
+            "step": "attn_plan + %d x attn_decode_paged" % spec.layers,
+            "l2": "inputs larger than L2 (each layer reads its own >1 GB pool)",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+            "kernel": "attn_decode_paged call (decode_splitkv_kernel + merge_kernel), per-layer CUDA events",
+            "peak_source": peak_src,
+        },
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(work.e2e_h2d),
+                "d2h_bytes_per_step": int(work.e2e_d2h), "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": work.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nbytes, secs, sample = work.oracle_sample()
+        line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, spec, cls):
+    """The oracle as it stands, on the host cores, on a bounded sample per step."""
+    from oracle import attention as oa
+    batch = wl.make_batch(spec, "cpu")
+    n_pools = 1
+    k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
+    q = wl.make_bf16_queries(spec, spec.batch, 0, "cpu")
+    kb = k.view(torch.int16).numpy().view(np.uint16)
+    vb = v.view(torch.int16).numpy().view(np.uint16)
+    qb = q.view(torch.int16).numpy().view(np.uint16)
+    table = batch.page_table.numpy()
+    lens = batch.seq_lens.numpy()
+    per_step = 2                         # requests per step: a bounded sample of the batch
+    times, nbytes = [], 0.0
+    r = 0
+    for s in range(args.warmup + args.steps):
+        rs = [(r + i) % spec.batch for i in range(per_step)]
+        r += per_step
+        t0 = time.perf_counter()
+        for x in rs:
+            oa.decode(qb[x:x + 1], kb, vb, table[x:x + 1], lens[x:x + 1], spec.page_size, spec.sm_scale)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            nbytes += sum(wl.decode_kv_bytes([int(lens[x])], spec.hkv, spec.head_dim, 2, spec.page_size, spec.hq, 2, 2) for x in rs)
+    total = sum(times)
+    value = nbytes / total / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]",
+                   "hq": spec.hq, "hkv": spec.hkv, "head_dim": spec.head_dim, "page_size": spec.page_size,
+                   "layers": spec.layers},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{per_step} requests of layer 0 per step, oracle.attention.decode in fp64"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

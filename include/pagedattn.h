@@ -1,0 +1,261 @@
+/*
+ * pagedattn.h - C ABI of a B200 (sm_100a) attention library over a paged KV cache.
+ *
+ * The library computes FlashAttention-style tiled, online-softmax attention
+ * over a two-level KV cache: a table maps (request, position) to a token slot
+ * ("req_to_token") and per-layer pools map a slot to that layer's K and V rows
+ * ("token_to_kv_pool")  ["Implement Flash Attention Back End in SGLang -
+ * Basics and KV Cache", KV-cache passage; "Flash Attention Backend in SGLang:
+ * Grundlagen und KV Cache optimal nutzen", req_to_token / token_to_kv_pool
+ * paragraph].  With a page size P > 1 the table holds page numbers
+ * ["PagedAttention: 优化 KV Cache 的管理和利用率", section 2, 工作原理]:
+ *
+ *     slot(r, j) = page_table[r * pt_pitch + j / P] * P + j % P
+ *
+ * Two forward modes are provided, DECODE (one query token per request) and
+ * EXTEND (new tokens attending causally to a cached prefix and to themselves)
+ * [forward modes in the same two SGLang pages], plus the 8-bit "Sage" decode
+ * ["FlashInfer PrimTS, Sage Attention 도입으로 8비트 양자화 및 성능 최적화 달성",
+ * section "코드 분석" items 1 and 4].
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers prefixed d_ or naming device tensors are DEVICE pointers; struct
+ *   pointers (pa_plan_params*, size_t*) are HOST pointers.  The caller owns
+ *   every buffer, including the plan workspace; the library allocates and
+ *   frees nothing and keeps no pointer between calls.
+ * - bf16 tensors are passed as raw 16-bit bit patterns (uint16_t); E4M3
+ *   tensors as raw bytes (uint8_t).
+ * - Layouts (row-major, innermost last):
+ *     K/V pools       [num_slots][Hkv][D]        per layer
+ *     page_table      int32 [B][pt_pitch]        page (or, for P = 1, slot) ids
+ *     DECODE Q, O     [B][Hq][D];  lse [B][Hq]
+ *     EXTEND Q, O     [sum_r n_r][Hq][D];  lse [sum_r n_r][Hq]
+ *   Query head h reads KV head h / (Hq / Hkv).
+ * - Every call only enqueues work on `stream` and never synchronises the host
+ *   (except pa_read_device_error), so a plan followed by per-layer calls can
+ *   be captured in a CUDA graph.  Launch geometry depends only on the host
+ *   parameters, never on device data.
+ * - Functions return a status and never throw.  Scale values and table
+ *   contents are not validated on the host; a slot or page id outside the pool
+ *   is skipped (its row reads as zero) and recorded in the workspace's device
+ *   error word, which pa_read_device_error reports as PA_ERR_DEVICE_INDEX.
+ * - Head dimension D must be 128; the page size must be a power of two
+ *   <= 256; Hq / Hkv must be 1, 2, 4 or 8.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,       /* NULL where required, inconsistent sizes, misaligned buffer,
+                               an input the mode does not use passed non-NULL, bad plan mode */
+  PA_ERR_UNSUPPORTED = 2,   /* head_dim != 128, page size not a power of two <= 256,
+                               Hq / Hkv not in {1,2,4,8}, Sage shared-memory budget exceeded,
+                               EXTEND page size < 8 */
+  PA_ERR_ARCH = 3,          /* the current device is not sm_100 (B200) */
+  PA_ERR_WORKSPACE = 4,     /* workspace too small, or a run call's mode differs from the plan's */
+  PA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_DEVICE_INDEX = 6   /* (pa_read_device_error only) a kernel met an out-of-range
+                               slot/page id or sequence length, or gave up a bounded wait */
+} pa_status;
+
+typedef enum {
+  PA_MODE_DECODE = 0,       /* bf16 split-KV decode + log-sum-exp merge */
+  PA_MODE_EXTEND = 1,       /* bf16 causal extend over a cached prefix (tcgen05 / TMEM) */
+  PA_MODE_SAGE_DECODE = 2   /* INT8 Q/K, E4M3 P and V, per-block scales, bf16 output */
+} pa_mode;
+
+/*
+ * Plan-time parameters: fixed per batch, shared by every layer's run call
+ * ("the recipe is fixed at plan time, the scales are given at every run",
+ * "FlashInfer PrimTS, Sage Attention ..." section "코드 분석" items 1 and 5).
+ */
+typedef struct {
+  int32_t mode;          /* pa_mode */
+  int32_t batch;         /* B, number of requests, 1 .. 8192 */
+  int32_t hq;            /* query heads */
+  int32_t hkv;           /* KV heads; hq % hkv == 0 and hq / hkv in {1, 2, 4, 8} */
+  int32_t head_dim;      /* D, must be 128 */
+  int32_t page_size;     /* P: power of two, 1 .. 256 (EXTEND: 8 .. 256; SAGE: == sage_k_block) */
+  int32_t max_kv_len;    /* upper bound on every seq_lens[r]; longer lengths are clamped and flagged */
+  int32_t max_q_tokens;  /* EXTEND: upper bound on sum of new tokens (sizes the grid); else 0 */
+  int32_t num_sms;       /* SMs the plan schedules for; 0 = query the current device */
+  int32_t max_splits;    /* DECODE: cap on splits per request, >= 1 (0 = 64) */
+  int32_t sage_k_block;  /* SAGE: keys per sfK block, must be 64; else 0 */
+  int32_t reserved;      /* must be 0 */
+} pa_plan_params;
+
+/*
+ * Workspace bytes needed by attn_plan and the run calls for `params`
+ * (header, per-request arrays, the work list and, for DECODE, the split
+ * partials).  Writes *bytes; returns PA_ERR_INVALID / PA_ERR_UNSUPPORTED for
+ * parameters that attn_plan would reject.  Host only, no CUDA work except a
+ * device-attribute query when num_sms == 0.
+ */
+pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
+
+/*
+ * attn_plan - build the per-batch scheduling metadata once, for reuse by every
+ * layer ["SGLang의 FA3 디코드 최적화: get_scheduler_metadata 도입", 코드 분석
+ * items 1-3 and 왜 이게 좋은가 item 1: the metadata depends only on the
+ * sequence lengths and the optional cumulative query lengths].
+ *
+ * d_seq_lens     int32 [B], device: total KV length L_r of each request (for
+ *                EXTEND, prefix plus new tokens).
+ * d_cu_seqlens_q int32 [B+1], device: EXTEND only (exclusive prefix sums of
+ *                the new-token counts); must be NULL for the other modes.
+ * d_ws           device workspace of ws_bytes >= pa_plan_workspace_size().
+ *
+ * One single-CTA kernel computes, from the lengths alone (integer arithmetic):
+ *   DECODE: T = max(64, P) keys per tile, tiles_r = ceil(L_r / T),
+ *     total = sum tiles_r * Hkv, slots = num_sms * 8,
+ *     chunk = max(1, ceil(total / slots)) tiles per split;
+ *     L_r == 0 gives one empty split; otherwise splits_r = ceil(tiles_r / chunk)
+ *     and, if that exceeds max_splits, chunk_r = ceil(tiles_r / max_splits),
+ *     splits_r = ceil(tiles_r / chunk_r); split s covers keys
+ *     [s chunk_r T, min((s+1) chunk_r T, L_r)).
+ *   EXTEND: query tiles of 128 new tokens; tile t of request r covers new
+ *     tokens [128 t, min(128 t + 128, n_r)) and reads key tiles
+ *     0 .. ceil((p_r + q_end) / 128) - 1, p_r = L_r - n_r.
+ *   SAGE_DECODE: one item per request covering [0, L_r).
+ * The items are ordered by work (key count, key-tile count or L_r) descending,
+ * ties by (request, split) order, so the in-order block dispatch of the run
+ * kernels schedules the longest work first.  At most ceil(num_sms * 8 / Hkv)
+ * + B items (DECODE), ceil(max_q_tokens / 128) + B (EXTEND) or B (SAGE).
+ *
+ * Workspace layout (for introspection; all int32, offsets in bytes):
+ *   [0, 64)   header: magic 0x4C504150, mode, batch, hq, hkv, head_dim,
+ *             page_size, num_items, max_items, tile, chunk_tiles, error word,
+ *             num_sms, max_splits, reserved x2
+ *   then      req_splits[B] (items of request r), req_base[B+1] (exclusive
+ *             prefix sum of req_splits), req_len[B] (L_r as used), req_aux[B]
+ *             (DECODE: chunk_r tiles per split; EXTEND: cu_seqlens_q[r]),
+ *             req_prefix[B] (EXTEND: p_r), padded to 16 B, then the items
+ *             int32x4 [max_items] = {r, split, begin, end} in execution order,
+ *             256-byte aligned, then (DECODE) fp32 partial outputs
+ *             [max_items][Hq][D] and partial LSEs (log2 units) [max_items][Hq],
+ *             each 256-byte aligned.  The partial of split s of request r,
+ *             head h, sits at row (req_base[r] + s) * Hq + h.
+ * Lengths < 0 or > max_kv_len are clamped to [0, max_kv_len] and set the
+ * error word.  Returns PA_ERR_ARCH off sm_100, PA_ERR_WORKSPACE if ws_bytes
+ * is short, PA_ERR_INVALID for NULL pointers or a cu_seqlens_q that does not
+ * match the mode.
+ */
+pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
+                    const int32_t* d_cu_seqlens_q, void* d_ws, size_t ws_bytes,
+                    pa_stream_t stream);
+
+/*
+ * attn_decode_paged - bf16 DECODE over the paged cache for one layer.
+ * For each request r and query head h:  s_j = sm_scale * q . K_j,
+ * O = sum_j softmax(s)_j V_j over j in [0, L_r), lse = log sum_j exp(s_j)
+ * ["FlashAttention: 优化计算过程中的临时显存占用", section 1 (the standard
+ * definition) and section 2 (tiling reaches it without the N x N matrix)].
+ * Each (request, KV head, split) CTA gathers its K/V rows with 16-byte
+ * copies through the slot table, packs the Hq / Hkv query heads of the KV head
+ * so each row is read once, and keeps a running max / sum; requests split
+ * into several ranges are combined by a log-sum-exp merge kernel.
+ *
+ * params, d_ws    the plan (mode PA_MODE_DECODE) built by attn_plan.
+ * d_q             bf16 [B][Hq][D];  d_k_pool, d_v_pool bf16 [num_slots][Hkv][D].
+ * d_page_table    int32 [B][pt_pitch] (pt_pitch >= ceil(max_kv_len / P)).
+ * d_out           bf16 [B][Hq][D];  d_lse_out fp32 [B][Hq] natural log, or NULL.
+ * All device pointers 16-byte aligned.  Empty requests give O = 0, lse = -inf.
+ */
+pa_status attn_decode_paged(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                            const uint16_t* d_q, const uint16_t* d_k_pool,
+                            const uint16_t* d_v_pool, int64_t num_slots,
+                            const int32_t* d_page_table, int64_t pt_pitch, float sm_scale,
+                            uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
+
+/*
+ * attn_extend_paged - bf16 causal EXTEND for one layer.  New token i of
+ * request r (row cu_seqlens_q[r] + i of Q) sits at absolute position p_r + i
+ * and attends to keys j <= p_r + i, whose K/V (prefix and new tokens alike)
+ * are already in the pool.  O = softmax(sm_scale Q K^T + mask) V.
+ * Query tiles of 128 rows per head; key pages arrive by TMA; QK^T and PV run on
+ * tcgen05 tensor cores with TMEM accumulators; key tiles above the diagonal
+ * are skipped.
+ *
+ * params, d_ws    the plan (mode PA_MODE_EXTEND); page_size must be >= 8.
+ * d_q, d_out      bf16 [sum n][Hq][D];  d_lse_out fp32 [sum n][Hq] or NULL.
+ * Pools and table as for attn_decode_paged; num_slots < 2^31.
+ */
+pa_status attn_extend_paged(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                            const uint16_t* d_q, const uint16_t* d_k_pool,
+                            const uint16_t* d_v_pool, int64_t num_slots,
+                            const int32_t* d_page_table, int64_t pt_pitch, float sm_scale,
+                            uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
+
+/*
+ * attn_decode_paged_sage - 8-bit Sage DECODE for one layer
+ * ["FlashInfer PrimTS, Sage Attention ...", 코드 분석 item 1, README formula]:
+ *   S_j  = sfQ[r][h] * sfK[slot_j / 64][h_kv] * (Q8 . K8_j)      (exact int dot)
+ *   m    = max_j S_j over the whole row,  p_j = exp(S_j - m),  l = sum_j p_j
+ *   P8_j = E4M3(448 p_j)                (round to nearest even, saturating)
+ *   O[d] = sfV[h_kv][d] * (sum_j P8_j V8_j[d]) / (448 l) + v_mean[h_kv][d]
+ * The scales enter before the max and the exponential and sfV is applied in
+ * the epilogue (same page, item 4).  S is formed in float32 as
+ * (sfQ * sfK) * float(dot).  There is no separate softmax scale: fold it into
+ * sfQ.  Scales must be finite and positive and are NOT checked (same page,
+ * item 1).
+ *
+ * params, d_ws    the plan (mode PA_MODE_SAGE_DECODE, sage_k_block = 64 = page_size).
+ * d_q8 int8 [B][Hq][D];  d_sf_q fp32 [B][Hq].
+ * d_k8_pool int8, d_v8_pool E4M3 bytes, both [num_slots][Hkv][D].
+ * d_sf_k fp32 [num_slots / 64][Hkv];  d_sf_v fp32 [Hkv][D];
+ * d_v_mean fp32 [Hkv][D] or NULL (then 0).   d_out bf16 [B][Hq][D].
+ * The whole row of scores is kept on chip, so G * max_kv_len * 4 bytes must fit
+ * the kernel's shared-memory budget (checked at plan time: PA_ERR_UNSUPPORTED).
+ * Empty requests give O = v_mean.
+ */
+pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                                 const int8_t* d_q8, const float* d_sf_q,
+                                 const int8_t* d_k8_pool, const uint8_t* d_v8_pool,
+                                 const float* d_sf_k, const float* d_sf_v, const float* d_v_mean,
+                                 int64_t num_slots, const int32_t* d_page_table, int64_t pt_pitch,
+                                 uint16_t* d_out, pa_stream_t stream);
+
+/*
+ * attn_debug_gather - copy, for request r and KV head h_kv, the slot ids and
+ * the K rows the kernels gather: d_slots_out int32 [L], d_rows_out bf16 [L][D]
+ * for positions 0 .. L-1, L = min(d_seq_lens[r], max_len).  Out-of-range ids
+ * are written as -1 with zero rows.  A test hook for checking the slot/page
+ * indexing bit for bit; same table convention as the run calls.
+ */
+pa_status attn_debug_gather(const int32_t* d_seq_lens, int32_t r, int32_t h_kv, int32_t hkv,
+                            int32_t head_dim, int32_t page_size, int32_t max_len,
+                            const uint16_t* d_k_pool, int64_t num_slots,
+                            const int32_t* d_page_table, int64_t pt_pitch,
+                            int32_t* d_slots_out, uint16_t* d_rows_out, pa_stream_t stream);
+
+/*
+ * pa_read_device_error - synchronise `stream`, read the workspace's device
+ * error word and clear it.  PA_OK if clean, PA_ERR_DEVICE_INDEX if a kernel
+ * recorded an out-of-range id or length, PA_ERR_WORKSPACE if a run kernel
+ * found a workspace built for another mode, PA_ERR_CUDA on a CUDA error.
+ */
+pa_status pa_read_device_error(void* d_ws, pa_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* pa_status_string(pa_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,153 @@
+// common.cuh - workspace layout and small device helpers shared by the kernels.
+//
+// The PTX wrappers below are thin spellings of documented sm_80+/sm_100a
+// instructions (cp.async, ldmatrix, mma.sync, movmatrix, ex2.approx) so that
+// the kernels read as the algorithm.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+constexpr int32_t kMagic = 0x4C504150;          // "PAPL"
+constexpr int kHeadDim = 128;
+constexpr int kDecodeMinTile = 64;               // keys per decode tile (and split granularity floor)
+constexpr int kDecodeCtasPerSm = 8;              // decode CTAs a plan aims for, per SM
+constexpr int kExtendQTile = 128;
+constexpr int kExtendKvTile = 128;
+constexpr int kSageBlock = 64;
+constexpr int kMaxBatch = 8192;
+constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capacity
+
+// 64-byte header at the start of the workspace (layout documented in pagedattn.h).
+struct PlanHeader {
+  int32_t magic, mode, batch, hq, hkv, head_dim, page_size, num_items;
+  int32_t max_items, tile, chunk_tiles, error_word;
+  int32_t num_sms, max_splits, reserved0, reserved1;
+};
+static_assert(sizeof(PlanHeader) == 64, "header is 64 bytes");
+
+// Byte offsets of the workspace arrays.
+struct WsLayout {
+  size_t req_splits, req_base, req_len, req_aux, req_prefix, items, partial_o, partial_lse, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int mode, int batch, int hq, int head_dim, int max_items) {
+  WsLayout w{};
+  size_t off = sizeof(PlanHeader);
+  w.req_splits = off; off += 4 * (size_t)batch;
+  w.req_base = off;   off += 4 * (size_t)(batch + 1);
+  w.req_len = off;    off += 4 * (size_t)batch;
+  w.req_aux = off;    off += 4 * (size_t)batch;
+  w.req_prefix = off; off += 4 * (size_t)batch;
+  off = align_up(off, 16);
+  w.items = off;      off += 16 * (size_t)max_items;
+  off = align_up(off, 256);
+  if (mode == PA_MODE_DECODE) {
+    w.partial_o = off;   off += 4 * (size_t)max_items * hq * head_dim;
+    off = align_up(off, 256);
+    w.partial_lse = off; off += 4 * (size_t)max_items * hq;
+    off = align_up(off, 256);
+  }
+  w.total = off;
+  return w;
+}
+
+// Plain-data view of the workspace that kernels receive by value.
+struct WsView {
+  PlanHeader* hdr;
+  int32_t* req_splits;
+  int32_t* req_base;
+  int32_t* req_len;
+  int32_t* req_aux;
+  int32_t* req_prefix;
+  int4* items;
+  float* partial_o;
+  float* partial_lse;
+};
+
+inline WsView ws_view(void* ws, const WsLayout& w) {
+  char* b = static_cast<char*>(ws);
+  WsView v;
+  v.hdr = reinterpret_cast<PlanHeader*>(b);
+  v.req_splits = reinterpret_cast<int32_t*>(b + w.req_splits);
+  v.req_base = reinterpret_cast<int32_t*>(b + w.req_base);
+  v.req_len = reinterpret_cast<int32_t*>(b + w.req_len);
+  v.req_aux = reinterpret_cast<int32_t*>(b + w.req_aux);
+  v.req_prefix = reinterpret_cast<int32_t*>(b + w.req_prefix);
+  v.items = reinterpret_cast<int4*>(b + w.items);
+  v.partial_o = w.partial_o ? reinterpret_cast<float*>(b + w.partial_o) : nullptr;
+  v.partial_lse = w.partial_lse ? reinterpret_cast<float*>(b + w.partial_lse) : nullptr;
+  return v;
+}
+
+// Records the first device-side error in the header (later ones are dropped).
+__device__ __forceinline__ void set_device_error(PlanHeader* hdr, int code) {
+  atomicCAS(&hdr->error_word, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global->shared copy; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per thread.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// 2^x (hardware approximation; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two floats to a packed bf16 pair, round to nearest even; `lo` lands in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+}  // namespace pa

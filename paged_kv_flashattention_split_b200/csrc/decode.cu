@@ -1,0 +1,337 @@
+// decode.cu - bf16 split-KV decode over the paged cache, and the log-sum-exp merge.
+//
+// One CTA per (request, KV head, split) work item of the plan.  The CTA's four
+// warps share a 3-stage cp.async ring of 64-key tiles: each thread gathers one
+// key's half row of K and of V (8 x 16 B each) through the slot table into an
+// XOR-swizzled shared-memory tile.  Each warp then takes 16 keys of the tile
+// and computes, on the tensor cores,
+//     S^T[16 keys x 8 heads] = K[16 x 128] . Q^T      (mma.m16n8k16, keys as M)
+// for the Hq / Hkv <= 8 query heads that read this KV head, so every K/V row
+// is fetched from HBM once for all of them.  The online softmax keeps a
+// running max and sum per head (warp shuffles over the 8 key rows), the
+// probabilities are rounded to bf16, transposed in registers with movmatrix
+// and used as the B operand of
+//     O^T[128 d x 8 heads] += V^T[128 x 16 keys] . P^T
+// At the end the four warps' partial states are combined through shared
+// memory.  A request covered by one split writes its bf16 output directly;
+// otherwise each split writes (O_s, lse_s) and merge_kernel computes
+//     lse = log2 sum_s 2^lse_s,  O = sum_s 2^(lse_s - lse) O_s.
+//
+// This is the tiled online-softmax evaluation of softmax(scale q K^T) V that
+// "FlashAttention: 优化计算过程中的临时显存占用" (sections 1-2) describes:
+// no score matrix ever reaches HBM, and the result equals the standard one.
+#include "kernels.h"
+
+namespace pa {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTileKeys = 64;
+constexpr int kStages = 3;
+constexpr int kRowBytes = kHeadDim * 2;                    // 256 B per (slot, head) row
+constexpr int kHalfStage = kTileKeys * kRowBytes;          // 16 KB of K (or V) per tile
+constexpr int kStageBytes = 2 * kHalfStage;
+constexpr int kDecodeSmem = kStages * kStageBytes;         // 96 KB: two CTAs per SM
+constexpr float kLn2 = 0.693147180559945309f;
+
+__device__ __forceinline__ bool workspace_ok(const PlanHeader* hdr, int mode) {
+  return hdr->magic == kMagic && hdr->mode == mode;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunch a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  PlanHeader* hdr = a.ws.hdr;
+  if (!workspace_ok(hdr, PA_MODE_DECODE)) {
+    if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
+    return;
+  }
+  const int num_items = hdr->num_items;
+  const int w = blockIdx.x;
+  if (w >= num_items * a.hkv) return;
+  const int4 it = a.ws.items[w / a.hkv];
+  const int h_kv = w % a.hkv;
+  const int r = it.x, split = it.y, kv0 = it.z, kv1 = it.w;
+  const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+
+  // Q^T as the B operand: b0 = Q[head gid][16kk + 2tig .. +1], b1 = the same at +8.
+  uint32_t qb0[8], qb1[8];
+  {
+    const uint32_t* qrow =
+        reinterpret_cast<const uint32_t*>(a.q + ((size_t)r * a.hq + (size_t)h_kv * G + gid) * kHeadDim);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qb0[kk] = gid < G ? __ldg(qrow + 8 * kk + tig) : 0u;
+      qb1[kk] = gid < G ? __ldg(qrow + 8 * kk + 4 + tig) : 0u;
+    }
+  }
+
+  // Gather assignment: thread -> (key ld_key of the tile, half row ld_half).
+  const int ld_key = tid >> 1, ld_half = tid & 1;
+  const int page_shift = a.page_shift;
+  const int page_mask = (1 << page_shift) - 1;
+  const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
+  const size_t head_off = (size_t)h_kv * kHeadDim;
+  const size_t slot_stride = (size_t)a.hkv * kHeadDim;
+
+  auto slot_of = [&](int j) -> long long {
+    if (j >= kv1) return -1;
+    const int page = __ldg(table + (j >> page_shift));
+    const long long slot = ((long long)page << page_shift) + (j & page_mask);
+    if (page < 0 || slot >= a.num_slots) {
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      return -1;
+    }
+    return slot;
+  };
+  const uint32_t smem_base = smem_u32(smem);
+  auto issue = [&](int tile, long long slot) {
+    const uint32_t kdst = smem_base + (tile % kStages) * kStageBytes + ld_key * kRowBytes;
+    const uint32_t vdst = kdst + kHalfStage;
+    const size_t row = slot >= 0 ? (size_t)slot * slot_stride + head_off : 0;
+    const uint16_t* ks = a.k_pool + row;
+    const uint16_t* vs = a.v_pool + row;
+    const int bytes = slot >= 0 ? 16 : 0;  // rows past the split (or bad ids) are zero-filled
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int chunk = ld_half * 8 + c;
+      const uint32_t off = (uint32_t)((chunk ^ (ld_key & 7)) << 4);
+      cp_async_16(kdst + off, ks + chunk * 8, bytes);
+      cp_async_16(vdst + off, vs + chunk * 8, bytes);
+    }
+  };
+
+  long long next_slot = slot_of(kv0 + ld_key);
+#pragma unroll
+  for (int t = 0; t < kStages - 1; ++t) {
+    if (t < n_tiles) issue(t, next_slot);
+    cp_async_commit();
+    next_slot = slot_of(kv0 + (t + 1) * kTileKeys + ld_key);
+  }
+
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  float m_run0 = NEG_INF, m_run1 = NEG_INF, l_run0 = 0.f, l_run1 = 0.f;
+  float o[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+  // ldmatrix row/chunk roles of this lane (see the fragment layouts of mma.m16n8k16)
+  const int mat = lane >> 3;
+  const int k_row = warp * 16 + (lane & 7) + ((mat & 1) << 3);   // K: A rows, chunk + (mat >> 1)
+  const int v_row = warp * 16 + (lane & 7) + ((mat >> 1) << 3);  // V: A^T rows, chunk + (mat & 1)
+
+  for (int t = 0; t < n_tiles; ++t) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    {
+      const int tp = t + kStages - 1;
+      if (tp < n_tiles) issue(tp, next_slot);
+      cp_async_commit();
+      next_slot = slot_of(kv0 + (tp + 1) * kTileKeys + ld_key);
+    }
+    const uint32_t kst = smem_base + (t % kStages) * kStageBytes;
+    const uint32_t vst = kst + kHalfStage;
+
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t af[4];
+      const int chunk = 2 * kk + (mat >> 1);
+      ldmatrix_x4(af, kst + k_row * kRowBytes + ((chunk ^ (k_row & 7)) << 4));
+      mma_bf16_16816(s, af, qb0[kk], qb1[kk]);
+    }
+    const int key0 = kv0 + t * kTileKeys + warp * 16 + gid;
+    const int key1 = key0 + 8;
+    const float x00 = key0 < kv1 ? s[0] * a.scale_log2 : NEG_INF;
+    const float x01 = key0 < kv1 ? s[1] * a.scale_log2 : NEG_INF;
+    const float x10 = key1 < kv1 ? s[2] * a.scale_log2 : NEG_INF;
+    const float x11 = key1 < kv1 ? s[3] * a.scale_log2 : NEG_INF;
+    float mx0 = fmaxf(x00, x10), mx1 = fmaxf(x01, x11);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
+    const float mu0 = mn0 == NEG_INF ? 0.f : mn0;
+    const float mu1 = mn1 == NEG_INF ? 0.f : mn1;
+    const float al0 = ex2(m_run0 - mu0), al1 = ex2(m_run1 - mu1);
+    m_run0 = mn0;
+    m_run1 = mn1;
+    const uint32_t pk0 = pack_bf16x2(ex2(x00 - mu0), ex2(x01 - mu1));
+    const uint32_t pk1 = pack_bf16x2(ex2(x10 - mu0), ex2(x11 - mu1));
+    // the row sum uses the same bf16-rounded probabilities as the PV product
+    l_run0 = l_run0 * al0 + bf16lo_to_f32(pk0) + bf16lo_to_f32(pk1);
+    l_run1 = l_run1 * al1 + bf16hi_to_f32(pk0) + bf16hi_to_f32(pk1);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      o[mt][0] *= al0;
+      o[mt][1] *= al1;
+      o[mt][2] *= al0;
+      o[mt][3] *= al1;
+    }
+    const uint32_t pb0 = movmatrix_trans(pk0);  // P^T[key 2tig..+1][head gid], keys 0-7
+    const uint32_t pb1 = movmatrix_trans(pk1);  // keys 8-15
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t af[4];
+      const int chunk = 2 * mt + (mat & 1);
+      ldmatrix_x4_trans(af, vst + v_row * kRowBytes + ((chunk ^ (v_row & 7)) << 4));
+      mma_bf16_16816(o[mt], af, pb0, pb1);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // Combine the four warps' (m, l, O) through shared memory.
+  float* red_o = reinterpret_cast<float*>(smem);   // [4 warps][8 heads][128 d]
+  float* red_m = red_o + 4 * 8 * kHeadDim;         // [4][8]
+  float* red_l = red_m + 32;                       // [4][8]
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l_run0 += __shfl_xor_sync(0xffffffffu, l_run0, off);
+    l_run1 += __shfl_xor_sync(0xffffffffu, l_run1, off);
+  }
+  if (gid == 0) {
+    red_m[warp * 8 + 2 * tig] = m_run0;
+    red_m[warp * 8 + 2 * tig + 1] = m_run1;
+    red_l[warp * 8 + 2 * tig] = l_run0;
+    red_l[warp * 8 + 2 * tig + 1] = l_run1;
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int d = 16 * mt + gid;
+    float* h0 = red_o + (warp * 8 + 2 * tig) * kHeadDim;
+    float* h1 = h0 + kHeadDim;
+    h0[d] = o[mt][0];
+    h1[d] = o[mt][1];
+    h0[d + 8] = o[mt][2];
+    h1[d + 8] = o[mt][3];
+  }
+  __syncthreads();
+
+  const int splits = a.ws.req_splits[r];
+  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
+    const int h = idx / kHeadDim, d = idx % kHeadDim;
+    float M = NEG_INF;
+#pragma unroll
+    for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, red_m[ww * 8 + h]);
+    float O = 0.f, lse2 = NEG_INF;
+    if (M != NEG_INF) {
+      float wsum = 0.f, acc = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < 4; ++ww) {
+        const float f = ex2(red_m[ww * 8 + h] - M);
+        wsum += red_l[ww * 8 + h] * f;
+        acc += red_o[(ww * 8 + h) * kHeadDim + d] * f;
+      }
+      O = acc / wsum;
+      lse2 = M + __log2f(wsum);
+    }
+    const int hq_idx = h_kv * G + h;
+    if (splits == 1) {
+      a.out[((size_t)r * a.hq + hq_idx) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(O));
+      if (d == 0 && a.lse_out) a.lse_out[(size_t)r * a.hq + hq_idx] = lse2 * kLn2;
+    } else {
+      const size_t p = (size_t)(a.ws.req_base[r] + split) * a.hq + hq_idx;
+      a.ws.partial_o[p * kHeadDim + d] = O;
+      if (d == 0) a.ws.partial_lse[p] = lse2;
+    }
+  }
+}
+
+// One warp per (request, query head) whose request was split: combine the
+// split partials, lse = log2 sum_s 2^lse_s, O = sum_s 2^(lse_s - lse) O_s.
+__global__ void __launch_bounds__(128) merge_kernel(DecodeLaunch a) {
+  PlanHeader* hdr = a.ws.hdr;
+  if (!workspace_ok(hdr, PA_MODE_DECODE)) return;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (gw >= a.batch * a.hq) return;
+  const int r = gw / a.hq, h = gw % a.hq;
+  const int splits = a.ws.req_splits[r];
+  if (splits <= 1) return;
+  const int base = a.ws.req_base[r];
+  if (base + splits > a.max_items) return;  // only after a plan overflow, which the plan flags
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  float M = NEG_INF;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, a.ws.partial_lse[(size_t)(base + s) * a.hq + h]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (M != NEG_INF) {
+    for (int s = 0; s < splits; ++s) {
+      const size_t p = (size_t)(base + s) * a.hq + h;
+      const float f = ex2(a.ws.partial_lse[p] - M);
+      const float4 v = reinterpret_cast<const float4*>(a.ws.partial_o + p * kHeadDim)[lane];
+      wsum += f;
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+      acc.z += f * v.z;
+      acc.w += f * v.w;
+    }
+    const float inv = 1.f / wsum;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+  }
+  uint2 packed;
+  packed.x = pack_bf16x2(acc.x, acc.y);
+  packed.y = pack_bf16x2(acc.z, acc.w);
+  reinterpret_cast<uint2*>(a.out + ((size_t)r * a.hq + h) * kHeadDim)[lane] = packed;
+  if (lane == 0 && a.lse_out)
+    a.lse_out[(size_t)r * a.hq + h] = M == NEG_INF ? NEG_INF : (M + __log2f(wsum)) * kLn2;
+}
+
+__global__ void debug_gather_kernel(GatherLaunch a) {
+  const int L = min(a.seq_lens[a.r], a.max_len);
+  const int P = 1 << a.page_shift;
+  const int32_t* table = a.page_table + (size_t)a.r * a.pt_pitch;
+  for (int j = blockIdx.x; j < L; j += gridDim.x) {
+    const int page = table[j >> a.page_shift];
+    long long slot = (long long)page * P + (j & (P - 1));
+    const bool ok = page >= 0 && slot < a.num_slots;
+    if (threadIdx.x == 0) a.slots_out[j] = ok ? (int32_t)slot : -1;
+    const uint16_t* src = a.k_pool + ((size_t)(ok ? slot : 0) * a.hkv + a.h_kv) * kHeadDim;
+    for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x)
+      a.rows_out[(size_t)j * kHeadDim + d] = ok ? src[d] : (uint16_t)0;
+  }
+}
+
+template <int G>
+cudaError_t launch_decode_g(const DecodeLaunch& a, cudaStream_t s) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kDecodeSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  decode_splitkv_kernel<G><<<a.max_items * a.hkv, kThreads, kDecodeSmem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  merge_kernel<<<(a.batch * a.hq + 3) / 4, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s) {
+  switch (a.hq / a.hkv) {
+    case 1: return launch_decode_g<1>(a, s);
+    case 2: return launch_decode_g<2>(a, s);
+    case 4: return launch_decode_g<4>(a, s);
+    case 8: return launch_decode_g<8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_debug_gather(const GatherLaunch& a, cudaStream_t s) {
+  debug_gather_kernel<<<256, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,250 @@
+// plan.cu - the per-batch scheduling plan (one CTA, integer arithmetic only).
+//
+// The scheduling metadata is a function of the sequence lengths (and, for a
+// prefill, the cumulative query lengths) alone, so it is built once per batch
+// and reused by every layer ("SGLang의 FA3 디코드 최적화: get_scheduler_metadata
+// 도입", 코드 분석 items 1-3, 왜 이게 좋은가 item 1).  The algorithm is the one
+// stated at attn_plan in pagedattn.h; every step is integer so the result is
+// exact and identical on recomputation.
+#include "kernels.h"
+
+namespace pa {
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ long long cdiv_ll(long long a, long long b) { return (a + b - 1) / b; }
+
+// Block-wide sum of one int64 per thread.
+__device__ long long block_sum(long long v, long long* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long t = 0;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  t = red[0];
+  __syncthreads();
+  return t;
+}
+
+// Block-wide exclusive scan of one int per thread; returns this thread's prefix.
+__device__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  const int tid = threadIdx.x;
+  scratch[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < blockDim.x; off <<= 1) {
+    int add = tid >= off ? scratch[tid - off] : 0;
+    __syncthreads();
+    scratch[tid] += add;
+    __syncthreads();
+  }
+  int incl = scratch[tid];
+  *total = scratch[blockDim.x - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+// Work of item (r, s) for the sort key; items run longest first.
+__device__ __forceinline__ int item_work(int mode, int s, int L, int chunk_r, int tile, int prefix, int n) {
+  if (mode == PA_MODE_DECODE) {
+    if (chunk_r == 0) return 0;
+    const long long a = (long long)s * chunk_r * tile;
+    const long long b = min((long long)(s + 1) * chunk_r * tile, (long long)L);
+    return (int)(b - a);
+  }
+  if (mode == PA_MODE_EXTEND) {
+    const int q1 = min((s + 1) * kExtendQTile, n);
+    return (int)cdiv_ll(prefix + q1, kExtendKvTile);
+  }
+  return L;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
+  extern __shared__ unsigned long long keys[];
+  __shared__ long long red[32];
+  __shared__ int scan[kPlanThreads];
+  const int tid = threadIdx.x, nt = blockDim.x;
+  WsView ws = a.ws;
+  PlanHeader* hdr = ws.hdr;
+  const int B = a.batch;
+  if (tid == 0) hdr->error_word = 0;  // every new plan starts with a clean error word
+  __syncthreads();
+
+  // 1. lengths (clamped and flagged when out of range), tiles per request
+  long long my_tiles = 0;
+  for (int r = tid; r < B; r += nt) {
+    int L = a.seq_lens[r];
+    if (L < 0 || L > a.max_kv_len) {
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      L = max(0, min(L, a.max_kv_len));
+    }
+    ws.req_len[r] = L;
+    if (a.mode == PA_MODE_DECODE) my_tiles += cdiv_ll(L, a.tile);
+  }
+  const long long total = block_sum(my_tiles, red) * a.hkv;
+  int chunk = 0;
+  if (a.mode == PA_MODE_DECODE) {
+    const long long slots = (long long)a.num_sms * kDecodeCtasPerSm;
+    chunk = (int)max(1LL, cdiv_ll(total, slots));
+  }
+
+  // 2. splits (DECODE), query tiles (EXTEND) or one item (SAGE) per request
+  for (int r = tid; r < B; r += nt) {
+    const int L = ws.req_len[r];
+    int splits = 1, aux = 0, prefix = 0;
+    if (a.mode == PA_MODE_DECODE) {
+      const int tiles = (int)cdiv_ll(L, a.tile);
+      if (tiles == 0) {
+        splits = 1;
+        aux = 0;
+      } else {
+        int chunk_r = chunk;
+        int s = (int)cdiv_ll(tiles, chunk_r);
+        if (s > a.max_splits) {
+          chunk_r = (int)cdiv_ll(tiles, a.max_splits);
+          s = (int)cdiv_ll(tiles, chunk_r);
+        }
+        splits = s;
+        aux = chunk_r;
+      }
+    } else if (a.mode == PA_MODE_EXTEND) {
+      const int q0 = a.cu_seqlens_q[r], q1 = a.cu_seqlens_q[r + 1];
+      int n = q1 - q0;
+      if (n < 0 || n > L) {
+        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+        n = max(0, min(n, L));
+      }
+      splits = (int)cdiv_ll(n, kExtendQTile);
+      aux = q0;
+      prefix = L - n;
+    }
+    ws.req_splits[r] = splits;
+    ws.req_aux[r] = aux;
+    ws.req_prefix[r] = prefix;
+  }
+  __syncthreads();
+
+  // 3. req_base = exclusive prefix sum of the per-request item counts
+  const int per = (B + nt - 1) / nt;
+  const int r0 = min(B, tid * per), r1 = min(B, r0 + per);
+  int local = 0;
+  for (int r = r0; r < r1; ++r) local += ws.req_splits[r];
+  int total_items = 0;
+  int run = block_exclusive_scan(local, scan, &total_items);
+  for (int r = r0; r < r1; ++r) {
+    ws.req_base[r] = run;
+    run += ws.req_splits[r];
+  }
+  if (tid == 0) ws.req_base[B] = total_items;
+  int n_items = total_items;
+  if (n_items > a.max_items) {  // cannot happen for lengths within bounds; keep the grid safe
+    if (tid == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    n_items = a.max_items;
+  }
+  for (int i = tid; i < a.sort_n; i += nt) keys[i] = ~0ull;
+  __syncthreads();
+
+  // 4. sort keys: (0x7FFFFFFF - work) in the high word, generation index in the low word
+  for (int r = tid; r < B; r += nt) {
+    const int base = ws.req_base[r], splits = ws.req_splits[r];
+    const int L = ws.req_len[r], aux = ws.req_aux[r], prefix = ws.req_prefix[r];
+    const int n = L - prefix;
+    for (int s = 0; s < splits; ++s) {
+      const int g = base + s;
+      if (g >= n_items) break;
+      const unsigned work = (unsigned)item_work(a.mode, s, L, aux, a.tile, prefix, n);
+      keys[g] = ((unsigned long long)(0x7FFFFFFFu - work) << 32) | (unsigned)g;
+    }
+  }
+  __syncthreads();
+
+  // 5. bitonic sort, ascending (unique keys, so the order is fully determined)
+  for (int k = 2; k <= a.sort_n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < a.sort_n; i += nt) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          const bool up = (i & k) == 0;
+          if ((x > y) == up) {
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // 6. items in execution order
+  for (int i = tid; i < n_items; i += nt) {
+    const int g = (int)(keys[i] & 0xFFFFFFFFu);
+    int lo = 0, hi = B;  // find r with req_base[r] <= g < req_base[r+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ws.req_base[mid] <= g) lo = mid; else hi = mid;
+    }
+    const int r = lo, s = g - ws.req_base[r];
+    const int L = ws.req_len[r], aux = ws.req_aux[r], prefix = ws.req_prefix[r];
+    int4 it;
+    it.x = r;
+    it.y = s;
+    if (a.mode == PA_MODE_DECODE) {
+      const long long b0 = (long long)s * aux * a.tile;
+      it.z = (int)min(b0, (long long)L);
+      it.w = (int)min((long long)(s + 1) * aux * a.tile, (long long)L);
+    } else if (a.mode == PA_MODE_EXTEND) {
+      const int n = L - prefix;
+      it.z = s * kExtendQTile;
+      it.w = min((s + 1) * kExtendQTile, n);
+    } else {
+      it.z = 0;
+      it.w = L;
+    }
+    ws.items[i] = it;
+  }
+
+  // 7. header
+  if (tid == 0) {
+    hdr->magic = kMagic;
+    hdr->mode = a.mode;
+    hdr->batch = B;
+    hdr->hq = a.hq;
+    hdr->hkv = a.hkv;
+    hdr->head_dim = a.head_dim;
+    hdr->page_size = a.page_size;
+    hdr->num_items = n_items;
+    hdr->max_items = a.max_items;
+    hdr->tile = a.tile;
+    hdr->chunk_tiles = chunk;
+    hdr->num_sms = a.num_sms;
+    hdr->max_splits = a.max_splits;
+    hdr->reserved0 = 0;
+    hdr->reserved1 = 0;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s) {
+  const size_t smem = sizeof(unsigned long long) * (size_t)a.sort_n;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(unsigned long long) * kMaxSortItems));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  plan_kernel<<<1, kPlanThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pa
