@@ -91,7 +91,7 @@ typedef struct {
   int32_t max_kv_len;    /* upper bound on every seq_lens[r]; longer lengths are clamped and flagged */
   int32_t max_q_tokens;  /* EXTEND: upper bound on sum of new tokens (sizes the grid); else 0 */
   int32_t num_sms;       /* SMs the plan schedules for; 0 = query the current device */
-  int32_t max_splits;    /* DECODE: cap on splits per request, >= 1 (0 = 64) */
+  int32_t max_splits;    /* DECODE: cap on splits per request, >= 1 (0 = 128) */
   int32_t sage_k_block;  /* SAGE: keys per sfK block, must be 64; else 0 */
   int32_t reserved;      /* must be 0 */
 } pa_plan_params;
@@ -118,9 +118,10 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  * d_ws           device workspace of ws_bytes >= pa_plan_workspace_size().
  *
  * One single-CTA kernel computes, from the lengths alone (integer arithmetic):
- *   DECODE: T = max(64, P) keys per tile, tiles_r = ceil(L_r / T),
- *     total = sum tiles_r * Hkv, slots = num_sms * 8,
- *     chunk = max(1, ceil(total / slots)) tiles per split;
+ *   DECODE: T = max(64, P) keys per tile, tiles_r = ceil(L_r / T); one CTA
+ *     covers HG = the largest of 8, 4, 2, 1 dividing Hkv KV heads, so an item
+ *     takes groups = Hkv / HG CTAs; total = sum tiles_r * groups,
+ *     slots = num_sms * 4, chunk = max(1, ceil(total / slots)) tiles per split;
  *     L_r == 0 gives one empty split; otherwise splits_r = ceil(tiles_r / chunk)
  *     and, if that exceeds max_splits, chunk_r = ceil(tiles_r / max_splits),
  *     splits_r = ceil(tiles_r / chunk_r); split s covers keys
@@ -131,7 +132,7 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  *   SAGE_DECODE: one item per request covering [0, L_r).
  * The items are ordered by work (key count, key-tile count or L_r) descending,
  * ties by (request, split) order, so the in-order block dispatch of the run
- * kernels schedules the longest work first.  At most ceil(num_sms * 8 / Hkv)
+ * kernels schedules the longest work first.  At most ceil(num_sms * 4 / groups)
  * + B items (DECODE), ceil(max_q_tokens / 128) + B (EXTEND) or B (SAGE).
  *
  * Workspace layout (for introspection; all int32, offsets in bytes):

@@ -11,9 +11,11 @@ must reproduce it bit for bit.
 
 DECODE (split-KV work list)
   T        = max(64, page_size)                  keys per tile
+  HG       = the largest of 8, 4, 2, 1 dividing Hkv   (KV heads one CTA covers)
+  groups   = Hkv / HG                            CTAs per work item
   tiles_r  = ceil(L_r / T)
-  total    = sum_r tiles_r * Hkv                 tile-head units of work
-  slots    = num_sms * 8                         CTAs one decode launch aims for
+  total    = sum_r tiles_r * groups              units of work
+  slots    = num_sms * 4                         CTAs one decode launch aims for
   chunk    = max(1, ceil(total / slots))         tiles per split
   L_r == 0 : one split, the empty range [0, 0)
   else     : splits_r = ceil(tiles_r / chunk), chunk_r = chunk;
@@ -25,7 +27,7 @@ DECODE (split-KV work list)
   hardware's in-order block dispatch is a longest-processing-time schedule).
   req_base = exclusive prefix sum of splits_r (the merge's index of split 0).
   Bound used to size the grid and the workspace:
-  num_items <= ceil(slots / Hkv) + B.
+  num_items <= ceil(slots / groups) + B.
 
 EXTEND (query-tile work list)
   n_r = cu[r+1] - cu[r], p_r = L_r - n_r, query tiles of 128 rows:
@@ -41,7 +43,7 @@ from __future__ import annotations
 
 MODE_DECODE, MODE_EXTEND, MODE_SAGE_DECODE = 0, 1, 2
 DECODE_MIN_TILE = 64
-DECODE_CTAS_PER_SM = 8
+DECODE_CTAS_PER_SM = 4
 EXTEND_Q_TILE = 128
 EXTEND_KV_TILE = 128
 
@@ -54,10 +56,18 @@ def decode_tile(page_size: int) -> int:
     return max(DECODE_MIN_TILE, page_size)
 
 
+def decode_head_groups(hkv: int) -> int:
+    """Number of CTAs per decode work item: Hkv / (largest of 8, 4, 2, 1 dividing Hkv)."""
+    for hg in (8, 4, 2, 1):
+        if hkv % hg == 0:
+            return hkv // hg
+    raise ValueError("hkv must be positive")
+
+
 def max_items(mode: int, batch: int, hkv: int, num_sms: int, max_q_tokens: int = 0) -> int:
     """The host-side bound on the number of work items for a plan of this shape."""
     if mode == MODE_DECODE:
-        return _cdiv(num_sms * DECODE_CTAS_PER_SM, hkv) + batch
+        return _cdiv(num_sms * DECODE_CTAS_PER_SM, decode_head_groups(hkv)) + batch
     if mode == MODE_EXTEND:
         return _cdiv(max_q_tokens, EXTEND_Q_TILE) + batch
     return batch
@@ -82,7 +92,7 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
     if mode == MODE_DECODE:
         tile = decode_tile(page_size)
         tiles = [_cdiv(x, tile) for x in L]
-        total = sum(tiles) * hkv
+        total = sum(tiles) * decode_head_groups(hkv)
         slots = num_sms * DECODE_CTAS_PER_SM
         chunk = max(1, _cdiv(total, slots))
         for r in range(B):

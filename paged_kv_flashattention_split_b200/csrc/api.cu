@@ -72,7 +72,7 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
   switch (p->mode) {
     case PA_MODE_DECODE:
       if (p->max_q_tokens != 0 || p->sage_k_block != 0) return PA_ERR_INVALID;
-      d->max_splits = p->max_splits == 0 ? 64 : p->max_splits;
+      d->max_splits = p->max_splits == 0 ? 128 : p->max_splits;
       if (d->max_splits > 4096) return PA_ERR_INVALID;
       d->tile = P > kDecodeMinTile ? P : kDecodeMinTile;
       break;
@@ -98,7 +98,10 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
   d->num_sms = sms;
   long long mi = 0;
   if (p->mode == PA_MODE_DECODE)
-    mi = ((long long)sms * kDecodeCtasPerSm + p->hkv - 1) / p->hkv + p->batch;
+  {
+    const int groups = p->hkv / decode_heads_per_cta(p->hkv);
+    mi = ((long long)sms * kDecodeCtasPerSm + groups - 1) / groups + p->batch;
+  }
   else if (p->mode == PA_MODE_EXTEND)
     mi = ((long long)p->max_q_tokens + kExtendQTile - 1) / kExtendQTile + p->batch;
   else

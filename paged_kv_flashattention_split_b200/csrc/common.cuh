@@ -16,7 +16,7 @@ namespace pa {
 constexpr int32_t kMagic = 0x4C504150;          // "PAPL"
 constexpr int kHeadDim = 128;
 constexpr int kDecodeMinTile = 64;               // keys per decode tile (and split granularity floor)
-constexpr int kDecodeCtasPerSm = 8;              // decode CTAs a plan aims for, per SM
+constexpr int kDecodeCtasPerSm = 4;              // decode CTAs a plan aims for, per SM
 constexpr int kExtendQTile = 128;
 constexpr int kExtendKvTile = 128;
 constexpr int kSageBlock = 64;
@@ -37,6 +37,11 @@ struct WsLayout {
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// KV heads one decode CTA covers: the largest of 8, 4, 2, 1 that divides Hkv.
+__host__ __device__ inline int decode_heads_per_cta(int hkv) {
+  return hkv % 8 == 0 ? 8 : hkv % 4 == 0 ? 4 : hkv % 2 == 0 ? 2 : 1;
+}
 
 inline WsLayout ws_layout(int mode, int batch, int hq, int head_dim, int max_items) {
   WsLayout w{};

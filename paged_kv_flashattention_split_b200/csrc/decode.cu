@@ -1,20 +1,24 @@
 // decode.cu - bf16 split-KV decode over the paged cache, and the log-sum-exp merge.
 //
-// One CTA per (request, KV head, split) work item of the plan.  The CTA's four
-// warps share a 3-stage cp.async ring of 64-key tiles: each thread gathers one
-// key's half row of K and of V (8 x 16 B each) through the slot table into an
-// XOR-swizzled shared-memory tile.  Each warp then takes 16 keys of the tile
-// and computes, on the tensor cores,
+// One CTA per (work item, group of HG KV heads), HG = the largest of 8, 4, 2, 1
+// dividing Hkv, so a CTA gathers each token slot's K and V rows of all its
+// heads as one contiguous HG * 256-byte run (2 KB at Hkv = 8): a warp's
+// 16-byte cp.async copies cover 512 consecutive bytes, and the slots'
+// rows are fetched from HBM once for all query heads that read them.  Tiles
+// of TK = 16 * 8 / HG keys flow through a 3-stage, XOR-swizzled shared-memory
+// ring (64 KB per stage); the slot ids of a tile are read from the table one
+// tile ahead, by TK threads, with the load's latency hidden behind a tile of
+// compute.  Warp (hw, kb) takes KV head hw of the group and keys
+// [16 kb, 16 kb + 16) of every tile and computes, on the tensor cores,
 //     S^T[16 keys x 8 heads] = K[16 x 128] . Q^T      (mma.m16n8k16, keys as M)
-// for the Hq / Hkv <= 8 query heads that read this KV head, so every K/V row
-// is fetched from HBM once for all of them.  The online softmax keeps a
-// running max and sum per head (warp shuffles over the 8 key rows), the
-// probabilities are rounded to bf16, transposed in registers with movmatrix
-// and used as the B operand of
+// for the G = Hq / Hkv <= 8 query heads that read this KV head.  The online
+// softmax keeps a running max and sum per head (warp shuffles over the 8 key
+// rows); the probabilities are rounded to bf16, transposed in registers with
+// movmatrix and used as the B operand of
 //     O^T[128 d x 8 heads] += V^T[128 x 16 keys] . P^T
-// At the end the four warps' partial states are combined through shared
-// memory.  A request covered by one split writes its bf16 output directly;
-// otherwise each split writes (O_s, lse_s) and merge_kernel computes
+// The warps of a head are combined through shared memory at the end.  A
+// request covered by one split writes its bf16 output directly; otherwise
+// each split writes (O_s, lse_s) and merge_kernel computes
 //     lse = log2 sum_s 2^lse_s,  O = sum_s 2^(lse_s - lse) O_s.
 //
 // This is the tiled online-softmax evaluation of softmax(scale q K^T) V that
@@ -25,22 +29,30 @@
 namespace pa {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kTileKeys = 64;
+constexpr int kThreads = 256;
 constexpr int kStages = 3;
-constexpr int kRowBytes = kHeadDim * 2;                    // 256 B per (slot, head) row
-constexpr int kHalfStage = kTileKeys * kRowBytes;          // 16 KB of K (or V) per tile
+constexpr int kHalfStage = 32 * 1024;                      // K (or V) bytes of one tile
 constexpr int kStageBytes = 2 * kHalfStage;
-constexpr int kDecodeSmem = kStages * kStageBytes;         // 96 KB: two CTAs per SM
+constexpr int kSlotBufBytes = 2 * 128 * 4;                 // slot ids of two tiles
+constexpr int kDecodeSmem = kStages * kStageBytes + kSlotBufBytes;   // 193 KB: one CTA per SM
 constexpr float kLn2 = 0.693147180559945309f;
 
 __device__ __forceinline__ bool workspace_ok(const PlanHeader* hdr, int mode) {
   return hdr->magic == kMagic && hdr->mode == mode;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunch a) {
+template <int HG, int G>
+__global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunch a) {
+  constexpr int WPH = 8 / HG;                 // warps per KV head
+  constexpr int TK = 16 * WPH;                // keys per tile
+  constexpr int CH = HG * 16;                 // 16-byte chunks in one key's row of HG heads
+  constexpr int ROW = CH * 16;                // bytes of that row
+  constexpr int LOADS = kHalfStage / 16 / kThreads;   // copies per thread per tile, K and V each
+  constexpr int KEY_STEP = kThreads / CH;     // keys one pass of the block covers
+  static_assert(TK * ROW == kHalfStage && KEY_STEP * LOADS == TK, "tile geometry");
+
   extern __shared__ __align__(128) uint8_t smem[];
+  int32_t* sbuf = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes);   // [2][TK]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
   PlanHeader* hdr = a.ws.hdr;
@@ -48,13 +60,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
     if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
     return;
   }
-  const int num_items = hdr->num_items;
-  const int w = blockIdx.x;
-  if (w >= num_items * a.hkv) return;
-  const int4 it = a.ws.items[w / a.hkv];
-  const int h_kv = w % a.hkv;
+  const int groups = a.hkv / HG;
+  const int item = blockIdx.x / groups, grp = blockIdx.x % groups;
+  if (item >= hdr->num_items) return;
+  const int4 it = a.ws.items[item];
   const int r = it.x, split = it.y, kv0 = it.z, kv1 = it.w;
-  const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+  const int n_tiles = (kv1 - kv0 + TK - 1) / TK;
+  const int hw = warp % HG, kb = warp / HG;
+  const int h_kv = grp * HG + hw;
 
   // Q^T as the B operand: b0 = Q[head gid][16kk + 2tig .. +1], b1 = the same at +8.
   uint32_t qb0[8], qb1[8];
@@ -68,47 +81,55 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
     }
   }
 
-  // Gather assignment: thread -> (key ld_key of the tile, half row ld_half).
-  const int ld_key = tid >> 1, ld_half = tid & 1;
   const int page_shift = a.page_shift;
   const int page_mask = (1 << page_shift) - 1;
   const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
-  const size_t head_off = (size_t)h_kv * kHeadDim;
-  const size_t slot_stride = (size_t)a.hkv * kHeadDim;
-
-  auto slot_of = [&](int j) -> long long {
+  // raw table entry for key j (or -1 past the split); checked when it is stored
+  auto table_entry = [&](int j) -> int { return j < kv1 ? __ldg(table + (j >> page_shift)) : -1; };
+  auto entry_to_slot = [&](int page, int j) -> int {
     if (j >= kv1) return -1;
-    const int page = __ldg(table + (j >> page_shift));
     const long long slot = ((long long)page << page_shift) + (j & page_mask);
     if (page < 0 || slot >= a.num_slots) {
       set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-      return -1;
+      return -1;                                   // skipped: the row reads as zero
     }
-    return slot;
+    return (int)slot;
   };
+
+  // Gather roles: thread -> chunk ld_c of keys ld_k0 + KEY_STEP * i.
+  const int ld_c = tid % CH, ld_k0 = tid / CH;
+  const size_t slot_stride = (size_t)a.hkv * kHeadDim;
+  const size_t grp_off = (size_t)grp * HG * kHeadDim + (size_t)ld_c * 8;
   const uint32_t smem_base = smem_u32(smem);
-  auto issue = [&](int tile, long long slot) {
-    const uint32_t kdst = smem_base + (tile % kStages) * kStageBytes + ld_key * kRowBytes;
-    const uint32_t vdst = kdst + kHalfStage;
-    const size_t row = slot >= 0 ? (size_t)slot * slot_stride + head_off : 0;
-    const uint16_t* ks = a.k_pool + row;
-    const uint16_t* vs = a.v_pool + row;
-    const int bytes = slot >= 0 ? 16 : 0;  // rows past the split (or bad ids) are zero-filled
+  auto issue = [&](int tile) {
+    const uint32_t kst = smem_base + (tile % kStages) * kStageBytes;
+    const int32_t* sl = sbuf + (tile & 1) * TK;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int chunk = ld_half * 8 + c;
-      const uint32_t off = (uint32_t)((chunk ^ (ld_key & 7)) << 4);
-      cp_async_16(kdst + off, ks + chunk * 8, bytes);
-      cp_async_16(vdst + off, vs + chunk * 8, bytes);
+    for (int i = 0; i < LOADS; ++i) {
+      const int key = ld_k0 + KEY_STEP * i;
+      const int slot = sl[key];
+      const size_t off = slot >= 0 ? (size_t)slot * slot_stride + grp_off : 0;
+      const int bytes = slot >= 0 ? 16 : 0;      // rows past the split (or bad ids) are zero-filled
+      const uint32_t dst = kst + key * ROW + ((ld_c ^ (key & 7)) << 4);
+      cp_async_16(dst, a.k_pool + off, bytes);
+      cp_async_16(dst + kHalfStage, a.v_pool + off, bytes);
     }
   };
 
-  long long next_slot = slot_of(kv0 + ld_key);
-#pragma unroll
-  for (int t = 0; t < kStages - 1; ++t) {
-    if (t < n_tiles) issue(t, next_slot);
-    cp_async_commit();
-    next_slot = slot_of(kv0 + (t + 1) * kTileKeys + ld_key);
+  if (tid < TK) {
+    const int j0 = kv0 + tid, j1 = kv0 + TK + tid;
+    sbuf[tid] = entry_to_slot(table_entry(j0), j0);
+    sbuf[TK + tid] = entry_to_slot(table_entry(j1), j1);
+  }
+  __syncthreads();
+  if (0 < n_tiles) issue(0);
+  cp_async_commit();
+  if (1 < n_tiles) issue(1);
+  cp_async_commit();
+  __syncthreads();
+  if (tid < TK) {
+    const int j2 = kv0 + 2 * TK + tid;
+    sbuf[tid] = entry_to_slot(table_entry(j2), j2);
   }
 
   const float NEG_INF = -__int_as_float(0x7f800000);
@@ -117,32 +138,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
-  // ldmatrix row/chunk roles of this lane (see the fragment layouts of mma.m16n8k16)
+  // ldmatrix row/chunk roles of this lane (fragment layouts of mma.m16n8k16)
   const int mat = lane >> 3;
-  const int k_row = warp * 16 + (lane & 7) + ((mat & 1) << 3);   // K: A rows, chunk + (mat >> 1)
-  const int v_row = warp * 16 + (lane & 7) + ((mat >> 1) << 3);  // V: A^T rows, chunk + (mat & 1)
+  const int k_row = kb * 16 + (lane & 7) + ((mat & 1) << 3);   // K as A: chunk + (mat >> 1)
+  const int v_row = kb * 16 + (lane & 7) + ((mat >> 1) << 3);  // V^T as A: chunk + (mat & 1)
+  const uint32_t k_row_off = k_row * ROW, v_row_off = v_row * ROW;
+  const int head_chunk = hw * 16;
 
   for (int t = 0; t < n_tiles; ++t) {
     cp_async_wait<kStages - 2>();
     __syncthreads();
-    {
-      const int tp = t + kStages - 1;
-      if (tp < n_tiles) issue(tp, next_slot);
-      cp_async_commit();
-      next_slot = slot_of(kv0 + (tp + 1) * kTileKeys + ld_key);
-    }
+    if (t + 2 < n_tiles) issue(t + 2);
+    cp_async_commit();
+    const int j_next = kv0 + (t + 3) * TK + tid;
+    const int page_next = tid < TK ? table_entry(j_next) : -1;   // latency hidden by this tile
+
     const uint32_t kst = smem_base + (t % kStages) * kStageBytes;
     const uint32_t vst = kst + kHalfStage;
-
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       uint32_t af[4];
-      const int chunk = 2 * kk + (mat >> 1);
-      ldmatrix_x4(af, kst + k_row * kRowBytes + ((chunk ^ (k_row & 7)) << 4));
+      const int chunk = head_chunk + 2 * kk + (mat >> 1);
+      ldmatrix_x4(af, kst + k_row_off + ((chunk ^ (k_row & 7)) << 4));
       mma_bf16_16816(s, af, qb0[kk], qb1[kk]);
     }
-    const int key0 = kv0 + t * kTileKeys + warp * 16 + gid;
+    const int key0 = kv0 + t * TK + kb * 16 + gid;
     const int key1 = key0 + 8;
     const float x00 = key0 < kv1 ? s[0] * a.scale_log2 : NEG_INF;
     const float x01 = key0 < kv1 ? s[1] * a.scale_log2 : NEG_INF;
@@ -177,18 +198,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
       uint32_t af[4];
-      const int chunk = 2 * mt + (mat & 1);
-      ldmatrix_x4_trans(af, vst + v_row * kRowBytes + ((chunk ^ (v_row & 7)) << 4));
+      const int chunk = head_chunk + 2 * mt + (mat & 1);
+      ldmatrix_x4_trans(af, vst + v_row_off + ((chunk ^ (v_row & 7)) << 4));
       mma_bf16_16816(o[mt], af, pb0, pb1);
     }
+    if (tid < TK) sbuf[((t + 3) & 1) * TK + tid] = entry_to_slot(page_next, j_next);
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Combine the four warps' (m, l, O) through shared memory.
-  float* red_o = reinterpret_cast<float*>(smem);   // [4 warps][8 heads][128 d]
-  float* red_m = red_o + 4 * 8 * kHeadDim;         // [4][8]
-  float* red_l = red_m + 32;                       // [4][8]
+  // Combine the warps of each head through shared memory.
+  float* red_o = reinterpret_cast<float*>(smem);   // [8 warps][8 heads][128 d]
+  float* red_m = red_o + 8 * 8 * kHeadDim;         // [8][8]
+  float* red_l = red_m + 64;                       // [8][8]
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l_run0 += __shfl_xor_sync(0xffffffffu, l_run0, off);
@@ -213,24 +235,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
   __syncthreads();
 
   const int splits = a.ws.req_splits[r];
-  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-    const int h = idx / kHeadDim, d = idx % kHeadDim;
+  for (int idx = tid; idx < HG * G * kHeadDim; idx += kThreads) {
+    const int hl = idx / (G * kHeadDim), g = (idx / kHeadDim) % G, d = idx % kHeadDim;
     float M = NEG_INF;
 #pragma unroll
-    for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, red_m[ww * 8 + h]);
+    for (int k2 = 0; k2 < WPH; ++k2) M = fmaxf(M, red_m[(k2 * HG + hl) * 8 + g]);
     float O = 0.f, lse2 = NEG_INF;
     if (M != NEG_INF) {
       float wsum = 0.f, acc = 0.f;
 #pragma unroll
-      for (int ww = 0; ww < 4; ++ww) {
-        const float f = ex2(red_m[ww * 8 + h] - M);
-        wsum += red_l[ww * 8 + h] * f;
-        acc += red_o[(ww * 8 + h) * kHeadDim + d] * f;
+      for (int k2 = 0; k2 < WPH; ++k2) {
+        const int wi = (k2 * HG + hl) * 8 + g;
+        const float f = ex2(red_m[wi] - M);
+        wsum += red_l[wi] * f;
+        acc += red_o[wi * kHeadDim + d] * f;
       }
       O = acc / wsum;
       lse2 = M + __log2f(wsum);
     }
-    const int hq_idx = h_kv * G + h;
+    const int hq_idx = (grp * HG + hl) * G + g;
     if (splits == 1) {
       a.out[((size_t)r * a.hq + hq_idx) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(O));
       if (d == 0 && a.lse_out) a.lse_out[(size_t)r * a.hq + hq_idx] = lse2 * kLn2;
@@ -299,22 +322,33 @@ __global__ void debug_gather_kernel(GatherLaunch a) {
   }
 }
 
-template <int G>
-cudaError_t launch_decode_g(const DecodeLaunch& a, cudaStream_t s) {
+template <int HG, int G>
+cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<G>,
+    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<HG, G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDecodeSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  decode_splitkv_kernel<G><<<a.max_items * a.hkv, kThreads, kDecodeSmem, s>>>(a);
+  const int groups = a.hkv / HG;
+  decode_splitkv_kernel<HG, G><<<a.max_items * groups, kThreads, kDecodeSmem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   merge_kernel<<<(a.batch * a.hq + 3) / 4, 128, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_decode_g(const DecodeLaunch& a, cudaStream_t s) {
+  switch (decode_heads_per_cta(a.hkv)) {
+    case 8: return launch_decode_hg<8, G>(a, s);
+    case 4: return launch_decode_hg<4, G>(a, s);
+    case 2: return launch_decode_hg<2, G>(a, s);
+    default: return launch_decode_hg<1, G>(a, s);
+  }
 }
 
 }  // namespace

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     ws.req_len[r] = L;
     if (a.mode == PA_MODE_DECODE) my_tiles += cdiv_ll(L, a.tile);
   }
-  const long long total = block_sum(my_tiles, red) * a.hkv;
+  const long long total = block_sum(my_tiles, red) * (a.hkv / decode_heads_per_cta(a.hkv));
   int chunk = 0;
   if (a.mode == PA_MODE_DECODE) {
     const long long slots = (long long)a.num_sms * kDecodeCtasPerSm;

@@ -91,7 +91,7 @@ def _gpu_plan(mode, lens, cu=None, hq=8, hkv=2, page_size=1, max_splits=0, max_k
 
 
 def _oracle_plan(mode, lens, cu=None, hkv=2, page_size=1, max_splits=0, max_q=0):
-    ms = (64 if max_splits == 0 else max_splits) if mode == 0 else 1
+    ms = (128 if max_splits == 0 else max_splits) if mode == 0 else 1
     return op.plan(mode, lens, cu, hkv=hkv, page_size=page_size, num_sms=num_sms(), max_splits=ms,
                    max_q_tokens=max_q)
 

@@ -69,11 +69,17 @@ def test_decode_plan_at_the_workload_shapes():
     rng = np.random.default_rng(31)
     lens = [int(x) for x in rng.integers(512, 8193, 64)]
     _check_decode_invariants(lens, 8, 1, 148, 64)
+    pl = op.plan(op.MODE_DECODE, [131072] * 8, hkv=8, page_size=64, num_sms=148, max_splits=128)
+    # one CTA covers all 8 KV heads: total = 8 * 2048 tiles over 148 * 4 slots,
+    # chunk = ceil(16384 / 592) = 28 tiles, splits = ceil(2048 / 28) = 74 per request
+    assert pl["chunk_tiles"] == 28
+    assert pl["req_splits"] == [74] * 8
+    assert pl["num_items"] == 592 <= op.max_items(op.MODE_DECODE, 8, 8, 148) == 600
+    # with a cap of 64 splits: chunk_r = ceil(2048 / 64) = 32 tiles, exactly 64 splits
     pl = op.plan(op.MODE_DECODE, [131072] * 8, hkv=8, page_size=64, num_sms=148, max_splits=64)
-    # total = 8 * 2048 * 8 tile-heads over 148 * 8 slots: chunk = ceil(131072 / 1184) = 111 tiles
-    assert pl["chunk_tiles"] == 111
-    assert pl["req_splits"] == [19] * 8
-    assert pl["num_items"] == 152 <= op.max_items(op.MODE_DECODE, 8, 8, 148)
+    assert pl["req_splits"] == [64] * 8 and pl["items"][0] == (0, 0, 0, 32 * 64)
+    # 16 KV heads: two CTAs per item, so half the items for the same slots
+    assert op.decode_head_groups(16) == 2 and op.decode_head_groups(12) == 3 and op.decode_head_groups(8) == 1
 
 
 def test_plan_is_a_function_of_lengths_only():
