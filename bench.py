@@ -228,6 +228,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_llama3_8b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: fewer layer calls per step than the workload defines")
+    ap.add_argument("--distinct-pools", type=int, default=0,
+                    help="profiling only: allocate fewer pools (layers rotate over them)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -242,6 +246,10 @@ def main():
 
     cfg_id, cls = WORKLOADS[args.workload]
     spec = wl.CONFIGS[cfg_id]
+    if args.layers:
+        spec = spec.scaled(layers=args.layers)
+    if args.distinct_pools:
+        spec = spec.scaled(distinct_pools=args.distinct_pools)
     hbm_peak, bf16_peak, bf16_sus, peak_src = load_peaks()
 
     if args.impl == "reference":
