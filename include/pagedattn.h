@@ -229,6 +229,34 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
                                  uint16_t* d_out, pa_stream_t stream);
 
 /*
+ * attn_decode_paged_noalloc - attn_plan followed by attn_decode_paged in one
+ * call, for callers that cannot allocate device memory (a host framework that
+ * owns every device allocation and offers no allocator, a plugin that must not
+ * touch its host process's memory pool, or a call site where an allocation
+ * would synchronise the device or exceed a fixed memory budget).  The pages
+ * have no counterpart to this entry point; it exists for such callers.
+ *
+ * Arguments are those of attn_plan (mode PA_MODE_DECODE, no cu_seqlens_q) and
+ * attn_decode_paged, without the workspace: the plan, work list and split
+ * partials live in a 16 MiB array inside the library, which every GPU that
+ * loads the library holds until the process exits.  The call allocates and
+ * frees nothing.  Plans whose pa_plan_workspace_size() exceeds 16 MiB are
+ * rejected with PA_ERR_WORKSPACE (the Llama-3-8B decode shape, batch 64 x
+ * Hq 32 on 148 SMs, needs about 11 MB).  The first call on a device looks up
+ * the array's device address (once per device, with that device current); make
+ * that first call before any stream capture.  All calls share the array and it
+ * keeps the last call's contents: calls that overlap on the GPU (other streams
+ * or host threads) race and must be ordered by the caller.  Device-side errors
+ * are recorded in the array's header and are not readable through
+ * pa_read_device_error, which needs a workspace pointer.
+ */
+pa_status attn_decode_paged_noalloc(const pa_plan_params* params, const int32_t* d_seq_lens,
+                                    const uint16_t* d_q, const uint16_t* d_k_pool,
+                                    const uint16_t* d_v_pool, int64_t num_slots,
+                                    const int32_t* d_page_table, int64_t pt_pitch, float sm_scale,
+                                    uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
+
+/*
  * attn_debug_gather - copy, for request r and KV head h_kv, the slot ids and
  * the K rows the kernels gather: d_slots_out int32 [L], d_rows_out bf16 [L][D]
  * for positions 0 .. L-1, L = min(d_seq_lens[r], max_len).  Out-of-range ids

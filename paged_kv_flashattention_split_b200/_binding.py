@@ -21,7 +21,7 @@ PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE = 0, 1, 2
 
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
-            "pa_status_string", "pa_version")
+            "pa_status_string", "pa_version", "attn_decode_paged_noalloc")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "attn_debug_gather": (_I32, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _I64, _P, _I64,
                                          _P, _P, _P]),
             "pa_read_device_error": (_I32, [_P, _P]),
+            "attn_decode_paged_noalloc": (_I32, [PP, _P, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
             "pa_status_string": (ctypes.c_char_p, [_I32]),
             "pa_version": (_I32, []),
         }
@@ -162,6 +163,17 @@ def attn_debug_gather(seq_lens, r, h_kv, hkv, page_size, max_len, k_pool, page_t
                                  _ptr(k_pool), int(num_slots), _ptr(page_table), int(pt_pitch),
                                  _ptr(slots_out), _ptr(rows_out), _stream(stream))
     return _check(st, "attn_debug_gather", raise_on_error)
+
+
+def attn_decode_paged_noalloc(params, seq_lens, q, k_pool, v_pool, page_table, sm_scale, out, lse_out=None,
+                              num_slots=None, pt_pitch=None, stream=None, raise_on_error=True) -> int:
+    """Plan and decode without a caller workspace (the library's fixed 16 MiB array is used)."""
+    num_slots = k_pool.shape[0] if num_slots is None else num_slots
+    pt_pitch = page_table.shape[-1] if pt_pitch is None else pt_pitch
+    st = lib().attn_decode_paged_noalloc(ctypes.byref(params), _ptr(seq_lens), _ptr(q), _ptr(k_pool),
+                                         _ptr(v_pool), int(num_slots), _ptr(page_table), int(pt_pitch),
+                                         float(sm_scale), _ptr(out), _ptr(lse_out), _stream(stream))
+    return _check(st, "attn_decode_paged_noalloc", raise_on_error)
 
 
 def pa_read_device_error(ws, stream=None) -> int:
