@@ -211,7 +211,61 @@ class DecodeWorkload:
         return nbytes, done, f"oracle.attention.decode on requests 0..{r - 1} of layer 0 ({r} of {spec.batch} requests, {int(lens[:r].sum())} keys); host copy {prep:.1f}s untimed"
 
 
+class SageWorkload(DecodeWorkload):
+    """plan + L layer calls of the 8-bit Sage decode, each layer with its own 8-bit pools."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        import paged_kv_flashattention_split_b200 as pa
+        self.pa, self.spec, self.dev = pa, spec, device
+        self.batch = wl.make_batch(spec, device)
+        n_pools = spec.distinct_pools or spec.layers
+        self.layers_data = [wl.make_sage_layer(spec, self.batch, l, device) for l in range(n_pools)]
+        self.q = [self.layers_data[l % n_pools].q8 for l in range(spec.layers)]
+        self.out = [torch.empty((spec.batch, spec.hq, spec.head_dim), dtype=torch.bfloat16, device=device)
+                    for _ in range(spec.layers)]
+        self.params = pa.make_params(pa.PA_MODE_SAGE_DECODE, spec.batch, spec.hq, spec.hkv, spec.head_dim, 64,
+                                     max_kv_len=self.batch.page_table.shape[1] * 64, sage_k_block=64)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        L = self.batch.seq_lens.cpu().tolist()
+        # K8 + V8 rows (1 B each), one sfK per 64-key block and head, page ids, Q8 + sfQ, bf16 O
+        self.layer_bytes = float(sum(L) * spec.hkv * spec.head_dim * 2
+                                 + sum((x + 63) // 64 for x in L) * (spec.hkv * 4 + 4)
+                                 + spec.batch * spec.hq * (spec.head_dim * 1 + 4 + spec.head_dim * 2))
+        self.step_bytes = self.layer_bytes * spec.layers
+        self.launches_per_step = 1 + spec.layers
+
+    def layer(self, l):
+        d = self.layers_data[l % len(self.layers_data)]
+        self.pa.attn_decode_paged_sage(self.params, self.ws, d.q8, d.sf_q, d.k8, d.v8, d.sf_k, d.sf_v, d.v_mean,
+                                       self.batch.page_table, self.out[l])
+
+    def setup_e2e(self):
+        self.h_q = [x.cpu().pin_memory() for x in self.q]
+        self.h_lens = self.batch.seq_lens.cpu().pin_memory()
+        self.h_table = self.batch.page_table.cpu().pin_memory()
+        self.h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in self.out]
+        self.e2e_h2d = sum(x.numel() for x in self.h_q) + self.h_lens.numel() * 4 + self.h_table.numel() * 4
+        self.e2e_d2h = sum(x.numel() * 2 for x in self.h_out)
+
+    def oracle_sample(self, seconds=12.0):
+        from oracle import sage as osg
+        spec = self.spec
+        d = self.layers_data[0]
+        host = {k: getattr(d, k).cpu().numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        nbytes, r = 0.0, 0
+        t0 = time.perf_counter()
+        while r < spec.batch and (time.perf_counter() - t0) < seconds:
+            osg.sage_decode(host["q8"][r:r + 1], host["sf_q"][r:r + 1], host["k8"], host["v8"], host["sf_k"],
+                            host["sf_v"], host["v_mean"], table[r:r + 1], lens[r:r + 1], 64)
+            nbytes += self.layer_bytes * float(lens[r]) / float(lens.sum())
+            r += 1
+        return nbytes, time.perf_counter() - t0, f"oracle.sage.sage_decode on requests 0..{r - 1} of layer 0"
+
+
 WORKLOADS = {
+    "sage_decode": (5, SageWorkload),
     "decode_llama3_8b": (2, DecodeWorkload),
     "decode_long_llama3_70b": (4, DecodeWorkload),
     "decode_tiny": (1, DecodeWorkload),
@@ -318,7 +372,8 @@ def main():
 
     avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
     achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_" + args.workload, source_hash("decode.cu", "common.cuh"))
+    kernel_src = ("sage.cu", "common.cuh") if args.workload == "sage_decode" else ("decode.cu", "common.cuh")
+    traffic = recorded_traffic(args.workload, source_hash(*kernel_src))
 
     line = {
         "metric": METRIC,
@@ -331,21 +386,23 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "int8/e4m3 in, fp32 math, bf16 out" if args.workload == "sage_decode" else "bf16",
         "data": "synthetic",
         "config": {
             "workload": args.workload,
             "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
             "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
-            "step": "attn_plan + %d x attn_decode_paged" % spec.layers,
+            "step": "attn_plan + %d x %s" % (spec.layers, "attn_decode_paged_sage" if args.workload == "sage_decode"
+                                              else "attn_decode_paged"),
             "l2": "inputs larger than L2 (each layer reads its own >1 GB pool)",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-            "kernel": "attn_decode_paged call (decode_splitkv_kernel + merge_kernel), per-layer CUDA events",
+            "kernel": ("sage_decode_kernel (one launch per attn_decode_paged_sage call)" if args.workload == "sage_decode"
+                       else "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)") + ", per-layer CUDA events",
             "peak_source": peak_src,
         },
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(work.e2e_h2d),

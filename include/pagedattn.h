@@ -166,7 +166,7 @@ pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
  * Each (request, KV head, split) CTA gathers its K/V rows with 16-byte
  * copies through the slot table, packs the Hq / Hkv query heads of the KV head
  * so each row is read once, and keeps a running max / sum; requests split
- * into several ranges are combined by a log-sum-exp merge kernel.
+ * into several key ranges are combined by a log-sum-exp merge kernel.
  *
  * params, d_ws    the plan (mode PA_MODE_DECODE) built by attn_plan.
  * d_q             bf16 [B][Hq][D];  d_k_pool, d_v_pool bf16 [num_slots][Hkv][D].

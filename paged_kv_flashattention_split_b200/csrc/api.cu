@@ -23,8 +23,6 @@ struct Derived {
   WsLayout layout{};
 };
 
-constexpr size_t kSageScoreBudget = 64 * 1024;   // bytes of on-chip scores per Sage CTA
-
 int ilog2(int x) {
   int s = 0;
   while ((1 << s) < x) ++s;
@@ -85,7 +83,8 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
     case PA_MODE_SAGE_DECODE:
       if (p->max_q_tokens != 0 || p->max_splits > 1) return PA_ERR_INVALID;
       if (p->sage_k_block != kSageBlock || P != kSageBlock) return PA_ERR_UNSUPPORTED;
-      if ((size_t)G * (size_t)p->max_kv_len * 4 > kSageScoreBudget) return PA_ERR_UNSUPPORTED;
+      // shared-memory budget of the scores a CTA keeps (a quarter of the row per CTA)
+      if ((size_t)G * (size_t)sage_cap(p->max_kv_len) * 4 > kSageScoreBudget) return PA_ERR_UNSUPPORTED;
       d->max_splits = 1;
       d->tile = kSageBlock;
       break;
@@ -111,7 +110,7 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
   int n = 2;
   while (n < d->max_items) n <<= 1;
   d->sort_n = n;
-  d->layout = ws_layout(p->mode, p->batch, p->hq, p->head_dim, d->max_items);
+  d->layout = ws_layout(p->mode, p->batch, p->hq, p->hkv, p->head_dim, d->max_items);
   return PA_OK;
 }
 
@@ -215,9 +214,38 @@ pa_status attn_extend_paged(const pa_plan_params* params, const void* d_ws, size
                             const uint16_t* d_q, const uint16_t* d_k_pool, const uint16_t* d_v_pool,
                             int64_t num_slots, const int32_t* d_page_table, int64_t pt_pitch,
                             float sm_scale, uint16_t* d_out, float* d_lse_out, pa_stream_t stream) {
-  (void)params; (void)d_ws; (void)ws_bytes; (void)d_q; (void)d_k_pool; (void)d_v_pool; (void)num_slots;
-  (void)d_page_table; (void)pt_pitch; (void)sm_scale; (void)d_out; (void)d_lse_out; (void)stream;
-  return PA_ERR_UNSUPPORTED;
+  Derived d;
+  pa_status st = derive(params, &d);
+  if (st != PA_OK) return st;
+  if (params->mode != PA_MODE_EXTEND) return PA_ERR_WORKSPACE;
+  if (!d_ws || !d_q || !d_k_pool || !d_v_pool || !d_page_table || !d_out) return PA_ERR_INVALID;
+  if (!aligned16(d_ws) || !aligned16(d_q) || !aligned16(d_k_pool) || !aligned16(d_v_pool) || !aligned16(d_out))
+    return PA_ERR_INVALID;
+  if (d_lse_out && (reinterpret_cast<uintptr_t>(d_lse_out) & 3u)) return PA_ERR_INVALID;
+  if (num_slots < params->page_size || num_slots >= (1LL << 31) || pt_pitch < 1 || params->max_q_tokens < 1)
+    return PA_ERR_INVALID;
+  const long long need_pitch = ((long long)params->max_kv_len + params->page_size - 1) / params->page_size;
+  if (pt_pitch < need_pitch) return PA_ERR_INVALID;
+  if (ws_bytes < d.layout.total) return PA_ERR_WORKSPACE;
+  if ((st = check_arch()) != PA_OK) return st;
+  ExtendArgs a;
+  a.ws = ws_view(const_cast<void*>(d_ws), d.layout);
+  a.q = d_q;
+  a.k_pool = d_k_pool;
+  a.v_pool = d_v_pool;
+  a.q_rows = params->max_q_tokens;
+  a.num_slots = num_slots;
+  a.page_table = d_page_table;
+  a.pt_pitch = pt_pitch;
+  a.out = d_out;
+  a.lse_out = d_lse_out;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.hq = params->hq;
+  a.hkv = params->hkv;
+  a.page_size = params->page_size;
+  a.page_shift = d.page_shift;
+  a.max_items = d.max_items;
+  return from_cuda(launch_extend(a, (cudaStream_t)stream));
 }
 
 pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
@@ -225,10 +253,38 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
                                  const uint8_t* d_v8_pool, const float* d_sf_k, const float* d_sf_v,
                                  const float* d_v_mean, int64_t num_slots, const int32_t* d_page_table,
                                  int64_t pt_pitch, uint16_t* d_out, pa_stream_t stream) {
-  (void)params; (void)d_ws; (void)ws_bytes; (void)d_q8; (void)d_sf_q; (void)d_k8_pool; (void)d_v8_pool;
-  (void)d_sf_k; (void)d_sf_v; (void)d_v_mean; (void)num_slots; (void)d_page_table; (void)pt_pitch;
-  (void)d_out; (void)stream;
-  return PA_ERR_UNSUPPORTED;
+  Derived d;
+  pa_status st = derive(params, &d);
+  if (st != PA_OK) return st;
+  if (params->mode != PA_MODE_SAGE_DECODE) return PA_ERR_WORKSPACE;
+  if (!d_ws || !d_q8 || !d_sf_q || !d_k8_pool || !d_v8_pool || !d_sf_k || !d_sf_v || !d_page_table || !d_out)
+    return PA_ERR_INVALID;
+  if (!aligned16(d_ws) || !aligned16(d_q8) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) || !aligned16(d_out))
+    return PA_ERR_INVALID;
+  if (num_slots < kSageBlock || num_slots % kSageBlock != 0 || num_slots >= (1LL << 31) || pt_pitch < 1)
+    return PA_ERR_INVALID;
+  const long long need_pitch = ((long long)params->max_kv_len + params->page_size - 1) / params->page_size;
+  if (pt_pitch < need_pitch) return PA_ERR_INVALID;
+  if (ws_bytes < d.layout.total) return PA_ERR_WORKSPACE;
+  if ((st = check_arch()) != PA_OK) return st;
+  SageLaunchArgs a;
+  a.ws = ws_view(const_cast<void*>(d_ws), d.layout);
+  a.q8 = d_q8;
+  a.sf_q = d_sf_q;
+  a.k8 = d_k8_pool;
+  a.v8 = d_v8_pool;
+  a.sf_k = d_sf_k;
+  a.sf_v = d_sf_v;
+  a.v_mean = d_v_mean;
+  a.num_slots = num_slots;
+  a.page_table = d_page_table;
+  a.pt_pitch = pt_pitch;
+  a.out = d_out;
+  a.batch = params->batch;
+  a.hq = params->hq;
+  a.hkv = params->hkv;
+  a.max_kv_len = params->max_kv_len;
+  return from_cuda(launch_sage(a, (cudaStream_t)stream));
 }
 
 pa_status attn_debug_gather(const int32_t* d_seq_lens, int32_t r, int32_t h_kv, int32_t hkv,

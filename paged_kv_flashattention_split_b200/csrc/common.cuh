@@ -20,6 +20,7 @@ constexpr int kDecodeCtasPerSm = 4;              // decode CTAs a plan aims for,
 constexpr int kExtendQTile = 128;
 constexpr int kExtendKvTile = 128;
 constexpr int kSageBlock = 64;
+constexpr size_t kSageScoreBudget = 64 * 1024;  // bytes of on-chip scores per Sage CTA (G x keys x 4)
 constexpr int kMaxBatch = 8192;
 constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capacity
 
@@ -43,7 +44,7 @@ __host__ __device__ inline int decode_heads_per_cta(int hkv) {
   return hkv % 8 == 0 ? 8 : hkv % 4 == 0 ? 4 : hkv % 2 == 0 ? 2 : 1;
 }
 
-inline WsLayout ws_layout(int mode, int batch, int hq, int head_dim, int max_items) {
+inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, int max_items) {
   WsLayout w{};
   size_t off = sizeof(PlanHeader);
   w.req_splits = off; off += 4 * (size_t)batch;

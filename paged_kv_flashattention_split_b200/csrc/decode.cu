@@ -265,12 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunc
   }
 }
 
-// One warp per (request, query head) whose request was split: combine the
+// One warp per (request, query head) of a request that was split: combine the
 // split partials, lse = log2 sum_s 2^lse_s, O = sum_s 2^(lse_s - lse) O_s.
-__global__ void __launch_bounds__(128) merge_kernel(DecodeLaunch a) {
+// Lanes read the split LSEs in parallel; each lane owns 4 of the 128 outputs
+// and keeps up to 8 splits' loads in flight.
+__global__ void __launch_bounds__(256) merge_kernel(DecodeLaunch a) {
   PlanHeader* hdr = a.ws.hdr;
   if (!workspace_ok(hdr, PA_MODE_DECODE)) return;
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (gw >= a.batch * a.hq) return;
   const int r = gw / a.hq, h = gw % a.hq;
   const int splits = a.ws.req_splits[r];
@@ -278,33 +280,39 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeLaunch a) {
   const int base = a.ws.req_base[r];
   if (base + splits > a.max_items) return;  // only after a plan overflow, which the plan flags
   const float NEG_INF = -__int_as_float(0x7f800000);
+  const float* lse = a.ws.partial_lse + (size_t)base * a.hq + h;      // stride hq per split
+  const float* po = a.ws.partial_o + ((size_t)base * a.hq + h) * kHeadDim + 4 * lane;
   float M = NEG_INF;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, a.ws.partial_lse[(size_t)(base + s) * a.hq + h]);
+  for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, lse[(size_t)sp * a.hq]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
+  float wpart = 0.f;
   if (M != NEG_INF) {
-    for (int s = 0; s < splits; ++s) {
-      const size_t p = (size_t)(base + s) * a.hq + h;
-      const float f = ex2(a.ws.partial_lse[p] - M);
-      const float4 v = reinterpret_cast<const float4*>(a.ws.partial_o + p * kHeadDim)[lane];
-      wsum += f;
-      acc.x += f * v.x;
-      acc.y += f * v.y;
-      acc.z += f * v.z;
-      acc.w += f * v.w;
+    for (int s0 = 0; s0 < splits; s0 += 32) {
+      const float w_l = s0 + lane < splits ? ex2(lse[(size_t)(s0 + lane) * a.hq] - M) : 0.f;
+      wpart += w_l;
+      const int n = min(32, splits - s0);
+#pragma unroll 8
+      for (int j = 0; j < n; ++j) {
+        const float w = __shfl_sync(0xffffffffu, w_l, j);
+        const float4 v = *reinterpret_cast<const float4*>(po + (size_t)(s0 + j) * a.hq * kHeadDim);
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
+      }
     }
-    const float inv = 1.f / wsum;
-    acc.x *= inv;
-    acc.y *= inv;
-    acc.z *= inv;
-    acc.w *= inv;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wpart += __shfl_xor_sync(0xffffffffu, wpart, off);
+  const float inv = M == NEG_INF ? 0.f : 1.f / wpart;
   uint2 packed;
-  packed.x = pack_bf16x2(acc.x, acc.y);
-  packed.y = pack_bf16x2(acc.z, acc.w);
+  packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
   reinterpret_cast<uint2*>(a.out + ((size_t)r * a.hq + h) * kHeadDim)[lane] = packed;
   if (lane == 0 && a.lse_out)
-    a.lse_out[(size_t)r * a.hq + h] = M == NEG_INF ? NEG_INF : (M + __log2f(wsum)) * kLn2;
+    a.lse_out[(size_t)r * a.hq + h] = M == NEG_INF ? NEG_INF : (M + __log2f(wpart)) * kLn2;
 }
 
 __global__ void debug_gather_kernel(GatherLaunch a) {
@@ -337,7 +345,7 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   decode_splitkv_kernel<HG, G><<<a.max_items * groups, kThreads, kDecodeSmem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_kernel<<<(a.batch * a.hq + 3) / 4, 128, 0, s>>>(a);
+  merge_kernel<<<(a.batch * a.hq + 7) / 8, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -29,6 +29,41 @@ struct DecodeLaunch {
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s);
 
+struct SageLaunchArgs {
+  WsView ws;
+  const int8_t* q8;
+  const float* sf_q;
+  const int8_t* k8;
+  const uint8_t* v8;
+  const float* sf_k;
+  const float* sf_v;
+  const float* v_mean;
+  int64_t num_slots;
+  const int32_t* page_table;
+  int64_t pt_pitch;
+  uint16_t* out;
+  int batch, hq, hkv, max_kv_len;
+};
+cudaError_t launch_sage(const SageLaunchArgs& a, cudaStream_t s);
+int sage_cap(int max_kv_len);          // score keys per CTA per head for this max length
+size_t sage_smem_bytes(int G, int cap);
+
+struct ExtendArgs {
+  WsView ws;
+  const uint16_t* q;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  int64_t q_rows;          // rows of the Q / O buffers (max_q_tokens)
+  int64_t num_slots;
+  const int32_t* page_table;
+  int64_t pt_pitch;
+  uint16_t* out;
+  float* lse_out;
+  float scale_log2;
+  int hq, hkv, page_size, page_shift, max_items;
+};
+cudaError_t launch_extend(const ExtendArgs& a, cudaStream_t s);
+
 struct GatherLaunch {
   const int32_t* seq_lens;
   int r, h_kv, hkv, page_shift, max_len;

@@ -47,7 +47,7 @@ def sage_row_rel_error(gpu_bf16, ref):
     return float(np.max(num / den))
 
 
-def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 128):
+def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 128, hkv: int = 8):
     """Byte offsets of the workspace arrays, from the layout documented at attn_plan."""
     off = 64
     o = {}
@@ -74,8 +74,8 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
     """Parse the plan the GPU wrote into the workspace (host copy)."""
     raw = ws.cpu().numpy().view(np.uint8)
     hdr = raw[:64].view(np.int32)
-    num_items, max_items = int(hdr[7]), int(hdr[8])
-    o = ws_offsets(mode, batch, hq, max_items)
+    num_items, max_items, hkv = int(hdr[7]), int(hdr[8]), int(hdr[4])
+    o = ws_offsets(mode, batch, hq, max_items, hkv=hkv)
 
     def arr(name, n):
         return raw[o[name]:o[name] + 4 * n].view(np.int32).tolist()
@@ -84,7 +84,8 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
     return {"magic": int(hdr[0]), "mode": int(hdr[1]), "tile": int(hdr[9]), "chunk_tiles": int(hdr[10]),
             "error_word": int(hdr[11]), "num_items": num_items, "max_items": max_items,
             "req_splits": arr("req_splits", batch), "req_base": arr("req_base", batch + 1),
-            "req_len": arr("req_len", batch), "items": [tuple(int(x) for x in it) for it in items]}
+            "req_len": arr("req_len", batch),
+            "items": [tuple(int(x) for x in it) for it in items]}
 
 
 def alloc_ws(params, device="cuda"):

@@ -81,7 +81,7 @@ def test_workspace_size_matches_documented_layout(lib):
             mi = -(-9000 // 128) + 33
         else:
             mi = 33
-        assert n == ws_offsets(mode, 33, 32, mi)["total"]
+        assert n == ws_offsets(mode, 33, 32, mi, hkv=8)["total"]
 
 
 def test_host_checks_precede_device_use(lib):
