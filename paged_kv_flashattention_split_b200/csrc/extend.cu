@@ -1,0 +1,497 @@
+// extend.cu - bf16 causal EXTEND over the paged cache on the 5th-generation tensor cores.
+//
+// New token i of request r (absolute position p_r + i) attends to keys
+// 0 .. p_r + i of its cached prefix and of the new tokens, all already in the
+// pool: O = softmax(scale Q K^T + causal mask) V.  The tiled online softmax
+// gives the standard result without the score matrix ever reaching HBM
+// ("FlashAttention: 优化计算过程中的临时显存占用", sections 1-2); the two
+// forward modes are those of "Implement Flash Attention Back End in SGLang".
+//
+// One CTA per (query tile of 128 new tokens, query head), 6 warps:
+//   warp 0      producer: TMA loads of the Q tile once and of K/V key tiles
+//               (128 keys, i.e. 128 / P pages) into a 2-stage ring, each page
+//               one box of a 4-D tensor map over the pool [slot][head][d];
+//   warp 1      allocates TMEM and issues, from one thread,
+//                   S  = Q K^T   (tcgen05.mma kind::f16, M 128, N 128, S in TMEM)
+//                   O += P V     (P from shared memory, O accumulated in TMEM);
+//   warps 2-5   softmax: thread i owns query row i (TMEM lane i), reads its
+//               128 scores with tcgen05.ld, applies the causal mask on the
+//               diagonal tiles, keeps a running max (rescaling O in TMEM only
+//               when the max grows by more than 2^8) and writes P (bf16) to
+//               shared memory in the MMA's swizzled layout; at the end it
+//               normalises its O row and stores it.
+// The issue order S(0), then per tile S(j+1) before PV(j), lets the tensor
+// cores compute the next scores while the softmax works on the current ones.
+// Key tiles past the last one any row of the query tile can see are never
+// loaded (causal tile skipping).
+//
+// Every wait on an mbarrier is bounded: on timeout the CTA records
+// PA_ERR_DEVICE_INDEX in the workspace, every role stops, the MMA issuer
+// drains its tensor-core work, and TMEM is freed before the CTA exits.
+#include <cuda.h>
+
+#include "kernels.h"
+
+namespace pa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTileKeys = 128;
+constexpr int kNumStages = 2;
+constexpr int kChunkBytes = 128 * 128;           // one 64-column half of a 128 x 128 bf16 tile
+constexpr int kTileBytes = 2 * kChunkBytes;      // 32 KB
+constexpr uint32_t kTmemCols = 256;              // S: columns [0,128), O: [128, 256)
+constexpr uint32_t kWaitLimit = 1u << 20;
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kRescaleThreshold = 8.f;         // log2 units
+
+// shared-memory plan (offsets from a 1024-aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffV = kOffK + kNumStages * kTileBytes;
+constexpr int kOffP = kOffV + kNumStages * kTileBytes;
+constexpr int kOffBar = kOffP + kTileBytes;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers, TMEM address, flags, alignment slack
+
+struct ExtendLaunch {
+  CUtensorMap tm_q, tm_k, tm_v;   // 64-byte aligned kernel parameters
+  WsView ws;
+  const int32_t* page_table;
+  int64_t pt_pitch;
+  int64_t num_slots;
+  uint16_t* out;
+  float* lse_out;
+  float scale_log2;
+  int64_t q_rows;
+  int hq, hkv, page_size, page_shift, box_rows, max_items;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// smem matrix descriptor: 128B swizzle, 8-row groups 1024 B apart (SBO), LBO as given
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)(lbo_bytes >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// instruction descriptor, kind::f16: bf16 A and B, fp32 D, M = 128, N = 128
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescS = kIdescBase;                 // A (Q) and B (K) K-major
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);   // B (V) MN-major: d contiguous
+
+struct Shared {
+  uint32_t base;      // 1024-aligned shared address of the tile buffers
+  uint32_t bar_q, bar_k_full[kNumStages], bar_v_full[kNumStages], bar_kv_empty[kNumStages];
+  uint32_t bar_s_full, bar_s_free, bar_p_full, bar_o_done, bar_drain;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_constant__ ExtendLaunch a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  Shared sh;
+  sh.base = base;
+  const uint32_t bars = base + kOffBar;
+  sh.bar_q = bars;
+  for (int s = 0; s < kNumStages; ++s) {
+    sh.bar_k_full[s] = bars + 8 * (1 + s);
+    sh.bar_v_full[s] = bars + 8 * (1 + kNumStages + s);
+    sh.bar_kv_empty[s] = bars + 8 * (1 + 2 * kNumStages + s);
+  }
+  sh.bar_s_full = bars + 8 * (1 + 3 * kNumStages);
+  sh.bar_s_free = sh.bar_s_full + 8;
+  sh.bar_p_full = sh.bar_s_full + 16;
+  sh.bar_o_done = sh.bar_s_full + 24;
+  sh.bar_drain = sh.bar_s_full + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBar + 200);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  PlanHeader* hdr = a.ws.hdr;
+  if (hdr->magic != kMagic || hdr->mode != PA_MODE_EXTEND) {
+    if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
+    return;
+  }
+  const int item = blockIdx.x / a.hq, h = blockIdx.x % a.hq;
+  if (item >= hdr->num_items) return;
+  const int4 it = a.ws.items[item];
+  const int r = it.x, q_begin = it.z, q_end = it.w;
+  const int L = a.ws.req_len[r], prefix = a.ws.req_prefix[r], q_start = a.ws.req_aux[r];
+  const int h_kv = h / (a.hq / a.hkv);
+  const int kv_end = prefix + q_end;                          // keys any row of this tile can see
+  const int n_kv = (kv_end + kTileKeys - 1) / kTileKeys;
+
+  if (tid == 0) {
+    mbar_init(sh.bar_q, 1);
+    for (int s = 0; s < kNumStages; ++s) {
+      mbar_init(sh.bar_k_full[s], 1);
+      mbar_init(sh.bar_v_full[s], 1);
+      mbar_init(sh.bar_kv_empty[s], 1);
+    }
+    mbar_init(sh.bar_s_full, 1);
+    mbar_init(sh.bar_s_free, 128);
+    mbar_init(sh.bar_p_full, 128);
+    mbar_init(sh.bar_o_done, 1);
+    mbar_init(sh.bar_drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
+
+  // bounded wait: false (and the CTA-wide abort flag set) if the barrier never completes
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+    }
+    *abort_flag = 1;
+    set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    return false;
+  };
+  // key tile j: keys [128 j, 128 j + 128) clipped to L
+  auto tile_keys = [&](int j) { return min(kTileKeys, L - j * kTileKeys); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
+      mbar_expect_tx(sh.bar_q, 2 * kChunkBytes);
+      const int row0 = q_start + q_begin;
+      tma_load_4d(base + kOffQ, &a.tm_q, 0, row0, 0, h, sh.bar_q);
+      tma_load_4d(base + kOffQ + kChunkBytes, &a.tm_q, 0, row0, 1, h, sh.bar_q);
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kNumStages;
+        if (j >= kNumStages && !wait(sh.bar_kv_empty[s], ((j / kNumStages) + 1) & 1)) break;
+        const int nk = tile_keys(j);
+        const int n_ops = (nk + a.box_rows - 1) / a.box_rows;
+        const uint32_t bytes = (uint32_t)n_ops * a.box_rows * 128u * 2u;
+        mbar_expect_tx(sh.bar_k_full[s], bytes);
+        mbar_expect_tx(sh.bar_v_full[s], bytes);
+        for (int o = 0; o < n_ops; ++o) {
+          const int key = j * kTileKeys + o * a.box_rows;       // first key of this box
+          int page = __ldg(table + (key >> a.page_shift));
+          long long slot = ((long long)page << a.page_shift) + (key & (a.page_size - 1));
+          if (page < 0 || slot + a.box_rows > a.num_slots) {    // keep the copy in bounds, flag the id
+            set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+            slot = 0;
+          }
+          for (int ch = 0; ch < 2; ++ch) {
+            const uint32_t off = ch * kChunkBytes + o * a.box_rows * 128;
+            tma_load_4d(base + kOffK + s * kTileBytes + off, &a.tm_k, 0, (int)slot, ch, h_kv, sh.bar_k_full[s]);
+            tma_load_4d(base + kOffV + s * kTileBytes + off, &a.tm_v, 0, (int)slot, ch, h_kv, sh.bar_v_full[s]);
+          }
+        }
+        issued = j + 1;
+      }
+      // copies still in flight when the CTA gives up: wait (bounded) until they land
+      if (*abort_flag) {
+        for (int j = max(0, issued - kNumStages); j < issued; ++j) {
+          const int s = j % kNumStages;
+          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_k_full[s], (j / kNumStages) & 1); ++i) {}
+          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_v_full[s], (j / kNumStages) & 1); ++i) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      auto issue_s = [&](int j) {
+        const uint32_t kb = base + kOffK + (j % kNumStages) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // 8 steps of 16 over d
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          tc_mma(tmem_s, smem_desc(base + kOffQ + off, 16), smem_desc(kb + off, 16), kIdescS, kk > 0);
+        }
+        tc_commit(sh.bar_s_full);
+      };
+      bool ok = wait(sh.bar_q, 0);
+      if (ok) ok = wait(sh.bar_k_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j % kNumStages;
+        if (j + 1 < n_kv) {
+          ok = wait(sh.bar_s_free, j & 1) && wait(sh.bar_k_full[(j + 1) % kNumStages], ((j + 1) / kNumStages) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        ok = wait(sh.bar_p_full, j & 1) && wait(sh.bar_v_full[s], (j / kNumStages) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const int nsteps = (tile_keys(j) + 15) / 16;           // 16-key steps that hold live keys
+        const uint32_t vb = base + kOffV + s * kTileBytes;
+        for (int kk = 0; kk < nsteps; ++kk) {
+          const uint32_t pa_off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;   // P: K-major over keys
+          tc_mma(tmem_o, smem_desc(base + kOffP + pa_off, 16), smem_desc(vb + kk * 16 * 128, kChunkBytes),
+                 kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(sh.bar_kv_empty[s]);
+        tc_commit(sh.bar_o_done);
+      }
+      // all issued tensor-core work has finished before TMEM is released
+      tc_commit(sh.bar_drain);
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_drain, 0); ++i) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int row = 32 * (warp & 3) + lane;                    // TMEM lane = query row of the tile
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int q_local = q_begin + row;
+    const bool row_valid = q_local < q_end && q_start + q_local < a.q_rows;   // never store past the O buffer
+    const int limit = row_valid ? prefix + q_local : L - 1;    // last visible key (inclusive)
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    float m_used = NEG_INF, l = 0.f;
+    uint8_t* prow = base_ptr + kOffP;
+    bool ok = true;
+    // tcgen05.ld/st are warp-collective: every wait result is made uniform across the warp
+    auto wwait = [&](uint32_t bar, uint32_t parity) { return __all_sync(0xffffffffu, wait(bar, parity)) != 0; };
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (!(ok = wwait(sh.bar_s_full, j & 1))) break;
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_off + 32 * c, sv[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sh.bar_s_free);
+      // scores in log2 units, causal mask on tiles that reach past this tile's first row
+      const int key0 = j * kTileKeys;
+      const bool diag = key0 + kTileKeys - 1 > prefix + q_begin || key0 + kTileKeys > L;
+      float mx = NEG_INF;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = __uint_as_float(sv[c][e]) * a.scale_log2;
+          if (diag && key0 + 32 * c + e > limit) x = NEG_INF;
+          sv[c][e] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      float alpha = 1.f;
+      if (m_used == NEG_INF) {
+        m_used = mx;
+      } else if (mx > m_used + kRescaleThreshold) {
+        alpha = ex2(m_used - mx);
+        m_used = mx;
+      }
+      if (j > 0 && !(ok = wwait(sh.bar_o_done, (j - 1) & 1))) break;  // PV(j-1) done: P and O are free
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {                      // rescale rows of O in TMEM
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tmem_o + lane_off + 32 * c, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tmem_o + lane_off + 32 * c, ov);
+        }
+        tmem_wait_st();
+        l *= alpha;
+      }
+      // P = 2^(x - m) as bf16, row-sum of the same rounded values, into the swizzled P tile
+      const float mu = m_used == NEG_INF ? 0.f : m_used;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {   // 16-byte units of 8 keys
+        uint32_t pk[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = (8 * u + 2 * q) >> 5, e = (8 * u + 2 * q) & 31;
+          const uint32_t w = pack_bf16x2(ex2(__uint_as_float(sv[c][e]) - mu), ex2(__uint_as_float(sv[c][e + 1]) - mu));
+          l += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          pk[q] = w;
+        }
+        const int chunk = u >> 3, unit = u & 7;
+        const uint32_t off = chunk * kChunkBytes + row * 128 + ((unit ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // the last tile: V rows past L inside the last 16-key step must read as zero
+      const int nk = tile_keys(j);
+      if (nk < kTileKeys && (nk & 15) && warp == 2) {
+        const int s = j % kNumStages;
+        if (!(ok = wwait(sh.bar_v_full[s], (j / kNumStages) & 1))) break;
+        const int z0 = nk, z1 = (nk + 15) & ~15;
+        uint8_t* vt = base_ptr + kOffV + s * kTileBytes;
+        for (int idx = lane; idx < (z1 - z0) * 16; idx += 32) {   // 16-byte units of rows z0..z1-1, both halves
+          const int rr = z0 + idx / 16, ch = (idx / 8) & 1, un = idx & 7;
+          *reinterpret_cast<uint4*>(vt + ch * kChunkBytes + rr * 128 + un * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(sh.bar_p_full);
+    }
+    if (ok) ok = wwait(sh.bar_o_done, (n_kv - 1) & 1);
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint16_t* orow = a.out + ((size_t)(q_start + q_local) * a.hq + h) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tmem_o + lane_off + 32 * c, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(ov[8 * g + 0]) * inv, __uint_as_float(ov[8 * g + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(ov[8 * g + 2]) * inv, __uint_as_float(ov[8 * g + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(ov[8 * g + 4]) * inv, __uint_as_float(ov[8 * g + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(ov[8 * g + 6]) * inv, __uint_as_float(ov[8 * g + 7]) * inv);
+          if (row_valid) *reinterpret_cast<uint4*>(orow + 32 * c + 8 * g) = w;
+        }
+      }
+      if (a.lse_out && row_valid)
+        a.lse_out[(size_t)(q_start + q_local) * a.hq + h] = l > 0.f ? (m_used + __log2f(l)) * kLn2 : NEG_INF;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host: tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows][heads][128] bf16 viewed as 4-D {64 d, rows, 2 halves of d, heads}; box {64, box_rows, 1, 1}
+bool encode_rows(CUtensorMap* tm, const void* ptr, int64_t rows, int heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64, (cuuint64_t)rows, 2, (cuuint64_t)heads};
+  const cuuint64_t strides[3] = {(cuuint64_t)heads * 256, 128, 256};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_extend(const ExtendArgs& in, cudaStream_t s) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  ExtendLaunch a;
+  const int box_rows = in.page_size < kTileKeys ? in.page_size : kTileKeys;
+  if (!encode_rows(&a.tm_q, in.q, in.q_rows, in.hq, 128) ||
+      !encode_rows(&a.tm_k, in.k_pool, in.num_slots, in.hkv, box_rows) ||
+      !encode_rows(&a.tm_v, in.v_pool, in.num_slots, in.hkv, box_rows))
+    return cudaErrorInvalidValue;
+  a.ws = in.ws;
+  a.page_table = in.page_table;
+  a.pt_pitch = in.pt_pitch;
+  a.num_slots = in.num_slots;
+  a.out = in.out;
+  a.lse_out = in.lse_out;
+  a.scale_log2 = in.scale_log2;
+  a.hq = in.hq;
+  a.hkv = in.hkv;
+  a.page_size = in.page_size;
+  a.page_shift = in.page_shift;
+  a.box_rows = box_rows;
+  a.max_items = in.max_items;
+  a.q_rows = in.q_rows;
+  extend_kernel<<<in.max_items * in.hq, kThreads, kSmemBytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pa
