@@ -264,7 +264,89 @@ class SageWorkload(DecodeWorkload):
         return nbytes, time.perf_counter() - t0, f"oracle.sage.sage_decode on requests 0..{r - 1} of layer 0"
 
 
+class ExtendWorkload(DecodeWorkload):
+    """plan + L layer calls of the causal paged extend, each layer with its own pools."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        import paged_kv_flashattention_split_b200 as pa
+        self.pa, self.spec, self.dev = pa, spec, device
+        self.batch = wl.make_batch(spec, device)
+        n_pools = spec.distinct_pools or spec.layers
+        self.pools = [wl.make_bf16_pools(spec, self.batch, l, device) for l in range(n_pools)]
+        self.total_q = int(self.batch.cu_seqlens_q[-1])
+        self.q = [wl.make_bf16_queries(spec, self.total_q, l, device) for l in range(spec.layers)]
+        self.out = [torch.empty_like(x) for x in self.q]
+        self.params = pa.make_params(pa.PA_MODE_EXTEND, spec.batch, spec.hq, spec.hkv, spec.head_dim,
+                                     spec.page_size, max_kv_len=self.batch.page_table.shape[1] * spec.page_size,
+                                     max_q_tokens=self.total_q)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        L = self.batch.seq_lens.cpu().tolist()
+        n = self.batch.new_lens.cpu().tolist()
+        pairs = sum(ni * (Li - ni) + ni * (ni + 1) // 2 for Li, ni in zip(L, n))   # unmasked (q, k) pairs
+        self.layer_flops = 4.0 * spec.head_dim * spec.hq * pairs
+        self.step_flops = self.layer_flops * spec.layers
+        self.layer_bytes = self.layer_flops          # the metric for this workload is TFLOP/s
+        self.step_bytes = self.step_flops
+        self.unit, self.scale = "TFLOP/s", 1e12
+        self.launches_per_step = 1 + spec.layers
+
+    def layer(self, l):
+        k, v = self.pool(l)
+        self.pa.attn_extend_paged(self.params, self.ws, self.q[l], k, v, self.batch.page_table,
+                                  self.spec.sm_scale, self.out[l])
+
+    def step_e2e(self):
+        self.batch.seq_lens.copy_(self.h_lens, non_blocking=True)
+        self.batch.cu_seqlens_q.copy_(self.h_cu, non_blocking=True)
+        self.batch.page_table.copy_(self.h_table, non_blocking=True)
+        self.pa.attn_plan(self.params, self.batch.seq_lens, self.batch.cu_seqlens_q, self.ws)
+        for l in range(self.spec.layers):
+            self.q[l].copy_(self.h_q[l], non_blocking=True)
+            self.layer(l)
+            self.h_out[l].copy_(self.out[l], non_blocking=True)
+
+    def step(self, layer_events=None):
+        self.pa.attn_plan(self.params, self.batch.seq_lens, self.batch.cu_seqlens_q, self.ws)
+        for l in range(self.spec.layers):
+            if layer_events is not None:
+                layer_events[l][0].record()
+            self.layer(l)
+            if layer_events is not None:
+                layer_events[l][1].record()
+
+    def setup_e2e(self):
+        super().setup_e2e()
+        self.h_cu = self.batch.cu_seqlens_q.cpu().pin_memory()
+        self.e2e_h2d += self.h_cu.numel() * 4
+
+    def oracle_sample(self, seconds=12.0):
+        from oracle import attention as oa
+        spec = self.spec
+        k, v = self.pool(0)
+        kb = k.view(torch.int16).cpu().numpy().view(np.uint16)
+        vb = v.view(torch.int16).cpu().numpy().view(np.uint16)
+        qb = self.q[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        cu = self.batch.cu_seqlens_q.cpu().numpy()
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        flops, r, h = 0.0, 0, 0
+        G = spec.hq // spec.hkv
+        t0 = time.perf_counter()
+        while (time.perf_counter() - t0) < seconds and r < spec.batch:
+            q0, q1 = int(cu[r]), int(cu[r + 1])
+            sub_cu = np.array([0, q1 - q0])
+            oa.extend(qb[q0:q1, h:h + 1], sub_cu, kb[:, h // G:h // G + 1], vb[:, h // G:h // G + 1],
+                      table[r:r + 1], lens[r:r + 1], spec.page_size, spec.sm_scale)
+            n = q1 - q0
+            flops += 4.0 * spec.head_dim * (n * (int(lens[r]) - n) + n * (n + 1) // 2)
+            h += 1
+            if h == spec.hq:
+                h, r = 0, r + 1
+        return flops, time.perf_counter() - t0, f"oracle.attention.extend, one query head at a time, {r * spec.hq + h} (request, head) pairs of layer 0"
+
+
 WORKLOADS = {
+    "extend_prefix": (3, ExtendWorkload),
     "sage_decode": (5, SageWorkload),
     "decode_llama3_8b": (2, DecodeWorkload),
     "decode_long_llama3_70b": (4, DecodeWorkload),
@@ -349,7 +431,8 @@ def main():
         total_ms = float(t.item())
         dist.barrier()
     ms_per_step = total_ms / args.steps
-    value = work.step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    scale = getattr(work, "scale", 1e9)
+    value = work.step_bytes * world / (ms_per_step * 1e-3) / scale
 
     # end to end through the public API with host buffers
     work.setup_e2e()
@@ -368,17 +451,23 @@ def main():
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    e2e_value = work.step_bytes * world / (e2e_ms * 1e-3) / 1e9
+    e2e_value = work.step_bytes * world / (e2e_ms * 1e-3) / scale
 
     avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
-    achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / 1e9
-    kernel_src = ("sage.cu", "common.cuh") if args.workload == "sage_decode" else ("decode.cu", "common.cuh")
+    achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / scale
+    kernel_src = {"sage_decode": ("sage.cu", "common.cuh"), "extend_prefix": ("extend.cu", "common.cuh")}.get(
+        args.workload, ("decode.cu", "common.cuh"))
     traffic = recorded_traffic(args.workload, source_hash(*kernel_src))
+    unit = getattr(work, "unit", "GB/s")
+    if unit == "TFLOP/s":
+        bound, peak, peak_note = "tensor", bf16_sus, peak_src + " (sustained bf16 dense, kernel timed inside a long step)"
+    else:
+        bound, peak, peak_note = "hbm", hbm_peak, peak_src
 
     line = {
         "metric": METRIC,
         "value": round(value, 1),
-        "unit": "GB/s",
+        "unit": unit,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": max(3, args.warmup),
@@ -393,26 +482,29 @@ def main():
             "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
             "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
-            "step": "attn_plan + %d x %s" % (spec.layers, "attn_decode_paged_sage" if args.workload == "sage_decode"
-                                              else "attn_decode_paged"),
+            "step": "attn_plan + %d x %s" % (spec.layers, {"sage_decode": "attn_decode_paged_sage",
+                                                            "extend_prefix": "attn_extend_paged"}.get(
+                                                               args.workload, "attn_decode_paged")),
             "l2": "inputs larger than L2 (each layer reads its own >1 GB pool)",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-            "kernel": ("sage_decode_kernel (one launch per attn_decode_paged_sage call)" if args.workload == "sage_decode"
-                       else "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)") + ", per-layer CUDA events",
-            "peak_source": peak_src,
+            "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": {"sage_decode": "sage_decode_kernel (one launch per attn_decode_paged_sage call)",
+                       "extend_prefix": "extend_kernel (one launch per attn_extend_paged call)"}.get(
+                           args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
+                      + ", per-layer CUDA events",
+            "peak_source": peak_note,
         },
-        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(work.e2e_h2d),
+        "e2e": {"value": round(e2e_value, 1), "unit": unit, "h2d_bytes_per_step": int(work.e2e_h2d),
                 "d2h_bytes_per_step": int(work.e2e_d2h), "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": work.launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nbytes, secs, sample = work.oracle_sample()
-        line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+        line["cpu_baseline"] = {"value": round(nbytes / secs / scale, 6), "unit": unit, "cores": blas_threads(),
                                 "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -73,7 +73,7 @@ CONFIGS = {
     2: Spec("decode_llama3_8b", 2, "decode", batch=64, len_lo=512, len_hi=8192, hq=32, hkv=8,
             page_size=1, pool_slots=600_000, layers=32),
     3: Spec("extend_prefix", 3, "extend", batch=8, len_lo=0, len_hi=4096, hq=32, hkv=8,
-            page_size=16, spare_pages=0.10, new_lo=128, new_hi=2048),
+            page_size=16, spare_pages=0.10, new_lo=128, new_hi=2048, layers=32),
     4: Spec("decode_long_llama3_70b", 4, "decode", batch=8, len_lo=131072, len_hi=131072, hq=64,
             hkv=8, page_size=64, layers=80, distinct_pools=8, peaked_frac=0.01, peaked_scale=8.0),
     5: Spec("sage_decode", 5, "sage", batch=32, len_lo=1024, len_hi=4096, hq=32, hkv=8,
