@@ -9,8 +9,10 @@
 //
 // One CTA per (query tile of 128 new tokens, query head), 6 warps:
 //   warp 0      producer: TMA loads of the Q tile once and of K/V key tiles
-//               (128 keys, i.e. 128 / P pages) into a 2-stage ring, each page
+//               (128 keys, i.e. 128 / P pages) into 2-stage rings, each page
 //               one box of a 4-D tensor map over the pool [slot][head][d];
+//               lane o reads box o's page id one tile ahead, and a K stage is
+//               refilled as soon as its S MMA is done (a V stage after its PV);
 //   warp 1      allocates TMEM and issues, from one thread,
 //                   S  = Q K^T   (tcgen05.mma kind::f16, M 128, N 128, S in TMEM)
 //                   O += P V     (P from shared memory, O accumulated in TMEM);
@@ -18,7 +20,8 @@
 //               128 scores with tcgen05.ld, applies the causal mask on the
 //               diagonal tiles, keeps a running max (rescaling O in TMEM only
 //               when the max grows by more than 2^8) and writes P (bf16) to
-//               shared memory in the MMA's swizzled layout; at the end it
+//               one of two shared-memory buffers in the MMA's swizzled layout,
+//               so P(j+1) is written while PV(j) reads P(j); at the end it
 //               normalises its O row and stores it.
 // The issue order S(0), then per tile S(j+1) before PV(j), lets the tensor
 // cores compute the next scores while the softmax works on the current ones.
@@ -49,8 +52,8 @@ constexpr float kRescaleThreshold = 8.f;         // log2 units
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTileBytes;
 constexpr int kOffV = kOffK + kNumStages * kTileBytes;
-constexpr int kOffP = kOffV + kNumStages * kTileBytes;
-constexpr int kOffBar = kOffP + kTileBytes;
+constexpr int kOffP = kOffV + kNumStages * kTileBytes;   // two P buffers
+constexpr int kOffBar = kOffP + 2 * kTileBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers, TMEM address, flags, alignment slack
 
 struct ExtendLaunch {
@@ -140,33 +143,32 @@ constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3
 constexpr uint32_t kIdescS = kIdescBase;                 // A (Q) and B (K) K-major
 constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);   // B (V) MN-major: d contiguous
 
-struct Shared {
-  uint32_t base;      // 1024-aligned shared address of the tile buffers
-  uint32_t bar_q, bar_k_full[kNumStages], bar_v_full[kNumStages], bar_kv_empty[kNumStages];
-  uint32_t bar_s_full, bar_s_free, bar_p_full, bar_o_done, bar_drain;
+// mbarriers, 8 bytes each, in this order after the tile buffers
+enum Bar {
+  B_Q = 0,
+  B_K_FULL = 1,                       // [2] K tile landed
+  B_V_FULL = B_K_FULL + kNumStages,   // [2] V tile landed
+  B_K_EMPTY = B_V_FULL + kNumStages,  // [2] S MMA done with the K stage
+  B_V_EMPTY = B_K_EMPTY + kNumStages, // [2] PV MMA done with the V stage
+  B_S_FULL = B_V_EMPTY + kNumStages,  // S in TMEM
+  B_S_FREE,                           // softmax has read S (128 arrivals)
+  B_P_FULL,                           // [2] P buffer written (128 arrivals)
+  B_P_FREE = B_P_FULL + 2,            // [2] PV MMA done with the P buffer
+  B_O_DONE = B_P_FREE + 2,            // a PV MMA finished (O stable)
+  B_DRAIN,
+  B_COUNT
 };
+static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
 
 __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_constant__ ExtendLaunch a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  Shared sh;
-  sh.base = base;
   const uint32_t bars = base + kOffBar;
-  sh.bar_q = bars;
-  for (int s = 0; s < kNumStages; ++s) {
-    sh.bar_k_full[s] = bars + 8 * (1 + s);
-    sh.bar_v_full[s] = bars + 8 * (1 + kNumStages + s);
-    sh.bar_kv_empty[s] = bars + 8 * (1 + 2 * kNumStages + s);
-  }
-  sh.bar_s_full = bars + 8 * (1 + 3 * kNumStages);
-  sh.bar_s_free = sh.bar_s_full + 8;
-  sh.bar_p_full = sh.bar_s_full + 16;
-  sh.bar_o_done = sh.bar_s_full + 24;
-  sh.bar_drain = sh.bar_s_full + 32;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffBar + 192);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBar + 200);
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffBar + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBar + 8 * B_COUNT + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   PlanHeader* hdr = a.ws.hdr;
@@ -184,17 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
   const int n_kv = (kv_end + kTileKeys - 1) / kTileKeys;
 
   if (tid == 0) {
-    mbar_init(sh.bar_q, 1);
-    for (int s = 0; s < kNumStages; ++s) {
-      mbar_init(sh.bar_k_full[s], 1);
-      mbar_init(sh.bar_v_full[s], 1);
-      mbar_init(sh.bar_kv_empty[s], 1);
-    }
-    mbar_init(sh.bar_s_full, 1);
-    mbar_init(sh.bar_s_free, 128);
-    mbar_init(sh.bar_p_full, 128);
-    mbar_init(sh.bar_o_done, 1);
-    mbar_init(sh.bar_drain, 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i == B_S_FREE || i == B_P_FULL || i == B_P_FULL + 1) ? 128 : 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -210,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
   const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
 
   // bounded wait: false (and the CTA-wide abort flag set) if the barrier never completes
-  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
-      if (mbar_try_wait(bar, parity)) return true;
+      if (mbar_try_wait(b, parity)) return true;
       if (*abort_flag) return false;
     }
     *abort_flag = 1;
@@ -221,91 +213,114 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
   };
   // key tile j: keys [128 j, 128 j + 128) clipped to L
   auto tile_keys = [&](int j) { return min(kTileKeys, L - j * kTileKeys); };
+  // parity of the completion of a 2-deep ring barrier that tile j waits for / releases
+  auto ring_parity = [](int j) -> uint32_t { return (uint32_t)(j >> 1) & 1u; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (whole warp)
+    const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
     if (lane == 0) {
-      const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
-      mbar_expect_tx(sh.bar_q, 2 * kChunkBytes);
+      mbar_expect_tx(bar(B_Q), 2 * kChunkBytes);
       const int row0 = q_start + q_begin;
-      tma_load_4d(base + kOffQ, &a.tm_q, 0, row0, 0, h, sh.bar_q);
-      tma_load_4d(base + kOffQ + kChunkBytes, &a.tm_q, 0, row0, 1, h, sh.bar_q);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % kNumStages;
-        if (j >= kNumStages && !wait(sh.bar_kv_empty[s], ((j / kNumStages) + 1) & 1)) break;
-        const int nk = tile_keys(j);
-        const int n_ops = (nk + a.box_rows - 1) / a.box_rows;
-        const uint32_t bytes = (uint32_t)n_ops * a.box_rows * 128u * 2u;
-        mbar_expect_tx(sh.bar_k_full[s], bytes);
-        mbar_expect_tx(sh.bar_v_full[s], bytes);
-        for (int o = 0; o < n_ops; ++o) {
-          const int key = j * kTileKeys + o * a.box_rows;       // first key of this box
-          int page = __ldg(table + (key >> a.page_shift));
-          long long slot = ((long long)page << a.page_shift) + (key & (a.page_size - 1));
-          if (page < 0 || slot + a.box_rows > a.num_slots) {    // keep the copy in bounds, flag the id
-            set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-            slot = 0;
-          }
-          for (int ch = 0; ch < 2; ++ch) {
-            const uint32_t off = ch * kChunkBytes + o * a.box_rows * 128;
-            tma_load_4d(base + kOffK + s * kTileBytes + off, &a.tm_k, 0, (int)slot, ch, h_kv, sh.bar_k_full[s]);
-            tma_load_4d(base + kOffV + s * kTileBytes + off, &a.tm_v, 0, (int)slot, ch, h_kv, sh.bar_v_full[s]);
-          }
-        }
-        issued = j + 1;
+      tma_load_4d(base + kOffQ, &a.tm_q, 0, row0, 0, h, bar(B_Q));
+      tma_load_4d(base + kOffQ + kChunkBytes, &a.tm_q, 0, row0, 1, h, bar(B_Q));
+    }
+    // lane o owns box o of each tile: its slot comes from one table read, issued before the waits
+    auto box_slot = [&](int j) -> int {
+      const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
+      if (lane >= n_ops) return -1;
+      const int key = j * kTileKeys + lane * a.box_rows;
+      const int page = __ldg(table + (key >> a.page_shift));
+      const long long slot = ((long long)page << a.page_shift) + (key & (a.page_size - 1));
+      if (page < 0 || slot + a.box_rows > a.num_slots) {       // keep the copy in bounds, flag the id
+        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+        return 0;
       }
-      // copies still in flight when the CTA gives up: wait (bounded) until they land
-      if (*abort_flag) {
-        for (int j = max(0, issued - kNumStages); j < issued; ++j) {
-          const int s = j % kNumStages;
-          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_k_full[s], (j / kNumStages) & 1); ++i) {}
-          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_v_full[s], (j / kNumStages) & 1); ++i) {}
-        }
+      return (int)slot;
+    };
+    int next_slot = box_slot(0);
+    int issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      const int slot = next_slot;
+      const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
+      const uint32_t bytes = (uint32_t)n_ops * a.box_rows * 128u * 2u;
+      const uint32_t off = (uint32_t)lane * a.box_rows * 128u;
+      // K stage s is free once S(j-2) is done
+      bool ok = true;
+      if (lane == 0) {
+        ok = j < kNumStages || wait(bar(B_K_EMPTY + s), ring_parity(j) ^ 1u);
+        if (ok) mbar_expect_tx(bar(B_K_FULL + s), bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane < n_ops)
+        for (int ch = 0; ch < 2; ++ch)
+          tma_load_4d(base + kOffK + s * kTileBytes + ch * kChunkBytes + off, &a.tm_k, 0, slot, ch, h_kv,
+                      bar(B_K_FULL + s));
+      // V stage s is free once PV(j-2) is done
+      if (lane == 0) {
+        ok = j < kNumStages || wait(bar(B_V_EMPTY + s), ring_parity(j) ^ 1u);
+        if (ok) mbar_expect_tx(bar(B_V_FULL + s), bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane < n_ops)
+        for (int ch = 0; ch < 2; ++ch)
+          tma_load_4d(base + kOffV + s * kTileBytes + ch * kChunkBytes + off, &a.tm_v, 0, slot, ch, h_kv,
+                      bar(B_V_FULL + s));
+      issued = j + 1;
+      if (j + 1 < n_kv) next_slot = box_slot(j + 1);
+    }
+    // copies still in flight when the CTA gives up: wait (bounded) until they land
+    if (lane == 0 && *abort_flag) {
+      for (int j = max(0, issued - kNumStages); j < issued; ++j) {
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_K_FULL + (j & 1)), ring_parity(j)); ++i) {}
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_V_FULL + (j & 1)), ring_parity(j)); ++i) {}
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       auto issue_s = [&](int j) {
-        const uint32_t kb = base + kOffK + (j % kNumStages) * kTileBytes;
+        const uint32_t kb = base + kOffK + (j & 1) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // 8 steps of 16 over d
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
           tc_mma(tmem_s, smem_desc(base + kOffQ + off, 16), smem_desc(kb + off, 16), kIdescS, kk > 0);
         }
-        tc_commit(sh.bar_s_full);
+        tc_commit(bar(B_S_FULL));
+        tc_commit(bar(B_K_EMPTY + (j & 1)));
       };
-      bool ok = wait(sh.bar_q, 0);
-      if (ok) ok = wait(sh.bar_k_full[0], 0);
+      bool ok = wait(bar(B_Q), 0) && wait(bar(B_K_FULL), 0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % kNumStages;
+        const int s = j & 1;
         if (j + 1 < n_kv) {
-          ok = wait(sh.bar_s_free, j & 1) && wait(sh.bar_k_full[(j + 1) % kNumStages], ((j + 1) / kNumStages) & 1);
+          ok = wait(bar(B_S_FREE), j & 1) && wait(bar(B_K_FULL + ((j + 1) & 1)), ring_parity(j + 1));
           if (!ok) break;
           tc_fence_after();
           issue_s(j + 1);
         }
-        ok = wait(sh.bar_p_full, j & 1) && wait(sh.bar_v_full[s], (j / kNumStages) & 1);
+        ok = wait(bar(B_P_FULL + s), ring_parity(j)) && wait(bar(B_V_FULL + s), ring_parity(j));
         if (!ok) break;
         tc_fence_after();
         const int nsteps = (tile_keys(j) + 15) / 16;           // 16-key steps that hold live keys
         const uint32_t vb = base + kOffV + s * kTileBytes;
+        const uint32_t pb = base + kOffP + s * kTileBytes;
         for (int kk = 0; kk < nsteps; ++kk) {
           const uint32_t pa_off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;   // P: K-major over keys
-          tc_mma(tmem_o, smem_desc(base + kOffP + pa_off, 16), smem_desc(vb + kk * 16 * 128, kChunkBytes),
-                 kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem_o, smem_desc(pb + pa_off, 16), smem_desc(vb + kk * 16 * 128, kChunkBytes), kIdescPV,
+                 (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(sh.bar_kv_empty[s]);
-        tc_commit(sh.bar_o_done);
+        tc_commit(bar(B_V_EMPTY + s));
+        tc_commit(bar(B_P_FREE + s));
+        tc_commit(bar(B_O_DONE));
       }
       // all issued tensor-core work has finished before TMEM is released
-      tc_commit(sh.bar_drain);
-      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(sh.bar_drain, 0); ++i) {}
+      tc_commit(bar(B_DRAIN));
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++i) {}
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroup
@@ -315,33 +330,40 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
     const bool row_valid = q_local < q_end && q_start + q_local < a.q_rows;   // never store past the O buffer
     const int limit = row_valid ? prefix + q_local : L - 1;    // last visible key (inclusive)
     const float NEG_INF = -__int_as_float(0x7f800000);
+    const float c = a.scale_log2;                              // > 0: the max commutes with the scale
     float m_used = NEG_INF, l = 0.f;
-    uint8_t* prow = base_ptr + kOffP;
     bool ok = true;
     // tcgen05.ld/st are warp-collective: every wait result is made uniform across the warp
-    auto wwait = [&](uint32_t bar, uint32_t parity) { return __all_sync(0xffffffffu, wait(bar, parity)) != 0; };
+    auto wwait = [&](uint32_t b, uint32_t parity) { return __all_sync(0xffffffffu, wait(b, parity)) != 0; };
     for (int j = 0; j < n_kv && ok; ++j) {
-      if (!(ok = wwait(sh.bar_s_full, j & 1))) break;
+      const int s = j & 1;
+      if (!(ok = wwait(bar(B_S_FULL), j & 1))) break;
       tc_fence_after();
       uint32_t sv[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_off + 32 * c, sv[c]);
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem_s + lane_off + 32 * cc, sv[cc]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(sh.bar_s_free);
-      // scores in log2 units, causal mask on tiles that reach past this tile's first row
+      mbar_arrive(bar(B_S_FREE));
+      // raw-score row max, causal mask on tiles that reach past this tile's first row
       const int key0 = j * kTileKeys;
       const bool diag = key0 + kTileKeys - 1 > prefix + q_begin || key0 + kTileKeys > L;
       float mx = NEG_INF;
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(sv[c][e]) * a.scale_log2;
-          if (diag && key0 + 32 * c + e > limit) x = NEG_INF;
-          sv[c][e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+          for (int e = 0; e < 32; ++e) {
+            if (key0 + 32 * cc + e > limit) sv[cc][e] = __float_as_uint(NEG_INF);
+            mx = fmaxf(mx, __uint_as_float(sv[cc][e]));
+          }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[cc][e]));
+      }
+      mx *= c;                                                  // log2 units
       float alpha = 1.f;
       if (m_used == NEG_INF) {
         m_used = mx;
@@ -349,42 +371,48 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
         alpha = ex2(m_used - mx);
         m_used = mx;
       }
-      if (j > 0 && !(ok = wwait(sh.bar_o_done, (j - 1) & 1))) break;  // PV(j-1) done: P and O are free
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {                      // rescale rows of O in TMEM
+      // P = 2^(c s - m) as bf16 (overwriting the scores), row sum of the same rounded values
+      const float neg_m = m_used == NEG_INF ? 0.f : -m_used;
+      float lt = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[cc][e]), c, neg_m)),
+                                         ex2(fmaf(__uint_as_float(sv[cc][e + 1]), c, neg_m)));
+          lt += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          sv[cc][e >> 1] = w;                                   // packed pairs in the low half of each row
+        }
+      if (j >= 2 && !(ok = wwait(bar(B_P_FREE + s), ring_parity(j) ^ 1u))) break;   // PV(j-2) released buffer s
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {                                   // rescale rows of O in TMEM
+        if (j > 0 && !(ok = wwait(bar(B_O_DONE), (j - 1) & 1))) break;              // PV(j-1) done: O stable
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t ov[32];
-          tmem_ld32(tmem_o + lane_off + 32 * c, ov);
+          tmem_ld32(tmem_o + lane_off + 32 * cc, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tmem_o + lane_off + 32 * c, ov);
+          tmem_st32(tmem_o + lane_off + 32 * cc, ov);
         }
         tmem_wait_st();
-        l *= alpha;
       }
-      // P = 2^(x - m) as bf16, row-sum of the same rounded values, into the swizzled P tile
-      const float mu = m_used == NEG_INF ? 0.f : m_used;
+      l = l * alpha + lt;
+      uint8_t* prow = base_ptr + kOffP + s * kTileBytes;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {   // 16-byte units of 8 keys
-        uint32_t pk[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = (8 * u + 2 * q) >> 5, e = (8 * u + 2 * q) & 31;
-          const uint32_t w = pack_bf16x2(ex2(__uint_as_float(sv[c][e]) - mu), ex2(__uint_as_float(sv[c][e + 1]) - mu));
-          l += bf16lo_to_f32(w) + bf16hi_to_f32(w);
-          pk[q] = w;
-        }
+      for (int u = 0; u < 16; ++u) {   // 16-byte units of 8 keys; pairs 4u .. 4u+3 of the row
+        const int p0 = 4 * u;          // pair index: row element 2 p0
+        const uint32_t w0 = sv[p0 >> 4][p0 & 15], w1 = sv[(p0 + 1) >> 4][(p0 + 1) & 15];
+        const uint32_t w2 = sv[(p0 + 2) >> 4][(p0 + 2) & 15], w3 = sv[(p0 + 3) >> 4][(p0 + 3) & 15];
         const int chunk = u >> 3, unit = u & 7;
         const uint32_t off = chunk * kChunkBytes + row * 128 + ((unit ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(w0, w1, w2, w3);
       }
       // the last tile: V rows past L inside the last 16-key step must read as zero
       const int nk = tile_keys(j);
       if (nk < kTileKeys && (nk & 15) && warp == 2) {
-        const int s = j % kNumStages;
-        if (!(ok = wwait(sh.bar_v_full[s], (j / kNumStages) & 1))) break;
+        if (!(ok = wwait(bar(B_V_FULL + s), ring_parity(j)))) break;
         const int z0 = nk, z1 = (nk + 15) & ~15;
         uint8_t* vt = base_ptr + kOffV + s * kTileBytes;
         for (int idx = lane; idx < (z1 - z0) * 16; idx += 32) {   // 16-byte units of rows z0..z1-1, both halves
@@ -394,17 +422,17 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       }
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(sh.bar_p_full);
+      mbar_arrive(bar(B_P_FULL + s));
     }
-    if (ok) ok = wwait(sh.bar_o_done, (n_kv - 1) & 1);
+    if (ok) ok = wwait(bar(B_O_DONE), (n_kv - 1) & 1);
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint16_t* orow = a.out + ((size_t)(q_start + q_local) * a.hq + h) * kHeadDim;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t ov[32];
-        tmem_ld32(tmem_o + lane_off + 32 * c, ov);
+        tmem_ld32(tmem_o + lane_off + 32 * cc, ov);
         tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -413,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
           w.y = pack_bf16x2(__uint_as_float(ov[8 * g + 2]) * inv, __uint_as_float(ov[8 * g + 3]) * inv);
           w.z = pack_bf16x2(__uint_as_float(ov[8 * g + 4]) * inv, __uint_as_float(ov[8 * g + 5]) * inv);
           w.w = pack_bf16x2(__uint_as_float(ov[8 * g + 6]) * inv, __uint_as_float(ov[8 * g + 7]) * inv);
-          if (row_valid) *reinterpret_cast<uint4*>(orow + 32 * c + 8 * g) = w;
+          if (row_valid) *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * g) = w;
         }
       }
       if (a.lse_out && row_valid)
