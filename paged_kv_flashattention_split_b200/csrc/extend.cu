@@ -135,6 +135,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n"
+               ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+// stores v[0..15] (the packed half of a 32-register row)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// D (TMEM) += A (TMEM, K-major bf16 pairs) x B (shared memory descriptor)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
@@ -348,21 +374,23 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       // raw-score row max, causal mask on tiles that reach past this tile's first row
       const int key0 = j * kTileKeys;
       const bool diag = key0 + kTileKeys - 1 > prefix + q_begin || key0 + kTileKeys > L;
-      float mx = NEG_INF;
       if (diag) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 32; ++e)
             if (key0 + 32 * cc + e > limit) sv[cc][e] = __float_as_uint(NEG_INF);
-            mx = fmaxf(mx, __uint_as_float(sv[cc][e]));
-          }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[cc][e]));
       }
+      // 8 independent partial maxima keep the reduction off a 128-long dependency chain
+      float mxp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mxp[i] = NEG_INF;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(sv[cc][e]));
+      float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       mx *= c;                                                  // log2 units
       float alpha = 1.f;
       if (m_used == NEG_INF) {
@@ -373,16 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       }
       // P = 2^(c s - m) as bf16 (overwriting the scores), row sum of the same rounded values
       const float neg_m = m_used == NEG_INF ? 0.f : -m_used;
-      float lt = 0.f;
+      float ltp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ltp[i] = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const uint32_t w = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[cc][e]), c, neg_m)),
                                          ex2(fmaf(__uint_as_float(sv[cc][e + 1]), c, neg_m)));
-          lt += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          ltp[(e >> 1) & 7] += bf16lo_to_f32(w) + bf16hi_to_f32(w);
           sv[cc][e >> 1] = w;                                   // packed pairs in the low half of each row
         }
+      const float lt = ((ltp[0] + ltp[1]) + (ltp[2] + ltp[3])) + ((ltp[4] + ltp[5]) + (ltp[6] + ltp[7]));
       if (j >= 2 && !(ok = wwait(bar(B_P_FREE + s), ring_parity(j) ^ 1u))) break;   // PV(j-2) released buffer s
       if (__any_sync(0xffffffffu, alpha != 1.f)) {                                   // rescale rows of O in TMEM
         if (j > 0 && !(ok = wwait(bar(B_O_DONE), (j - 1) & 1))) break;              // PV(j-1) done: O stable
@@ -456,6 +487,327 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
   }
 }
 
+
+// ======================================================================================
+// Two query tiles per CTA: heads h0 = 2 hp and h1 = 2 hp + 1 of the same KV group share
+// every K/V tile.  Warp 0 loads, warp 1 issues the MMAs, warps 2-5 and 6-9 are one
+// softmax warpgroup per query tile.  TMEM (512 columns): S0 [0,128), S1 [128,256),
+// O0 [256,384), O1 [384,512); P_t (bf16, two per 32-bit column) is written over the
+// first 64 columns of S_t once S_t has been read, and PV_t takes A from TMEM.  The
+// tensor cores execute one thread's MMAs in issue order, so S_t(j+1), issued after
+// PV_t(j), never overwrites P_t(j) before it has been read; and S_t(j) complete
+// implies PV_t(j-1) complete, so O_t is stable whenever softmax t reads S_t.
+// While one warpgroup runs its softmax the tensor cores work on the other tile.
+constexpr int kPairThreads = 320;
+constexpr int kPairOffQ = 0;                                   // Q0, Q1
+constexpr int kPairOffK = 2 * kTileBytes;
+constexpr int kPairOffV = kPairOffK + kNumStages * kTileBytes;
+constexpr int kPairOffBar = kPairOffV + kNumStages * kTileBytes;
+constexpr int kPairSmemBytes = kPairOffBar + 256 + 1024;
+constexpr uint32_t kPairTmemCols = 512;
+
+enum PairBar {
+  PB_Q = 0,
+  PB_K_FULL = 1,
+  PB_V_FULL = PB_K_FULL + kNumStages,
+  PB_K_EMPTY = PB_V_FULL + kNumStages,
+  PB_V_EMPTY = PB_K_EMPTY + kNumStages,
+  PB_S_FULL = PB_V_EMPTY + kNumStages,  // [2] per query tile
+  PB_P_FULL = PB_S_FULL + 2,            // [2] per query tile, 128 arrivals
+  PB_O_DONE = PB_P_FULL + 2,            // [2] per query tile
+  PB_DRAIN = PB_O_DONE + 2,
+  PB_COUNT
+};
+static_assert(PB_COUNT * 8 + 16 <= 256, "barrier area");
+
+__global__ void __launch_bounds__(kPairThreads, 1) extend_pair_kernel(const __grid_constant__ ExtendLaunch a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bars = base + kPairOffBar;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kPairOffBar + 8 * PB_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kPairOffBar + 8 * PB_COUNT + 8);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  PlanHeader* hdr = a.ws.hdr;
+  if (hdr->magic != kMagic || hdr->mode != PA_MODE_EXTEND) {
+    if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
+    return;
+  }
+  const int pairs = a.hq / 2;
+  const int item = blockIdx.x / pairs, hp = blockIdx.x % pairs;
+  if (item >= hdr->num_items) return;
+  const int4 it = a.ws.items[item];
+  const int r = it.x, q_begin = it.z, q_end = it.w;
+  const int L = a.ws.req_len[r], prefix = a.ws.req_prefix[r], q_start = a.ws.req_aux[r];
+  const int h0 = 2 * hp;
+  const int h_kv = h0 / (a.hq / a.hkv);
+  const int kv_end = prefix + q_end;
+  const int n_kv = (kv_end + kTileKeys - 1) / kTileKeys;
+
+  if (tid == 0) {
+    for (int i = 0; i < PB_COUNT; ++i) mbar_init(bar(i), (i == PB_P_FULL || i == PB_P_FULL + 1) ? 128 : 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+                 ::"r"(smem_u32(tmem_slot)), "r"(kPairTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+      if (mbar_try_wait(b, parity)) return true;
+      if (*abort_flag) return false;
+    }
+    *abort_flag = 1;
+    set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    return false;
+  };
+  auto tile_keys = [&](int j) { return min(kTileKeys, L - j * kTileKeys); };
+  auto ring_parity = [](int j) -> uint32_t { return (uint32_t)(j >> 1) & 1u; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (whole warp)
+    const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
+    if (lane == 0) {
+      mbar_expect_tx(bar(PB_Q), 4 * kChunkBytes);
+      const int row0 = q_start + q_begin;
+      for (int t = 0; t < 2; ++t)
+        for (int ch = 0; ch < 2; ++ch)
+          tma_load_4d(base + kPairOffQ + t * kTileBytes + ch * kChunkBytes, &a.tm_q, 0, row0, ch, h0 + t, bar(PB_Q));
+    }
+    auto box_slot = [&](int j) -> int {
+      const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
+      if (lane >= n_ops) return -1;
+      const int key = j * kTileKeys + lane * a.box_rows;
+      const int page = __ldg(table + (key >> a.page_shift));
+      const long long slot = ((long long)page << a.page_shift) + (key & (a.page_size - 1));
+      if (page < 0 || slot + a.box_rows > a.num_slots) {
+        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+        return 0;
+      }
+      return (int)slot;
+    };
+    int next_slot = box_slot(0);
+    int issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      const int slot = next_slot;
+      const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
+      const uint32_t bytes = (uint32_t)n_ops * a.box_rows * 128u * 2u;
+      const uint32_t off = (uint32_t)lane * a.box_rows * 128u;
+      bool ok = true;
+      if (lane == 0) {
+        ok = j < kNumStages || wait(bar(PB_K_EMPTY + s), ring_parity(j) ^ 1u);
+        if (ok) mbar_expect_tx(bar(PB_K_FULL + s), bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane < n_ops)
+        for (int ch = 0; ch < 2; ++ch)
+          tma_load_4d(base + kPairOffK + s * kTileBytes + ch * kChunkBytes + off, &a.tm_k, 0, slot, ch, h_kv,
+                      bar(PB_K_FULL + s));
+      if (lane == 0) {
+        ok = j < kNumStages || wait(bar(PB_V_EMPTY + s), ring_parity(j) ^ 1u);
+        if (ok) mbar_expect_tx(bar(PB_V_FULL + s), bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane < n_ops)
+        for (int ch = 0; ch < 2; ++ch)
+          tma_load_4d(base + kPairOffV + s * kTileBytes + ch * kChunkBytes + off, &a.tm_v, 0, slot, ch, h_kv,
+                      bar(PB_V_FULL + s));
+      issued = j + 1;
+      if (j + 1 < n_kv) next_slot = box_slot(j + 1);
+    }
+    if (lane == 0 && *abort_flag) {
+      for (int j = max(0, issued - kNumStages); j < issued; ++j) {
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(PB_K_FULL + (j & 1)), ring_parity(j)); ++i) {}
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(PB_V_FULL + (j & 1)), ring_parity(j)); ++i) {}
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      auto issue_s = [&](int t, int j) {            // S_t = Q_t K(j)^T
+        const uint32_t qb = base + kPairOffQ + t * kTileBytes;
+        const uint32_t kb = base + kPairOffK + (j & 1) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          tc_mma(tmem + 128 * t, smem_desc(qb + off, 16), smem_desc(kb + off, 16), kIdescS, kk > 0);
+        }
+        tc_commit(bar(PB_S_FULL + t));
+      };
+      auto issue_pv = [&](int t, int j) {           // O_t += P_t V(j), P_t from TMEM
+        const int nsteps = (tile_keys(j) + 15) / 16;
+        const uint32_t vb = base + kPairOffV + (j & 1) * kTileBytes;
+        for (int kk = 0; kk < nsteps; ++kk)
+          tc_mma_ts(tmem + 256 + 128 * t, tmem + 128 * t + 8 * kk, smem_desc(vb + kk * 16 * 128, kChunkBytes),
+                    kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(PB_O_DONE + t));
+      };
+      bool ok = wait(bar(PB_Q), 0) && wait(bar(PB_K_FULL), 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc_commit(bar(PB_K_EMPTY));
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1, s1 = (j + 1) & 1;
+        const bool more = j + 1 < n_kv;
+        if (!(ok = wait(bar(PB_V_FULL + s), ring_parity(j)) && wait(bar(PB_P_FULL), j & 1))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!(ok = wait(bar(PB_K_FULL + s1), ring_parity(j + 1)))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = wait(bar(PB_P_FULL + 1), j & 1))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        tc_commit(bar(PB_V_EMPTY + s));
+        if (more) {
+          issue_s(1, j + 1);
+          tc_commit(bar(PB_K_EMPTY + s1));
+        }
+      }
+      tc_commit(bar(PB_DRAIN));
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(PB_DRAIN), 0); ++i) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 2) >> 2;                             // query tile of this warpgroup
+    const int h = h0 + t;
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tmem_s = tmem + 128 * t, tmem_o = tmem + 256 + 128 * t;
+    const int q_local = q_begin + row;
+    const bool row_valid = q_local < q_end && q_start + q_local < a.q_rows;
+    const int limit = row_valid ? prefix + q_local : L - 1;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    const float c = a.scale_log2;
+    float m_used = NEG_INF, l = 0.f;
+    bool ok = true;
+    auto wwait = [&](uint32_t b, uint32_t parity) { return __all_sync(0xffffffffu, wait(b, parity)) != 0; };
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int s = j & 1;
+      if (!(ok = wwait(bar(PB_S_FULL + t), j & 1))) break;
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem_s + lane_off + 32 * cc, sv[cc]);
+      tmem_wait_ld();
+      const int key0 = j * kTileKeys;
+      const bool diag = key0 + kTileKeys - 1 > prefix + q_begin || key0 + kTileKeys > L;
+      if (diag) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (key0 + 32 * cc + e > limit) sv[cc][e] = __float_as_uint(NEG_INF);
+      }
+      float mxp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mxp[i] = NEG_INF;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(sv[cc][e]));
+      float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+      mx *= c;
+      float alpha = 1.f;
+      if (m_used == NEG_INF) {
+        m_used = mx;
+      } else if (mx > m_used + kRescaleThreshold) {
+        alpha = ex2(m_used - mx);
+        m_used = mx;
+      }
+      const float neg_m = m_used == NEG_INF ? 0.f : -m_used;
+      float ltp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ltp[i] = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[cc][e]), c, neg_m)),
+                                         ex2(fmaf(__uint_as_float(sv[cc][e + 1]), c, neg_m)));
+          ltp[(e >> 1) & 7] += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          sv[cc][e >> 1] = w;
+        }
+      const float lt = ((ltp[0] + ltp[1]) + (ltp[2] + ltp[3])) + ((ltp[4] + ltp[5]) + (ltp[6] + ltp[7]));
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {             // O_t is stable: PV_t(j-1) finished before S_t(j)
+#pragma unroll 1
+        for (int cc = 0; cc < 16; ++cc) {                        // 8 columns at a time keeps registers low
+          uint32_t ov[8];
+          tmem_ld8(tmem_o + lane_off + 8 * cc, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st8(tmem_o + lane_off + 8 * cc, ov);
+        }
+      }
+      l = l * alpha + lt;
+      // P_t over the first 64 columns of S_t: column p holds keys 2p (low half) and 2p + 1
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_st16(tmem_s + lane_off + 16 * cc, sv[cc]);
+      tmem_wait_st();
+      const int nk = tile_keys(j);
+      if (t == 0 && nk < kTileKeys && (nk & 15) && warp == 2) {   // V rows past L in the last 16-key step
+        if (!(ok = wwait(bar(PB_V_FULL + s), ring_parity(j)))) break;
+        const int z0 = nk, z1 = (nk + 15) & ~15;
+        uint8_t* vt = base_ptr + kPairOffV + s * kTileBytes;
+        for (int idx = lane; idx < (z1 - z0) * 16; idx += 32) {
+          const int rr = z0 + idx / 16, ch = (idx / 8) & 1, un = idx & 7;
+          *reinterpret_cast<uint4*>(vt + ch * kChunkBytes + rr * 128 + un * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(PB_P_FULL + t));
+    }
+    if (ok) ok = wwait(bar(PB_O_DONE + t), (n_kv - 1) & 1);
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint16_t* orow = a.out + ((size_t)(q_start + q_local) * a.hq + h) * kHeadDim;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(tmem_o + lane_off + 32 * cc, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(ov[8 * g + 0]) * inv, __uint_as_float(ov[8 * g + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(ov[8 * g + 2]) * inv, __uint_as_float(ov[8 * g + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(ov[8 * g + 4]) * inv, __uint_as_float(ov[8 * g + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(ov[8 * g + 6]) * inv, __uint_as_float(ov[8 * g + 7]) * inv);
+          if (row_valid) *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * g) = w;
+        }
+      }
+      if (a.lse_out && row_valid)
+        a.lse_out[(size_t)(q_start + q_local) * a.hq + h] = l > 0.f ? (m_used + __log2f(l)) * kLn2 : NEG_INF;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kPairTmemCols) : "memory");
+  }
+}
+
 // ---------------------------------------------------------------- host: tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -518,7 +870,18 @@ cudaError_t launch_extend(const ExtendArgs& in, cudaStream_t s) {
   a.box_rows = box_rows;
   a.max_items = in.max_items;
   a.q_rows = in.q_rows;
-  extend_kernel<<<in.max_items * in.hq, kThreads, kSmemBytes, s>>>(a);
+  if ((in.hq / in.hkv) % 2 == 0) {   // two heads of one KV group per CTA
+    static bool pair_attr[64] = {};
+    if (dev < 64 && !pair_attr[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(extend_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kPairSmemBytes);
+      if (e != cudaSuccess) return e;
+      pair_attr[dev] = true;
+    }
+    extend_pair_kernel<<<in.max_items * (in.hq / 2), kPairThreads, kPairSmemBytes, s>>>(a);
+  } else {
+    extend_kernel<<<in.max_items * in.hq, kThreads, kSmemBytes, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
