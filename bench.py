@@ -132,6 +132,32 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def init_ranks(world: int, local: int, backend: str):
+    """One process per GPU under torchrun: join the process group (None when alone)."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return dist
+
+
+def max_over_ranks(dist, value: float, device="cpu") -> float:
+    """The job's time is the slowest rank's device time."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_per_step: float, scale: float) -> float:
+    """Whole-job throughput: every rank's units over the max-over-ranks step time."""
+    return units_per_rank * world / (ms_per_step * 1e-3) / scale
+
+
 # --------------------------------------------------------------------------- decode workload
 
 class DecodeWorkload:
@@ -373,12 +399,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dist = init_ranks(world, local, "gloo" if args.impl == "reference" else "nccl")
 
     cfg_id, cls = WORKLOADS[args.workload]
     spec = wl.CONFIGS[cfg_id]
@@ -424,15 +445,12 @@ def main():
         torch.cuda.synchronize()
         # per-layer durations of the last step (the events are re-recorded every step)
         layer_ms = [a.elapsed_time(b) for a, b in layer_events]
-    total_ms = start.elapsed_time(end)
+    total_ms = max_over_ranks(dist, start.elapsed_time(end), dev)
     if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
     ms_per_step = total_ms / args.steps
     scale = getattr(work, "scale", 1e9)
-    value = work.step_bytes * world / (ms_per_step * 1e-3) / scale
+    value = job_throughput(work.step_bytes, world, ms_per_step, scale)
 
     # end to end through the public API with host buffers
     work.setup_e2e()
@@ -446,12 +464,8 @@ def main():
         work.step_e2e()
     e_end.record()
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = work.step_bytes * world / (e2e_ms * 1e-3) / scale
+    e2e_ms = max_over_ranks(dist, e_start.elapsed_time(e_end) / e_steps, dev)
+    e2e_value = job_throughput(work.step_bytes, world, e2e_ms, scale)
 
     avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
     achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / scale
@@ -514,42 +528,73 @@ def main():
 
 
 def run_reference(args, spec, cls):
-    """The oracle as it stands, on the host cores, on a bounded sample per step."""
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload per step."""
     from oracle import attention as oa
+    from oracle import sage as osg
     batch = wl.make_batch(spec, "cpu")
-    n_pools = 1
-    k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
-    q = wl.make_bf16_queries(spec, spec.batch, 0, "cpu")
-    kb = k.view(torch.int16).numpy().view(np.uint16)
-    vb = v.view(torch.int16).numpy().view(np.uint16)
-    qb = q.view(torch.int16).numpy().view(np.uint16)
     table = batch.page_table.numpy()
     lens = batch.seq_lens.numpy()
-    per_step = 2                         # requests per step: a bounded sample of the batch
-    times, nbytes = [], 0.0
-    r = 0
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    G = spec.hq // spec.hkv
+    if spec.mode == "sage":
+        d = wl.make_sage_layer(spec, batch, 0, "cpu")
+        host = {k: getattr(d, k).numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+        unit, scale = "GB/s", 1e9
+        per_key = spec.hkv * spec.head_dim * 2 + spec.hkv * 4 / 64
+
+        def one(i):
+            r = i % spec.batch
+            osg.sage_decode(host["q8"][r:r + 1], host["sf_q"][r:r + 1], host["k8"], host["v8"], host["sf_k"],
+                            host["sf_v"], host["v_mean"], table[r:r + 1], lens[r:r + 1], 64)
+            return float(lens[r]) * per_key
+        per_step, what = 2, "requests"
+    elif spec.mode == "extend":
+        k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
+        cu = batch.cu_seqlens_q.numpy()
+        q = wl.make_bf16_queries(spec, int(cu[-1]), 0, "cpu")
+        kb, vb, qb = bits(k), bits(v), bits(q)
+        unit, scale = "TFLOP/s", 1e12
+
+        def one(i):
+            r, h = (i // spec.hq) % spec.batch, i % spec.hq
+            q0, q1 = int(cu[r]), int(cu[r + 1])
+            oa.extend(qb[q0:q1, h:h + 1], np.array([0, q1 - q0]), kb[:, h // G:h // G + 1], vb[:, h // G:h // G + 1],
+                      table[r:r + 1], lens[r:r + 1], spec.page_size, spec.sm_scale)
+            n = q1 - q0
+            return 4.0 * spec.head_dim * (n * (int(lens[r]) - n) + n * (n + 1) // 2)
+        per_step, what = 2, "(request, query head) pairs"
+    else:
+        k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
+        q = wl.make_bf16_queries(spec, spec.batch, 0, "cpu")
+        kb, vb, qb = bits(k), bits(v), bits(q)
+        unit, scale = "GB/s", 1e9
+
+        def one(i):
+            r = i % spec.batch
+            oa.decode(qb[r:r + 1], kb, vb, table[r:r + 1], lens[r:r + 1], spec.page_size, spec.sm_scale)
+            return wl.decode_kv_bytes([int(lens[r])], spec.hkv, spec.head_dim, 2, spec.page_size, spec.hq, 2, 2)
+        per_step, what = 2, "requests"
+    times, units, i = [], 0.0, 0
     for s in range(args.warmup + args.steps):
-        rs = [(r + i) % spec.batch for i in range(per_step)]
-        r += per_step
         t0 = time.perf_counter()
-        for x in rs:
-            oa.decode(qb[x:x + 1], kb, vb, table[x:x + 1], lens[x:x + 1], spec.page_size, spec.sm_scale)
+        u = sum(one(i + x) for x in range(per_step))
         dt = time.perf_counter() - t0
+        i += per_step
         if s >= args.warmup:
             times.append(dt)
-            nbytes += sum(wl.decode_kv_bytes([int(lens[x])], spec.hkv, spec.head_dim, 2, spec.page_size, spec.hq, 2, 2) for x in rs)
+            units += u
     total = sum(times)
-    value = nbytes / total / 1e9
+    value = units / total / scale if total > 0 else 0.0
     line = {
-        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 0, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": 0, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * total / max(1, args.steps), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]",
                    "hq": spec.hq, "hkv": spec.hkv, "head_dim": spec.head_dim, "page_size": spec.page_size,
                    "layers": spec.layers},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"{per_step} requests of layer 0 per step, oracle.attention.decode in fp64"},
-        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{per_step} {what} of layer 0 per step, the fp64 oracle (oracle/)"},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 

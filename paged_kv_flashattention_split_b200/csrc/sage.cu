@@ -47,7 +47,7 @@ int sage_cap(int max_kv_len) {
 }
 size_t sage_smem_bytes(int G, int cap) {
   return (size_t)kStages * kTileBytes + (size_t)G * cap * 4 + (32 + 8 + 8) * 4 + (size_t)G * kHeadDim * 4 +
-         kStages * 4;
+         (size_t)(cap / kTileKeys) * 8;
 }
 static size_t sage_smem_bytes_max() { return sage_smem_bytes(8, (int)(kSageScoreBudget / (8 * 4))); }
 
@@ -128,7 +128,8 @@ sage_decode_kernel(SageLaunch a) {
   float* cta_max = red + 32;                                        // [8]
   float* part_l = cta_max + 8;                                      // [8]
   float* part_o = part_l + 8;                                       // [G][128]
-  int32_t* tile_page = reinterpret_cast<int32_t*>(part_o + G * kHeadDim);   // [kStages]
+  int32_t* tile_page = reinterpret_cast<int32_t*>(part_o + G * kHeadDim);   // [cap / 64] page of each tile
+  float* tile_sfk = reinterpret_cast<float*>(tile_page + a.cap / kTileKeys);  // [cap / 64] its K scale
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -152,21 +153,21 @@ sage_decode_kernel(SageLaunch a) {
   const size_t slot_stride = (size_t)a.hkv * kRowBytes;
   const uint32_t ring_base = smem_u32(ring);
 
-  // Tile t covers keys k0 + 64 t .. +63, all in one page (k0 is a multiple of 64).
-  auto tile_page_id = [&](int t) -> int {
-    const int j = k0 + t * kTileKeys;
-    const int page = __ldg(table + (j >> 6));
-    if (page < 0 || ((long long)page + 1) * kTileKeys > a.num_slots) {
-      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-      return -1;
-    }
-    return page;
-  };
+  // Tile t covers keys k0 + 64 t .. +63, all in one page (k0 is a multiple of 64).  The page
+  // ids and K scales of all this CTA's tiles are read once, up front, so no copy ever waits
+  // on a table read.
+  for (int t = tid; t < n_tiles; t += kThreads) {
+    const int page = __ldg(table + ((k0 + t * kTileKeys) >> 6));
+    const bool good = page >= 0 && ((long long)page + 1) * kTileKeys <= a.num_slots;
+    if (!good) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    tile_page[t] = good ? page : -1;
+    tile_sfk[t] = good ? __ldg(a.sf_k + (size_t)page * a.hkv + h_kv) : 0.f;
+  }
+  __syncthreads();
   // 64 rows x 128 B: thread -> chunk (tid % 8) of rows tid / 8 + 16 i
   auto issue = [&](const uint8_t* pool, int t) {
     const int stage = t % kStages;
-    const int page = tile_page_id(t);
-    if (tid == 0) tile_page[stage] = page;
+    const int page = tile_page[t];
     const uint32_t dst0 = ring_base + stage * kTileBytes;
     const int c = tid & 7;
 #pragma unroll
@@ -215,8 +216,7 @@ sage_decode_kernel(SageLaunch a) {
       ldmatrix_x4(af, kst + k_row * kRowBytes + ((chunk ^ (k_row & 7)) << 4));
       mma_s8_16832(acc, af, qb0[ks], qb1[ks]);
     }
-    const int page = tile_page[stage];
-    const float sfk = page >= 0 ? __ldg(a.sf_k + (size_t)page * a.hkv + h_kv) : 0.f;
+    const float sfk = tile_sfk[t];
     const int jl0 = t * kTileKeys + warp * 16 + gid, jl1 = jl0 + 8;   // key index within this CTA's range
     const bool v0 = k0 + jl0 < k1, v1 = k0 + jl1 < k1;
     // S = fp32(fp32(sfQ sfK) fp32(dot)); the int32 dot is exact and |dot| < 2^24
@@ -236,6 +236,12 @@ sage_decode_kernel(SageLaunch a) {
     }
   }
   cp_async_wait<0>();
+  __syncthreads();                                             // every warp is done with the K8 ring
+  // the first V8 tiles do not depend on the maximum: start them before the exchange
+  for (int t = 0; t < kStages - 1; ++t) {
+    if (t < n_tiles) issue(a.v8, t);
+    cp_async_commit();
+  }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -264,11 +270,6 @@ sage_decode_kernel(SageLaunch a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) oe[b][i] = oo[b][i] = 0.f;
 
-  __syncthreads();                                             // ring reuse: phase 1 reads are done
-  for (int t = 0; t < kStages - 1; ++t) {
-    if (t < n_tiles) issue(a.v8, t);
-    cp_async_commit();
-  }
   for (int t = 0; t < n_tiles; ++t) {
     cp_async_wait<kStages - 2>();
     __syncthreads();
