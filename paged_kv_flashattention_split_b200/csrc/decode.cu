@@ -52,6 +52,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunc
   static_assert(TK * ROW == kHalfStage && KEY_STEP * LOADS == TK, "tile geometry");
 
   extern __shared__ __align__(128) uint8_t smem[];
+  // the merge kernel (launched as a programmatic dependent) may be scheduled now; it
+  // waits for this whole grid to finish before it reads anything
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   int32_t* sbuf = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes);   // [2][TK]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -270,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunc
 // Lanes read the split LSEs in parallel; each lane owns 4 of the 128 outputs
 // and keeps up to 8 splits' loads in flight.
 __global__ void __launch_bounds__(256) merge_kernel(DecodeLaunch a) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the decode grid has completed and its writes are visible
   PlanHeader* hdr = a.ws.hdr;
   if (!workspace_ok(hdr, PA_MODE_DECODE)) return;
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -345,8 +349,18 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   decode_splitkv_kernel<HG, G><<<a.max_items * groups, kThreads, kDecodeSmem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_kernel<<<(a.batch * a.hq + 7) / 8, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  // the merge is a programmatic dependent of the decode grid: its launch overlaps the decode's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.batch * a.hq + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, a);
 }
 
 template <int G>
