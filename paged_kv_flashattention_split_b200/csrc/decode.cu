@@ -1,15 +1,15 @@
 // decode.cu - bf16 split-KV decode over the paged cache, and the log-sum-exp merge.
 //
-// One CTA per (work item, group of HG KV heads), HG = the largest of 8, 4, 2, 1
-// dividing Hkv, so a CTA gathers each token slot's K and V rows of all its
-// heads as one contiguous HG * 256-byte run (2 KB at Hkv = 8): a warp's
-// 16-byte cp.async copies cover 512 consecutive bytes, and the slots'
-// rows are fetched from HBM once for all query heads that read them.  Tiles
-// of TK = 16 * 8 / HG keys flow through a 3-stage, XOR-swizzled shared-memory
-// ring (64 KB per stage); the slot ids of a tile are read from the table one
-// tile ahead, by TK threads, with the load's latency hidden behind a tile of
-// compute.  Warp (hw, kb) takes KV head hw of the group and keys
-// [16 kb, 16 kb + 16) of every tile and computes, on the tensor cores,
+// One CTA (4 warps, 97 KB of shared memory, two CTAs per SM) per (work item,
+// group of HG KV heads), HG = 4 at Hkv = 8, so a CTA gathers each token slot's K
+// and V rows of its heads as one contiguous HG * 256-byte run (1 KB): a warp's
+// 16-byte cp.async copies cover 512 consecutive bytes, and the slots' rows are
+// fetched from HBM once for all query heads that read them.  Tiles of
+// TK = 16 * 4 / HG keys flow through a 3-stage, XOR-swizzled shared-memory ring;
+// the slot ids of a tile are read from the table one tile ahead, by TK threads,
+// with the load's latency hidden behind a tile of compute.  Warp (hw, kb) takes
+// KV head hw of the group and keys [16 kb, 16 kb + 16) of every tile and
+// computes, on the tensor cores,
 //     S^T[16 keys x 8 heads] = K[16 x 128] . Q^T      (mma.m16n8k16, keys as M)
 // for the G = Hq / Hkv <= 8 query heads that read this KV head.  The online
 // softmax keeps a running max and sum per head (warp shuffles over the 8 key
@@ -29,12 +29,13 @@
 namespace pa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
-constexpr int kHalfStage = 32 * 1024;                      // K (or V) bytes of one tile
+constexpr int kHalfStage = 16 * 1024;                      // K (or V) bytes of one tile
 constexpr int kStageBytes = 2 * kHalfStage;
-constexpr int kSlotBufBytes = 2 * 128 * 4;                 // slot ids of two tiles
-constexpr int kDecodeSmem = kStages * kStageBytes + kSlotBufBytes;   // 193 KB: one CTA per SM
+constexpr int kSlotBufBytes = 2 * 64 * 4;                  // slot ids of two tiles
+constexpr int kDecodeSmem = kStages * kStageBytes + kSlotBufBytes;   // 97 KB: two CTAs per SM
 constexpr float kLn2 = 0.693147180559945309f;
 
 __device__ __forceinline__ bool workspace_ok(const PlanHeader* hdr, int mode) {
@@ -42,8 +43,8 @@ __device__ __forceinline__ bool workspace_ok(const PlanHeader* hdr, int mode) {
 }
 
 template <int HG, int G>
-__global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunch a) {
-  constexpr int WPH = 8 / HG;                 // warps per KV head
+__global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunch a) {
+  constexpr int WPH = kWarps / HG;            // warps per KV head
   constexpr int TK = 16 * WPH;                // keys per tile
   constexpr int CH = HG * 16;                 // 16-byte chunks in one key's row of HG heads
   constexpr int ROW = CH * 16;                // bytes of that row
@@ -211,9 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_splitkv_kernel(DecodeLaunc
   __syncthreads();
 
   // Combine the warps of each head through shared memory.
-  float* red_o = reinterpret_cast<float*>(smem);   // [8 warps][8 heads][128 d]
-  float* red_m = red_o + 8 * 8 * kHeadDim;         // [8][8]
-  float* red_l = red_m + 64;                       // [8][8]
+  float* red_o = reinterpret_cast<float*>(smem);   // [warps][8 heads][128 d]
+  float* red_m = red_o + kWarps * 8 * kHeadDim;    // [warps][8]
+  float* red_l = red_m + kWarps * 8;               // [warps][8]
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l_run0 += __shfl_xor_sync(0xffffffffu, l_run0, off);
@@ -363,10 +364,12 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, merge_kernel, a);
 }
 
+// A plan item covers decode_heads_per_cta(Hkv) <= 8 KV heads; a CTA of four warps takes at
+// most four of them, so an item of eight heads is two CTAs.
 template <int G>
 cudaError_t launch_decode_g(const DecodeLaunch& a, cudaStream_t s) {
   switch (decode_heads_per_cta(a.hkv)) {
-    case 8: return launch_decode_hg<8, G>(a, s);
+    case 8:
     case 4: return launch_decode_hg<4, G>(a, s);
     case 2: return launch_decode_hg<2, G>(a, s);
     default: return launch_decode_hg<1, G>(a, s);
