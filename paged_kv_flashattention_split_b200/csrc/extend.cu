@@ -179,9 +179,8 @@ enum Bar {
   B_S_FULL = B_V_EMPTY + kNumStages,  // S in TMEM
   B_S_FREE,                           // softmax has read S (128 arrivals)
   B_P_FULL,                           // [2] P buffer written (128 arrivals)
-  B_P_FREE = B_P_FULL + 2,            // [2] PV MMA done with the P buffer
-  B_O_DONE = B_P_FREE + 2,            // a PV MMA finished (O stable)
-  B_DRAIN,
+  B_P_FREE = B_P_FULL + 2,            // [2] PV(j) finished (P buffer j % 2 free, O stable)
+  B_DRAIN = B_P_FREE + 2,
   B_COUNT
 };
 static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
@@ -342,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
         }
         tc_commit(bar(B_V_EMPTY + s));
         tc_commit(bar(B_P_FREE + s));
-        tc_commit(bar(B_O_DONE));
       }
       // all issued tensor-core work has finished before TMEM is released
       tc_commit(bar(B_DRAIN));
@@ -416,7 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       const float lt = ((ltp[0] + ltp[1]) + (ltp[2] + ltp[3])) + ((ltp[4] + ltp[5]) + (ltp[6] + ltp[7]));
       if (j >= 2 && !(ok = wwait(bar(B_P_FREE + s), ring_parity(j) ^ 1u))) break;   // PV(j-2) released buffer s
       if (__any_sync(0xffffffffu, alpha != 1.f)) {                                   // rescale rows of O in TMEM
-        if (j > 0 && !(ok = wwait(bar(B_O_DONE), (j - 1) & 1))) break;              // PV(j-1) done: O stable
+        // PV(j-1) done, so O is stable.  "PV(i) done" is always read from P_FREE[i % 2], whose
+        // phases this warpgroup observes in order, so a wait can never match an older phase.
+        if (j > 0 && !(ok = wwait(bar(B_P_FREE + ((j - 1) & 1)), ring_parity(j - 1)))) break;
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -455,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       tc_fence_before();
       mbar_arrive(bar(B_P_FULL + s));
     }
-    if (ok) ok = wwait(bar(B_O_DONE), (n_kv - 1) & 1);
+    // every PV has finished: PV(n-2) and PV(n-1) on their P_FREE barriers
+    if (ok && n_kv >= 2) ok = wwait(bar(B_P_FREE + ((n_kv - 2) & 1)), ring_parity(n_kv - 2));
+    if (ok) ok = wwait(bar(B_P_FREE + ((n_kv - 1) & 1)), ring_parity(n_kv - 1));
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -701,6 +703,9 @@ __global__ void __launch_bounds__(kPairThreads, 1) extend_pair_kernel(const __gr
     for (int j = 0; j < n_kv && ok; ++j) {
       const int s = j & 1;
       if (!(ok = wwait(bar(PB_S_FULL + t), j & 1))) break;
+      // PV_t(j-1) finished before S_t(j); its O_DONE phase is observed here so that every
+      // phase of that barrier is waited in order (the final wait below can never alias)
+      if (j > 0 && !(ok = wwait(bar(PB_O_DONE + t), (j - 1) & 1))) break;
       tc_fence_after();
       uint32_t sv[4][32];
 #pragma unroll
