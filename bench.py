@@ -452,6 +452,31 @@ def main():
     scale = getattr(work, "scale", 1e9)
     value = job_throughput(work.step_bytes, world, ms_per_step, scale)
 
+    # the same step captured once in a CUDA graph and replayed (launch overhead removed)
+    graph_info = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                work.step()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        g0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(dist, g0.elapsed_time(g1) / args.steps, dev)
+        graph_info = {"ms_per_step": round(g_ms, 4), "value": round(job_throughput(work.step_bytes, world, g_ms, getattr(work, "scale", 1e9)), 1)}
+        del graph
+    except Exception as exc:  # reported, never silently replaced
+        graph_info = {"error": str(exc)[:200]}
+
     # end to end through the public API with host buffers
     work.setup_e2e()
     for _ in range(2):
@@ -514,6 +539,7 @@ def main():
         "e2e": {"value": round(e2e_value, 1), "unit": unit, "h2d_bytes_per_step": int(work.e2e_h2d),
                 "d2h_bytes_per_step": int(work.e2e_d2h), "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": work.launches_per_step * args.steps,
+        "graph": graph_info,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -257,6 +257,25 @@ pa_status attn_decode_paged_noalloc(const pa_plan_params* params, const int32_t*
                                     uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
 
 /*
+ * attn_kv_store - write the K and V rows of new tokens into their pool slots: the cache
+ * update that precedes attention in a forward pass ("Flash Attention Backend in SGLang:
+ * Grundlagen und KV Cache optimal nutzen": the cache is updated within the forward
+ * methods; the slot of each new token, out_cache_loc, comes from the caller's allocator).
+ *
+ *   k_pool[out_cache_loc[t]][h][:] = k_new[t][h][:],  the same for V, t < n_tokens.
+ *
+ * d_k_new, d_v_new   bf16 [n_tokens][Hkv][D], device, 16-byte aligned.
+ * d_out_cache_loc    int32 [n_tokens], device: destination slot of each token.
+ * d_k_pool, d_v_pool bf16 [num_slots][Hkv][D], device, 16-byte aligned.
+ * d_ws               optional plan workspace: a slot outside [0, num_slots) is skipped and,
+ *                    when d_ws is given, recorded in its error word (pa_read_device_error).
+ * Two tokens with the same slot race (the last write wins, unspecified which).
+ */
+pa_status attn_kv_store(const uint16_t* d_k_new, const uint16_t* d_v_new, const int32_t* d_out_cache_loc,
+                        int64_t n_tokens, int32_t hkv, int32_t head_dim, uint16_t* d_k_pool,
+                        uint16_t* d_v_pool, int64_t num_slots, void* d_ws, pa_stream_t stream);
+
+/*
  * attn_debug_gather - copy, for request r and KV head h_kv, the slot ids and
  * the K rows the kernels gather: d_slots_out int32 [L], d_rows_out bf16 [L][D]
  * for positions 0 .. L-1, L = min(d_seq_lens[r], max_len).  Out-of-range ids

@@ -203,3 +203,20 @@ def materialised_score_bytes(seq_len: int, elem_bytes: int, batch: int = 1, head
     sample, and 32 GB at batch 8 with 32 heads.
     """
     return seq_len * seq_len * elem_bytes * batch * heads
+
+
+def kv_store(k_pool_bits, v_pool_bits, out_cache_loc, k_new_bits, v_new_bits):
+    """The cache update before attention: pool[loc[t]] = new[t] for every new token t.
+
+    "Flash Attention Backend in SGLang: Grundlagen und KV Cache optimal nutzen": the KV
+    cache is updated within the forward methods; each new token's slot (out_cache_loc)
+    comes from the caller.  Returns updated copies of the pools; a slot outside the pool
+    is skipped.  Raw bit patterns are copied unchanged.
+    """
+    k = np.array(k_pool_bits, copy=True)
+    v = np.array(v_pool_bits, copy=True)
+    for t, slot in enumerate(np.asarray(out_cache_loc, dtype=np.int64)):
+        if 0 <= slot < k.shape[0]:
+            k[slot] = k_new_bits[t]
+            v[slot] = v_new_bits[t]
+    return k, v

@@ -287,6 +287,31 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
   return from_cuda(launch_sage(a, (cudaStream_t)stream));
 }
 
+pa_status attn_kv_store(const uint16_t* d_k_new, const uint16_t* d_v_new, const int32_t* d_out_cache_loc,
+                        int64_t n_tokens, int32_t hkv, int32_t head_dim, uint16_t* d_k_pool, uint16_t* d_v_pool,
+                        int64_t num_slots, void* d_ws, pa_stream_t stream) {
+  if (n_tokens < 0 || hkv < 1 || num_slots < 1) return PA_ERR_INVALID;
+  if (head_dim != kHeadDim) return PA_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return PA_OK;
+  if (!d_k_new || !d_v_new || !d_out_cache_loc || !d_k_pool || !d_v_pool) return PA_ERR_INVALID;
+  if (!aligned16(d_k_new) || !aligned16(d_v_new) || !aligned16(d_k_pool) || !aligned16(d_v_pool) ||
+      (d_ws && !aligned16(d_ws)))
+    return PA_ERR_INVALID;
+  pa_status st = check_arch();
+  if (st != PA_OK) return st;
+  StoreLaunch a;
+  a.k_new = d_k_new;
+  a.v_new = d_v_new;
+  a.loc = d_out_cache_loc;
+  a.n_tokens = n_tokens;
+  a.hkv = hkv;
+  a.k_pool = d_k_pool;
+  a.v_pool = d_v_pool;
+  a.num_slots = num_slots;
+  a.hdr = static_cast<PlanHeader*>(d_ws);
+  return from_cuda(launch_kv_store(a, (cudaStream_t)stream));
+}
+
 pa_status attn_debug_gather(const int32_t* d_seq_lens, int32_t r, int32_t h_kv, int32_t hkv,
                             int32_t head_dim, int32_t page_size, int32_t max_len,
                             const uint16_t* d_k_pool, int64_t num_slots, const int32_t* d_page_table,

@@ -64,6 +64,19 @@ struct ExtendArgs {
 };
 cudaError_t launch_extend(const ExtendArgs& a, cudaStream_t s);
 
+struct StoreLaunch {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const int32_t* loc;
+  int64_t n_tokens;
+  int hkv;
+  uint16_t* k_pool;
+  uint16_t* v_pool;
+  int64_t num_slots;
+  PlanHeader* hdr;     // optional: where to record an out-of-range slot
+};
+cudaError_t launch_kv_store(const StoreLaunch& a, cudaStream_t s);
+
 struct GatherLaunch {
   const int32_t* seq_lens;
   int r, h_kv, hkv, page_shift, max_len;

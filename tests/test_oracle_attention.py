@@ -241,3 +241,16 @@ def test_materialised_memory_figure_from_the_page():
     assert per_head / 2 ** 20 == g["approx_mib_per_head"]
     total = oa.materialised_score_bytes(g["seq_len"], g["elem_bytes"], g["batch"], g["heads"])
     assert total / 2 ** 30 == g["approx_gib_total"]
+
+
+def test_kv_store_closed_form():
+    rng = np.random.default_rng(14)
+    k = _bf16(rng, 10, 2, 4)
+    v = _bf16(rng, 10, 2, 4)
+    kn = _bf16(rng, 3, 2, 4)
+    vn = _bf16(rng, 3, 2, 4)
+    k2, v2 = oa.kv_store(k, v, [7, 2, 99], kn, vn)          # slot 99 is outside the pool: skipped
+    assert np.array_equal(k2[7], kn[0]) and np.array_equal(v2[2], vn[1])
+    untouched = [s for s in range(10) if s not in (7, 2)]
+    assert np.array_equal(k2[untouched], k[untouched]) and np.array_equal(v2[untouched], v[untouched])
+    assert np.array_equal(k[7], k[7])                        # inputs are not modified in place

@@ -1,0 +1,128 @@
+"""GPU tests of the KV-cache store and of a CUDA-graph-captured decode step.
+
+The store is compared bit for bit with the oracle's scatter; a decode step that
+stores the new token's K/V and then attends (the order of a forward pass) matches
+the oracle; and the whole step (store, plan, per-layer decode) captured once in a
+CUDA graph and replayed with new inputs gives the same bits as eager calls.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_flashattention_split_b200 as pa
+import workloads as wl
+from oracle import attention as oa
+from tests.helpers import alloc_ws, assert_bf16_close, bits16
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    if not os.path.exists(pa.LIB_PATH):
+        from paged_kv_flashattention_split_b200 import build
+        build.build()
+    pa.lib()
+
+
+def test_store_is_bit_exact_and_flags_bad_slots():
+    g = torch.Generator(device=DEV).manual_seed(5)
+    k = torch.randn(5000, 8, 128, device=DEV, generator=g).to(torch.bfloat16)
+    v = torch.randn(5000, 8, 128, device=DEV, generator=g).to(torch.bfloat16)
+    kn = torch.randn(300, 8, 128, device=DEV, generator=g).to(torch.bfloat16)
+    vn = torch.randn(300, 8, 128, device=DEV, generator=g).to(torch.bfloat16)
+    loc = torch.randperm(5000, device=DEV, generator=g)[:300].to(torch.int32)
+    loc[17] = 5000                                            # outside the pool: skipped and flagged
+    ref_k, ref_v = oa.kv_store(bits16(k), bits16(v), loc.cpu().numpy(), bits16(kn), bits16(vn))
+    params = pa.make_params(pa.PA_MODE_DECODE, 1, 8, 8, 128, 1, max_kv_len=1, num_sms=0)
+    ws = alloc_ws(params)
+    pa.attn_kv_store(kn, vn, loc, k, v, ws=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits16(k), ref_k) and np.array_equal(bits16(v), ref_v)
+    assert pa.pa_read_device_error(ws) == pa.PA_ERR_DEVICE_INDEX
+
+
+def _decode_step_case():
+    spec = wl.CONFIGS[2].scaled(batch=8, pool_slots=60_000, len_hi=3000, layers=2)
+    batch = wl.make_batch(spec, DEV)
+    pools = [wl.make_bf16_pools(spec, batch, l, DEV) for l in range(spec.layers)]
+    # the decode token of every request goes to a fresh (unused, NaN-filled) slot, appended to its row
+    unused = torch.nonzero(~batch.used_slot_mask).flatten()[: spec.batch].to(torch.int32)
+    table = torch.zeros(spec.batch, batch.page_table.shape[1] + 1, dtype=torch.int32, device=DEV)
+    table[:, :-1] = batch.page_table
+    lens = batch.seq_lens.clone()
+    for r in range(spec.batch):
+        table[r, int(lens[r])] = unused[r]
+    lens += 1
+    return spec, wl.Batch(lens, table, batch.num_slots, batch.used_slot_mask), pools, unused
+
+
+def test_store_then_decode_matches_the_oracle():
+    spec, batch, pools, loc = _decode_step_case()
+    g = torch.Generator(device=DEV).manual_seed(9)
+    q = torch.randn(spec.batch, spec.hq, 128, device=DEV, generator=g).to(torch.bfloat16)
+    kn = torch.randn(spec.batch, spec.hkv, 128, device=DEV, generator=g).to(torch.bfloat16)
+    vn = torch.randn(spec.batch, spec.hkv, 128, device=DEV, generator=g).to(torch.bfloat16)
+    k, v = pools[0]
+    ref_k, ref_v = oa.kv_store(bits16(k), bits16(v), loc.cpu().numpy(), bits16(kn), bits16(vn))
+    params = pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, 128, 1,
+                            max_kv_len=batch.page_table.shape[1])
+    ws = alloc_ws(params)
+    pa.attn_kv_store(kn, vn, loc, k, v)
+    pa.attn_plan(params, batch.seq_lens, None, ws)
+    out = torch.empty_like(q)
+    pa.attn_decode_paged(params, ws, q, k, v, batch.page_table, spec.sm_scale, out)
+    torch.cuda.synchronize()
+    ref, _ = oa.decode(bits16(q), ref_k, ref_v, batch.page_table.cpu().numpy(), batch.seq_lens.cpu().numpy(), 1,
+                       spec.sm_scale)
+    assert_bf16_close(out, ref, "store + decode")
+
+
+def test_decode_step_captured_in_a_cuda_graph_replays_bit_exactly():
+    spec, batch, pools, loc = _decode_step_case()
+    params = pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, 128, 1,
+                            max_kv_len=batch.page_table.shape[1])
+    ws = alloc_ws(params)
+    shape_q, shape_kv = (spec.batch, spec.hq, 128), (spec.batch, spec.hkv, 128)
+    q = torch.zeros(spec.layers, *shape_q, dtype=torch.bfloat16, device=DEV)
+    kn = torch.zeros(spec.layers, *shape_kv, dtype=torch.bfloat16, device=DEV)
+    vn = torch.zeros_like(kn)
+    out = torch.zeros_like(q)
+
+    def step():
+        pa.attn_plan(params, batch.seq_lens, None, ws)
+        for l in range(spec.layers):
+            k, v = pools[l]
+            pa.attn_kv_store(kn[l], vn[l], loc, k, v)
+            pa.attn_decode_paged(params, ws, q[l], k, v, batch.page_table, spec.sm_scale, out[l])
+
+    def fill(seed):
+        g = torch.Generator(device=DEV).manual_seed(seed)
+        q.copy_(torch.randn(q.shape, device=DEV, generator=g).to(torch.bfloat16))
+        kn.copy_(torch.randn(kn.shape, device=DEV, generator=g).to(torch.bfloat16))
+        vn.copy_(torch.randn(vn.shape, device=DEV, generator=g).to(torch.bfloat16))
+
+    fill(1)
+    step()                                     # eager warm-up (sets kernel attributes before capture)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            step()
+    torch.cuda.synchronize()
+    for seed in (2, 3):
+        fill(seed)
+        step()
+        torch.cuda.synchronize()
+        eager = out.clone()
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    del graph
