@@ -258,7 +258,7 @@ class SageWorkload(DecodeWorkload):
                                  + sum((x + 63) // 64 for x in L) * (spec.hkv * 4 + 4)
                                  + spec.batch * spec.hq * (spec.head_dim * 1 + 4 + spec.head_dim * 2))
         self.step_bytes = self.layer_bytes * spec.layers
-        self.launches_per_step = 1 + spec.layers
+        self.launches_per_step = 1 + 3 * spec.layers   # plan, then score + value + merge per layer
 
     def layer(self, l):
         d = self.layers_data[l % len(self.layers_data)]
@@ -530,7 +530,7 @@ def main():
         "roofline": {
             "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": {"sage_decode": "sage_decode_kernel (one launch per attn_decode_paged_sage call)",
+            "kernel": {"sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
                        "extend_prefix": "extend_kernel (one launch per attn_extend_paged call)"}.get(
                            args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
                       + ", per-layer CUDA events",

@@ -91,7 +91,7 @@ typedef struct {
   int32_t max_kv_len;    /* upper bound on every seq_lens[r]; longer lengths are clamped and flagged */
   int32_t max_q_tokens;  /* EXTEND: upper bound on sum of new tokens (sizes the grid); else 0 */
   int32_t num_sms;       /* SMs the plan schedules for; 0 = query the current device */
-  int32_t max_splits;    /* DECODE: cap on splits per request, >= 1 (0 = 128) */
+  int32_t max_splits;    /* DECODE: cap on splits per request (0 = 128); EXTEND: 0 or 1; SAGE: 0 */
   int32_t sage_k_block;  /* SAGE: keys per sfK block, must be 64; else 0 */
   int32_t reserved;      /* must be 0 */
 } pa_plan_params;
@@ -129,25 +129,43 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  *   EXTEND: query tiles of 128 new tokens; tile t of request r covers new
  *     tokens [128 t, min(128 t + 128, n_r)) and reads key tiles
  *     0 .. ceil((p_r + q_end) / 128) - 1, p_r = L_r - n_r.
- *   SAGE_DECODE: one item per request covering [0, L_r).
- * The items are ordered by work (key count, key-tile count or L_r) descending,
- * ties by (request, split) order, so the in-order block dispatch of the run
- * kernels schedules the longest work first.  At most ceil(num_sms * 4 / groups)
- * + B items (DECODE), ceil(max_q_tokens / 128) + B (EXTEND) or B (SAGE).
+ *   DECODE and EXTEND items are ordered by work (key count or key-tile
+ *     count) descending, ties by (request, split) order, so the in-order block
+ *     dispatch of the run kernels schedules the longest work first.
+ *   SAGE_DECODE: a flat, balanced partition.  units_r = ceil(L_r / 32), HG and
+ *     groups as for DECODE, C = max(1, floor(num_sms * 2 / groups)) CTA slots
+ *     (one wave of two CTAs per SM), g_r = sum of the units of the requests
+ *     before r, total = sum units_r, per = max(1, ceil(total / C)),
+ *     used = ceil(total / per).  Slot c takes the concatenated units
+ *     [c per, (c+1) per); each maximal piece of that range within one request
+ *     is an item (r, s, 32 u0, min(32 u1, L_r)), u0/u1 relative to g_r and s
+ *     the piece's index within request r; an empty request is one item
+ *     (r, 0, 0, 0) of slot min(floor(g_r / per), max(used - 1, 0)).  Items are
+ *     listed r-major (which is also slot order, no sort) and slot_first[c],
+ *     c = 0 .. C, is the first item of slot c or later (num_items if none).
+ *     max_splits must be 0 (the slots are balanced by construction).
+ * At most ceil(num_sms * 4 / groups) + B items (DECODE), C + B (SAGE) or
+ * ceil(max_q_tokens / 128) + B (EXTEND).
  *
  * Workspace layout (for introspection; all int32, offsets in bytes):
  *   [0, 64)   header: magic 0x4C504150, mode, batch, hq, hkv, head_dim,
  *             page_size, num_items, max_items, tile, chunk_tiles, error word,
- *             num_sms, max_splits, reserved x2
+ *             num_sms, max_splits, slots (SAGE: C, else 0), reserved
  *   then      req_splits[B] (items of request r), req_base[B+1] (exclusive
  *             prefix sum of req_splits), req_len[B] (L_r as used), req_aux[B]
- *             (DECODE: chunk_r tiles per split; EXTEND: cu_seqlens_q[r]),
+ *             (DECODE: chunk_r tiles per split; EXTEND: cu_seqlens_q[r];
+ *             SAGE: g_r),
  *             req_prefix[B] (EXTEND: p_r), padded to 16 B, then the items
  *             int32x4 [max_items] = {r, split, begin, end} in execution order,
- *             256-byte aligned, then (DECODE) fp32 partial outputs
- *             [max_items][Hq][D] and partial LSEs (log2 units) [max_items][Hq],
- *             each 256-byte aligned.  The partial of split s of request r,
- *             head h, sits at row (req_base[r] + s) * Hq + h.
+ *             256-byte aligned, then (SAGE) slot_first int32 [C + 1], 256-byte
+ *             aligned, then (DECODE, SAGE) fp32 partial outputs
+ *             [max_items][Hq][D] and partial LSEs (DECODE: log2 units; SAGE:
+ *             the split's row sum l) [max_items][Hq], then (SAGE) the split
+ *             maxima fp32 [max_items][Hq] and the score rows fp32
+ *             [B][Hq][max(max_kv_len, 64) rounded up to 64], each 256-byte
+ *             aligned.
+ *             The partial of split s of request r, head h, sits at row
+ *             (req_base[r] + s) * Hq + h.
  * Lengths < 0 or > max_kv_len are clamped to [0, max_kv_len] and set the
  * error word.  Returns PA_ERR_ARCH off sm_100, PA_ERR_WORKSPACE if ws_bytes
  * is short, PA_ERR_INVALID for NULL pointers or a cu_seqlens_q that does not
@@ -217,8 +235,14 @@ pa_status attn_extend_paged(const pa_plan_params* params, const void* d_ws, size
  * d_k8_pool int8, d_v8_pool E4M3 bytes, both [num_slots][Hkv][D].
  * d_sf_k fp32 [num_slots / 64][Hkv];  d_sf_v fp32 [Hkv][D];
  * d_v_mean fp32 [Hkv][D] or NULL (then 0).   d_out bf16 [B][Hq][D].
- * The whole row of scores is kept on chip, so G * max_kv_len * 4 bytes must fit
- * the kernel's shared-memory budget (checked at plan time: PA_ERR_UNSUPPORTED).
+ * d_sf_k, d_sf_v and d_v_mean 16-byte aligned, like the 8-bit tensors and d_out.
+ * Three kernels over the plan's CTA slots: a score pass writes S of every key
+ * and query head to the workspace's score rows and each item's per-head
+ * maximum; a value pass takes m as the maximum of the request's item maxima
+ * (the exact row max), forms P8 from the stored S and accumulates P8 . V8 per
+ * item; a merge sums the items (no rescale: all used the same m).  Rows of
+ * any length up to max_kv_len are supported; the workspace grows with
+ * B * Hq * max_kv_len * 4 bytes of score rows.
  * Empty requests give O = v_mean.
  */
 pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,

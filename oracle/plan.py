@@ -36,14 +36,33 @@ EXTEND (query-tile work list)
   sorted by that key-tile count descending, ties by generation order.
   Bound: num_items <= ceil(max_q_tokens / 128) + B.
 
-SAGE_DECODE (one item per request)
-  items (r, 0, 0, L_r) sorted by L_r descending, ties by r.  num_items = B.
+SAGE_DECODE (flat, balanced partition over CTA slots)
+  U        = 32 keys per unit; units_r = ceil(L_r / U)
+  HG, groups as for DECODE (a CTA covers HG KV heads of one slot)
+  C        = max(1, floor(num_sms * 2 / groups))     CTA slots (one wave of
+                                                   two CTAs per SM)
+  g_r      = sum_{r' < r} units_r'                 request r's first unit in
+                                                   the concatenated sequence
+  total    = sum_r units_r, per = max(1, ceil(total / C)) units per slot,
+  used     = ceil(total / per)                     slots that get units
+  slot c takes the global units [c per, (c+1) per); each maximal piece of that
+  range inside one request is an item (r, s, U u0, min(U u1, L_r)) with u0, u1
+  the piece's unit bounds relative to g_r and s its index among request r's
+  pieces.  An empty request is one item (r, 0, 0, 0) in slot
+  min(floor(g_r / per), max(used - 1, 0)).  Items are listed r-major then s,
+  which is also slot order, so no sort is needed; slot_first[c] (c = 0 .. C)
+  is the first item of slot c or later (num_items if none), and slot c runs
+  items slot_first[c] .. slot_first[c+1] - 1.  req_base as for DECODE; every
+  slot has at most per units, so the slots finish together.
+  Bound: num_items <= C + B.
 """
 from __future__ import annotations
 
 MODE_DECODE, MODE_EXTEND, MODE_SAGE_DECODE = 0, 1, 2
 DECODE_MIN_TILE = 64
 DECODE_CTAS_PER_SM = 4
+SAGE_UNIT = 32
+SAGE_CTAS_PER_SM = 2
 EXTEND_Q_TILE = 128
 EXTEND_KV_TILE = 128
 
@@ -64,22 +83,30 @@ def decode_head_groups(hkv: int) -> int:
     raise ValueError("hkv must be positive")
 
 
+def sage_slots(hkv: int, num_sms: int) -> int:
+    """CTA slots of a Sage plan: max(1, floor(num_sms * 2 / groups))."""
+    return max(1, num_sms * SAGE_CTAS_PER_SM // decode_head_groups(hkv))
+
+
 def max_items(mode: int, batch: int, hkv: int, num_sms: int, max_q_tokens: int = 0) -> int:
     """The host-side bound on the number of work items for a plan of this shape."""
     if mode == MODE_DECODE:
         return _cdiv(num_sms * DECODE_CTAS_PER_SM, decode_head_groups(hkv)) + batch
+    if mode == MODE_SAGE_DECODE:
+        return sage_slots(hkv, num_sms) + batch
     if mode == MODE_EXTEND:
         return _cdiv(max_q_tokens, EXTEND_Q_TILE) + batch
-    return batch
+    raise ValueError("unknown mode")
 
 
 def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, num_sms: int,
          max_splits: int = 1 << 30, max_q_tokens: int = 0):
     """Return the plan as a dict of plain Python ints and lists.
 
-    Keys: ``tile``, ``chunk_tiles`` (DECODE; 0 otherwise), ``req_splits``,
-    ``req_base`` (length B + 1), ``items`` (list of 4-tuples, in execution
-    order) and ``num_items``.
+    Keys: ``tile``, ``chunk_tiles`` (DECODE: tiles per split; SAGE_DECODE:
+    units per slot; 0 otherwise), ``req_splits``, ``req_base`` (length B + 1),
+    ``items`` (list of 4-tuples, in execution order), ``num_items`` and, for
+    SAGE_DECODE, ``slot_first`` (length C + 1).
     """
     L = [int(x) for x in seq_lens]
     B = len(L)
@@ -89,6 +116,8 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
     splits = [0] * B
     chunk = 0
     tile = 0
+    if mode == MODE_SAGE_DECODE:
+        return _sage_plan(L, hkv, num_sms)
     if mode == MODE_DECODE:
         tile = decode_tile(page_size)
         tiles = [_cdiv(x, tile) for x in L]
@@ -124,11 +153,6 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
                 q0 = t * EXTEND_Q_TILE
                 q1 = min(q0 + EXTEND_Q_TILE, n)
                 gen.append((_cdiv(p + q1, EXTEND_KV_TILE), (r, t, q0, q1)))
-    elif mode == MODE_SAGE_DECODE:
-        tile = 64
-        for r in range(B):
-            splits[r] = 1
-            gen.append((L[r], (r, 0, 0, L[r])))
     else:
         raise ValueError("unknown mode")
     order = sorted(range(len(gen)), key=lambda i: (-gen[i][0], i))
@@ -138,3 +162,38 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
         base[r + 1] = base[r] + splits[r]
     return {"tile": tile, "chunk_tiles": chunk, "req_splits": splits, "req_base": base,
             "items": items, "num_items": len(items)}
+
+
+def _sage_plan(L, hkv: int, num_sms: int):
+    """The flat partition of SAGE_DECODE (module docstring), written out unit by unit."""
+    B = len(L)
+    units = [_cdiv(x, SAGE_UNIT) for x in L]
+    C = sage_slots(hkv, num_sms)
+    total = sum(units)
+    per = max(1, _cdiv(total, C))
+    used = _cdiv(total, per)
+    items, item_slot, splits = [], [], [0] * B
+    g = 0
+    for r in range(B):
+        if units[r] == 0:
+            splits[r] = 1
+            items.append((r, 0, 0, 0))
+            item_slot.append(min(g // per, max(used - 1, 0)))
+            continue
+        c_first, c_last = g // per, (g + units[r] - 1) // per
+        splits[r] = c_last - c_first + 1
+        for s, c in enumerate(range(c_first, c_last + 1)):
+            u0 = max(g, c * per) - g
+            u1 = min(g + units[r], (c + 1) * per) - g
+            items.append((r, s, SAGE_UNIT * u0, min(SAGE_UNIT * u1, L[r])))
+            item_slot.append(c)
+        g += units[r]
+    slot_first = []
+    for c in range(C + 1):
+        later = [i for i, sc in enumerate(item_slot) if sc >= c]
+        slot_first.append(later[0] if later else len(items))
+    base = [0] * (B + 1)
+    for r in range(B):
+        base[r + 1] = base[r] + splits[r]
+    return {"tile": SAGE_UNIT, "chunk_tiles": per, "req_splits": splits, "req_base": base,
+            "items": items, "num_items": len(items), "slot_first": slot_first}

@@ -19,7 +19,7 @@ using namespace pa;
 namespace {
 
 struct Derived {
-  int G = 0, num_sms = 0, max_splits = 0, max_items = 0, tile = 0, sort_n = 0, page_shift = 0;
+  int G = 0, num_sms = 0, max_splits = 0, max_items = 0, tile = 0, sort_n = 0, page_shift = 0, slots = 0;
   WsLayout layout{};
 };
 
@@ -81,12 +81,15 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
       d->tile = kExtendKvTile;
       break;
     case PA_MODE_SAGE_DECODE:
-      if (p->max_q_tokens != 0 || p->max_splits > 1) return PA_ERR_INVALID;
+      // the flat partition balances the slots itself: no split cap
+      if (p->max_q_tokens != 0 || p->max_splits != 0) return PA_ERR_INVALID;
       if (p->sage_k_block != kSageBlock || P != kSageBlock) return PA_ERR_UNSUPPORTED;
-      // shared-memory budget of the scores a CTA keeps (a quarter of the row per CTA)
-      if ((size_t)G * (size_t)sage_cap(p->max_kv_len) * 4 > kSageScoreBudget) return PA_ERR_UNSUPPORTED;
-      d->max_splits = 1;
-      d->tile = kSageBlock;
+      d->max_splits = 0;
+      // the score rows ([B][Hq][max_kv_len rounded up to 64] fp32) stay below 2^46 bytes
+      if ((double)p->batch * p->hq * ((double)p->max_kv_len + kSageBlock) * 4.0 > 7.0e13) return PA_ERR_UNSUPPORTED;
+      // the plan counts 32-key units in int32
+      if ((long long)p->batch * ((p->max_kv_len + kSageUnit - 1) / kSageUnit) >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+      d->tile = kSageUnit;
       break;
   }
   int sms = p->num_sms;
@@ -101,16 +104,19 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
     const int groups = p->hkv / decode_heads_per_cta(p->hkv);
     mi = ((long long)sms * kDecodeCtasPerSm + groups - 1) / groups + p->batch;
   }
-  else if (p->mode == PA_MODE_EXTEND)
-    mi = ((long long)p->max_q_tokens + kExtendQTile - 1) / kExtendQTile + p->batch;
+  else if (p->mode == PA_MODE_SAGE_DECODE)
+  {
+    d->slots = sage_slots(p->hkv, sms);
+    mi = (long long)d->slots + p->batch;
+  }
   else
-    mi = p->batch;
+    mi = ((long long)p->max_q_tokens + kExtendQTile - 1) / kExtendQTile + p->batch;
   if (mi > kMaxSortItems) return PA_ERR_UNSUPPORTED;
   d->max_items = (int)mi;
   int n = 2;
   while (n < d->max_items) n <<= 1;
   d->sort_n = n;
-  d->layout = ws_layout(p->mode, p->batch, p->hq, p->hkv, p->head_dim, d->max_items);
+  d->layout = ws_layout(p->mode, p->batch, p->hq, p->hkv, p->head_dim, d->max_items, p->max_kv_len, d->slots);
   return PA_OK;
 }
 
@@ -170,6 +176,7 @@ pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
   a.max_items = d.max_items;
   a.tile = d.tile;
   a.sort_n = d.sort_n;
+  a.slots = d.slots;
   return from_cuda(launch_plan(a, (cudaStream_t)stream));
 }
 
@@ -259,7 +266,8 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
   if (params->mode != PA_MODE_SAGE_DECODE) return PA_ERR_WORKSPACE;
   if (!d_ws || !d_q8 || !d_sf_q || !d_k8_pool || !d_v8_pool || !d_sf_k || !d_sf_v || !d_page_table || !d_out)
     return PA_ERR_INVALID;
-  if (!aligned16(d_ws) || !aligned16(d_q8) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) || !aligned16(d_out))
+  if (!aligned16(d_ws) || !aligned16(d_q8) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) || !aligned16(d_out) ||
+      !aligned16(d_sf_k) || !aligned16(d_sf_v) || (d_v_mean && !aligned16(d_v_mean)))
     return PA_ERR_INVALID;
   if (num_slots < kSageBlock || num_slots % kSageBlock != 0 || num_slots >= (1LL << 31) || pt_pitch < 1)
     return PA_ERR_INVALID;
@@ -283,7 +291,7 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
   a.batch = params->batch;
   a.hq = params->hq;
   a.hkv = params->hkv;
-  a.max_kv_len = params->max_kv_len;
+  a.slots = d.slots;
   return from_cuda(launch_sage(a, (cudaStream_t)stream));
 }
 

@@ -20,7 +20,8 @@ constexpr int kDecodeCtasPerSm = 4;              // decode CTAs a plan aims for,
 constexpr int kExtendQTile = 128;
 constexpr int kExtendKvTile = 128;
 constexpr int kSageBlock = 64;
-constexpr size_t kSageScoreBudget = 64 * 1024;  // bytes of on-chip scores per Sage CTA (G x keys x 4)
+constexpr int kSageUnit = 32;                    // keys per unit of the Sage partition
+constexpr int kSageCtasPerSm = 2;                // Sage CTAs resident per SM (one wave of slots)
 constexpr int kMaxBatch = 8192;
 constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capacity
 
@@ -28,13 +29,15 @@ constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capa
 struct PlanHeader {
   int32_t magic, mode, batch, hq, hkv, head_dim, page_size, num_items;
   int32_t max_items, tile, chunk_tiles, error_word;
-  int32_t num_sms, max_splits, reserved0, reserved1;
+  int32_t num_sms, max_splits, slots, reserved1;   // slots: SAGE CTA slots, else 0
 };
 static_assert(sizeof(PlanHeader) == 64, "header is 64 bytes");
 
 // Byte offsets of the workspace arrays.
 struct WsLayout {
-  size_t req_splits, req_base, req_len, req_aux, req_prefix, items, partial_o, partial_lse, total;
+  size_t req_splits, req_base, req_len, req_aux, req_prefix, items, slot_first, partial_o, partial_lse, item_max,
+      scores, total;
+  int64_t score_pitch;   // SAGE: keys per (request, head) row of the score scratch
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -44,7 +47,20 @@ __host__ __device__ inline int decode_heads_per_cta(int hkv) {
   return hkv % 8 == 0 ? 8 : hkv % 4 == 0 ? 4 : hkv % 2 == 0 ? 2 : 1;
 }
 
-inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, int max_items) {
+// Modes whose run kernels write split partials for a merge.
+__host__ __device__ inline bool splitkv_mode(int mode) {
+  return mode == PA_MODE_DECODE || mode == PA_MODE_SAGE_DECODE;
+}
+
+// CTA slots of a Sage plan: max(1, floor(num_sms * 2 / groups)).
+__host__ __device__ inline int sage_slots(int hkv, int num_sms) {
+  const int groups = hkv / decode_heads_per_cta(hkv);
+  const int c = num_sms * kSageCtasPerSm / groups;
+  return c > 1 ? c : 1;
+}
+
+inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, int max_items, int max_kv_len,
+                          int slots) {
   WsLayout w{};
   size_t off = sizeof(PlanHeader);
   w.req_splits = off; off += 4 * (size_t)batch;
@@ -55,10 +71,21 @@ inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, in
   off = align_up(off, 16);
   w.items = off;      off += 16 * (size_t)max_items;
   off = align_up(off, 256);
-  if (mode == PA_MODE_DECODE) {
+  if (mode == PA_MODE_SAGE_DECODE) {
+    w.slot_first = off; off += 4 * (size_t)(slots + 1);
+    off = align_up(off, 256);
+  }
+  if (splitkv_mode(mode)) {
     w.partial_o = off;   off += 4 * (size_t)max_items * hq * head_dim;
     off = align_up(off, 256);
     w.partial_lse = off; off += 4 * (size_t)max_items * hq;
+    off = align_up(off, 256);
+  }
+  if (mode == PA_MODE_SAGE_DECODE) {
+    w.item_max = off;    off += 4 * (size_t)max_items * hq;
+    off = align_up(off, 256);
+    w.score_pitch = (int64_t)align_up((size_t)(max_kv_len > kSageBlock ? max_kv_len : kSageBlock), kSageBlock);
+    w.scores = off;      off += 4 * (size_t)batch * hq * (size_t)w.score_pitch;
     off = align_up(off, 256);
   }
   w.total = off;
@@ -74,8 +101,12 @@ struct WsView {
   int32_t* req_aux;
   int32_t* req_prefix;
   int4* items;
+  int32_t* slot_first;  // SAGE: [slots + 1] first item of each CTA slot
   float* partial_o;
-  float* partial_lse;
+  float* partial_lse;   // DECODE: split LSE (log2); SAGE: split row sum l
+  float* item_max;      // SAGE: [max_items][Hq] maximum score of each split
+  float* scores;        // SAGE: [B][Hq][score_pitch] the scores S
+  int64_t score_pitch;
 };
 
 inline WsView ws_view(void* ws, const WsLayout& w) {
@@ -88,8 +119,12 @@ inline WsView ws_view(void* ws, const WsLayout& w) {
   v.req_aux = reinterpret_cast<int32_t*>(b + w.req_aux);
   v.req_prefix = reinterpret_cast<int32_t*>(b + w.req_prefix);
   v.items = reinterpret_cast<int4*>(b + w.items);
+  v.slot_first = w.slot_first ? reinterpret_cast<int32_t*>(b + w.slot_first) : nullptr;
   v.partial_o = w.partial_o ? reinterpret_cast<float*>(b + w.partial_o) : nullptr;
   v.partial_lse = w.partial_lse ? reinterpret_cast<float*>(b + w.partial_lse) : nullptr;
+  v.item_max = w.item_max ? reinterpret_cast<float*>(b + w.item_max) : nullptr;
+  v.scores = w.scores ? reinterpret_cast<float*>(b + w.scores) : nullptr;
+  v.score_pitch = w.score_pitch;
   return v;
 }
 

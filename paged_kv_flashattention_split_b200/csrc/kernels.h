@@ -11,6 +11,7 @@ struct PlanLaunch {
   const int32_t* cu_seqlens_q;
   int mode, batch, hq, hkv, head_dim, page_size, max_kv_len, num_sms, max_splits, max_items, tile;
   int sort_n;  // power of two >= max_items
+  int slots;   // SAGE: CTA slots
 };
 cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s);
 
@@ -42,11 +43,9 @@ struct SageLaunchArgs {
   const int32_t* page_table;
   int64_t pt_pitch;
   uint16_t* out;
-  int batch, hq, hkv, max_kv_len;
+  int batch, hq, hkv, slots;
 };
 cudaError_t launch_sage(const SageLaunchArgs& a, cudaStream_t s);
-int sage_cap(int max_kv_len);          // score keys per CTA per head for this max length
-size_t sage_smem_bytes(int G, int cap);
 
 struct ExtendArgs {
   WsView ws;

@@ -58,11 +58,90 @@ __device__ __forceinline__ int item_work(int mode, int s, int L, int chunk_r, in
     const long long b = min((long long)(s + 1) * chunk_r * tile, (long long)L);
     return (int)(b - a);
   }
-  if (mode == PA_MODE_EXTEND) {
-    const int q1 = min((s + 1) * kExtendQTile, n);
-    return (int)cdiv_ll(prefix + q1, kExtendKvTile);
+  const int q1 = min((s + 1) * kExtendQTile, n);
+  return (int)cdiv_ll(prefix + q1, kExtendKvTile);
+}
+
+// SAGE_DECODE: the flat partition of the requests' 32-key units over CTA slots (the
+// algorithm at attn_plan).  Items come out r-major, which is also slot order, so no sort.
+__device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* chunk_out, int* n_out) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  WsView ws = a.ws;
+  PlanHeader* hdr = ws.hdr;
+  const int B = a.batch;
+  // 1. lengths (clamped and flagged when out of range)
+  for (int r = tid; r < B; r += nt) {
+    int L = a.seq_lens[r];
+    if (L < 0 || L > a.max_kv_len) {
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      L = max(0, min(L, a.max_kv_len));
+    }
+    ws.req_len[r] = L;
   }
-  return L;
+  __syncthreads();
+  // 2. g_r = exclusive prefix sum of the units (kept in req_aux), total
+  const int per_t = (B + nt - 1) / nt;
+  const int r0 = min(B, tid * per_t), r1 = min(B, r0 + per_t);
+  long long local = 0;
+  for (int r = r0; r < r1; ++r) local += cdiv_ll(ws.req_len[r], kSageUnit);
+  int total = 0;
+  int run = block_exclusive_scan((int)local, scan, &total);
+  for (int r = r0; r < r1; ++r) {
+    ws.req_aux[r] = run;
+    run += (int)cdiv_ll(ws.req_len[r], kSageUnit);
+  }
+  const int per = (int)max(1LL, cdiv_ll(total, a.slots));
+  const int used = (int)cdiv_ll(total, per);
+  __syncthreads();
+  // 3. pieces per request, then req_base
+  for (int r = tid; r < B; r += nt) {
+    const int u = (int)cdiv_ll(ws.req_len[r], kSageUnit), g = ws.req_aux[r];
+    ws.req_splits[r] = u > 0 ? (g + u - 1) / per - g / per + 1 : 1;
+    ws.req_prefix[r] = 0;
+  }
+  __syncthreads();
+  int local_s = 0;
+  for (int r = r0; r < r1; ++r) local_s += ws.req_splits[r];
+  int n_items = 0;
+  int run_s = block_exclusive_scan(local_s, scan, &n_items);
+  for (int r = r0; r < r1; ++r) {
+    ws.req_base[r] = run_s;
+    run_s += ws.req_splits[r];
+  }
+  if (tid == 0) ws.req_base[B] = n_items;
+  if (n_items > a.max_items) {  // cannot happen (bound slots + B); keep the grid safe
+    if (tid == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    n_items = a.max_items;
+  }
+  __syncthreads();
+  // 4. the items and the slot of each
+  for (int r = tid; r < B; r += nt) {
+    const int L = ws.req_len[r], u = (int)cdiv_ll(L, kSageUnit), g = ws.req_aux[r], base = ws.req_base[r];
+    if (u == 0) {
+      if (base < n_items) {
+        ws.items[base] = make_int4(r, 0, 0, 0);
+        item_slot[base] = min(g / per, max(used - 1, 0));
+      }
+      continue;
+    }
+    const int c_first = g / per, c_last = (g + u - 1) / per;
+    for (int c = c_first; c <= c_last; ++c) {
+      const int i = base + (c - c_first);
+      if (i >= n_items) break;
+      const int u0 = max(g, c * per) - g, u1 = min(g + u, (c + 1) * per) - g;
+      ws.items[i] = make_int4(r, c - c_first, u0 * kSageUnit, min(u1 * kSageUnit, L));
+      item_slot[i] = c;
+    }
+  }
+  for (int c = tid; c <= a.slots; c += nt) ws.slot_first[c] = n_items;
+  __syncthreads();
+  // 5. slot_first[c] = first item whose slot is >= c (slots are non-decreasing along the list)
+  for (int i = tid; i < n_items; i += nt) {
+    const int c_prev = i > 0 ? item_slot[i - 1] : -1;
+    for (int c = c_prev + 1; c <= item_slot[i]; ++c) ws.slot_first[c] = i;
+  }
+  *chunk_out = per;
+  *n_out = n_items;
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
@@ -75,6 +154,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
   const int B = a.batch;
   if (tid == 0) hdr->error_word = 0;  // every new plan starts with a clean error word
   __syncthreads();
+  int chunk = 0, n_items = 0;
+  if (a.mode == PA_MODE_SAGE_DECODE) {
+    sage_plan(a, reinterpret_cast<int*>(keys), scan, &chunk, &n_items);
+  } else {
 
   // 1. lengths (clamped and flagged when out of range), tiles per request
   long long my_tiles = 0;
@@ -88,13 +171,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     if (a.mode == PA_MODE_DECODE) my_tiles += cdiv_ll(L, a.tile);
   }
   const long long total = block_sum(my_tiles, red) * (a.hkv / decode_heads_per_cta(a.hkv));
-  int chunk = 0;
   if (a.mode == PA_MODE_DECODE) {
     const long long slots = (long long)a.num_sms * kDecodeCtasPerSm;
     chunk = (int)max(1LL, cdiv_ll(total, slots));
   }
 
-  // 2. splits (DECODE), query tiles (EXTEND) or one item (SAGE) per request
+  // 2. splits (DECODE, SAGE) or query tiles (EXTEND) per request
   for (int r = tid; r < B; r += nt) {
     const int L = ws.req_len[r];
     int splits = 1, aux = 0, prefix = 0;
@@ -142,7 +224,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     run += ws.req_splits[r];
   }
   if (tid == 0) ws.req_base[B] = total_items;
-  int n_items = total_items;
+  n_items = total_items;
   if (n_items > a.max_items) {  // cannot happen for lengths within bounds; keep the grid safe
     if (tid == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
     n_items = a.max_items;
@@ -199,16 +281,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
       const long long b0 = (long long)s * aux * a.tile;
       it.z = (int)min(b0, (long long)L);
       it.w = (int)min((long long)(s + 1) * aux * a.tile, (long long)L);
-    } else if (a.mode == PA_MODE_EXTEND) {
+    } else {
       const int n = L - prefix;
       it.z = s * kExtendQTile;
       it.w = min((s + 1) * kExtendQTile, n);
-    } else {
-      it.z = 0;
-      it.w = L;
     }
     ws.items[i] = it;
   }
+  }  // DECODE, EXTEND
 
   // 7. header
   if (tid == 0) {
@@ -225,7 +305,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     hdr->chunk_tiles = chunk;
     hdr->num_sms = a.num_sms;
     hdr->max_splits = a.max_splits;
-    hdr->reserved0 = 0;
+    hdr->slots = a.mode == PA_MODE_SAGE_DECODE ? a.slots : 0;
     hdr->reserved1 = 0;
   }
 }

@@ -1,4 +1,4 @@
-// sage.cu - 8-bit "Sage" decode over the paged cache.
+// sage.cu - 8-bit "Sage" decode over the paged cache: a score pass, a value pass and a merge.
 //
 // The formula ("FlashInfer PrimTS, Sage Attention 도입으로 8비트 양자화 및 성능
 // 최적화 달성", 코드 분석 item 1, README "Sage attention"):
@@ -8,50 +8,80 @@
 // with the scales applied before the row max and the exponential and sfV in
 // the epilogue (same page, item 4).
 //
-// Quantising p needs the row max m over ALL keys before any P8 is formed.
-// A thread-block cluster of 4 CTAs takes one (request, KV head): CTA q scores
-// the q-th quarter of the keys, keeps its scores in shared memory, and the
-// four CTAs exchange their maxima through distributed shared memory, so every
-// CTA quantises against the exact global m.  Then each CTA streams its V8
-// rows, and the four partial sums are reduced through distributed shared
-// memory by CTA 0, which applies the epilogue.  No score ever reaches HBM and
-// no CTA waits on anything but the cluster barrier (its CTAs are co-scheduled).
+// Quantising p needs the row max m over ALL keys of the row before any P8 is
+// formed, so the work runs in two passes over the plan's CTA slots (a flat,
+// balanced partition of every request's 32-key units, one wave of two CTAs per
+// SM); a CTA takes one slot and one group of HG KV heads:
+//   score pass: S for every key of its items and every query head of the
+//     group, written to the workspace's score rows, and each head's maximum
+//     over each item;
+//   value pass (a programmatic dependent of the score pass): m = the maximum of
+//     the request's item maxima, which is the exact row max; P8 = E4M3(448
+//     exp(S - m)) from the stored S, l = sum exp(S - m), acc = P8 . V8.  A
+//     request covered by one item writes its output; otherwise (acc, l) per item;
+//   merge (a programmatic dependent of the value pass): O = sfV sum_s acc_s /
+//     (448 sum_s l_s) + v_mean.  All items used the same m, so the merge is a
+//     plain sum.
+// The scores cost 4 bytes per key and query head on top of the 128-byte K8 and
+// V8 rows per key and KV head (1/8 more at G = 4); they are written and read
+// back while they are still in L2.
 //
-// Per CTA (4 warps), in 64-key tiles (one 64-slot page each):
-//   QK: S^T[16 keys x 8 heads] = K8[16 x 128] . Q8^T on the INT8 tensor cores
-//       (mma.m16n8k32.s8, exact int32 dot), S = fp32(fp32(sfQ sfK) fp32(dot));
-//   PV: O[16 (G heads used) x 8 d] += P8[16 x 32 keys] . V8[32 keys x 8 d] on
-//       the FP8 tensor cores (mma.m16n8k32.e4m3, fp32 accumulation).  V8 is
-//       key-major in memory; ldmatrix.trans on byte pairs plus one byte
-//       permute gives 4 keys per register, with the keys of a register in a
-//       fixed order that P8's A fragment uses too (the sum over keys does not
-//       depend on their order).
+// Each CTA is one producer warp and eight consumer warps around a 3-stage ring.
+// A tile is 32 slots of one 64-slot page: the producer reads the page ids (and,
+// for the score pass, the K scales) of 32 tiles at once, one per lane, and
+// loads each tile with ONE TMA box {128 B, 32 slots, HG heads} of a 3-D tensor
+// map over the pool [slot][head][128 B], 128-byte swizzled, so shared memory
+// holds [head][slot][128 B] and the ldmatrix reads of 8 consecutive slots hit
+// 8 different bank groups.  In the value pass a second box brings the tile's
+// scores [query head][32 keys] (fp32, swizzled) from the score rows.  Consumer
+// warp w takes KV head w of the group (the value pass spreads a head's 8
+// 16-byte d-blocks over 8 / HG warps when HG < 8):
+//   score: S^T[16 keys x 8 heads] = K8[16 x 128] . Q8^T on the INT8 tensor cores
+//          (mma.m16n8k32.s8, exact int32 dot), S = fp32(fp32(sfQ sfK) fp32(dot));
+//   value: O^T[16 d x 8 heads] += V8^T[16 d x 32 keys] . P8^T on the FP8 tensor
+//          cores (mma.m16n8k32.e4m3, fp32 accumulation); ldmatrix.trans on byte
+//          pairs plus one byte permute gives 4 keys of one d per register, in a
+//          fixed key order that P8's fragment uses too (the sum over keys does
+//          not depend on their order).
+// Rows past the end of a request's last page share its box; their K8 only
+// produce scores that are never stored, and their V8 rows are zeroed in shared
+// memory before use.  Every mbarrier wait is bounded: on timeout the CTA
+// records PA_ERR_DEVICE_INDEX, its roles stop, and the producer waits for the
+// copies it issued before it exits.
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace pa {
 
 namespace {
-constexpr int kThreads = 128;
-constexpr int kClusterCtas = 4;
-constexpr int kTileKeys = 64;                      // = one sfK block = one page
-constexpr int kRowBytes = kHeadDim;                // 8-bit rows: 128 bytes per (slot, head)
-constexpr int kTileBytes = kTileKeys * kRowBytes;  // 8 KB
-constexpr int kStages = 4;
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kStages = 3;
+constexpr int kTileKeys = 32;
+constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2e = 1.4426950408889634f;
-}  // namespace
 
-// Keys of score storage per CTA and head: a quarter of max_kv_len, rounded up to whole tiles.
-int sage_cap(int max_kv_len) {
-  const int per = (max_kv_len + kClusterCtas - 1) / kClusterCtas;
-  return (per + kTileKeys - 1) / kTileKeys * kTileKeys;
-}
-size_t sage_smem_bytes(int G, int cap) {
-  return (size_t)kStages * kTileBytes + (size_t)G * cap * 4 + (32 + 8 + 8) * 4 + (size_t)G * kHeadDim * 4 +
-         (size_t)(cap / kTileKeys) * 8;
-}
-static size_t sage_smem_bytes_max() { return sage_smem_bytes(8, (int)(kSageScoreBudget / (8 * 4))); }
+// What the producer tells the consumers about the tile in a stage.
+struct StageInfo {
+  int kstart;      // first key of the tile
+  int nvalid;      // keys of the item in the tile (1 .. 32)
+  int page;        // the tile's page, -1 if its table entry was bad (nothing loaded)
+  int pad;
+};
 
-namespace {
+template <int HG, int G, bool VPASS>
+struct SageSmem {
+  static constexpr int KV = HG * kTileKeys * kHeadDim;            // [head][slot][128 B]
+  static constexpr int SB = VPASS ? HG * G * kTileKeys * 4 : 0;   // [query head][32] fp32
+  static constexpr int STAGE = (KV + SB + 1023) / 1024 * 1024;
+  static constexpr int OFF_SFK = kStages * STAGE;                              // [k][32] fp32, 128 B each
+  static constexpr int OFF_INFO = OFF_SFK + kStages * 128;
+  static constexpr int OFF_BAR = OFF_INFO + kStages * (int)sizeof(StageInfo);   // full[k], empty[k]
+  static constexpr int OFF_FLAG = OFF_BAR + 2 * kStages * 8;
+  static constexpr int OFF_RED = OFF_FLAG + 16;                                 // [8 warps][8] floats
+  static constexpr int BYTES = OFF_RED + kConsumerWarps * 8 * 4 + 1024;         // + alignment slack
+  static_assert(OFF_BAR % 8 == 0, "barrier alignment");
+};
 
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -61,13 +91,12 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  const uint32_t zero = 0u;   // A rows 8..15 (heads 8..15) are empty for G <= 8
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(zero), "r"(a2), "r"(zero), "r"(b0), "r"(b1));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // Two floats to E4M3 (round to nearest even, saturating); `lo` in the low byte.
@@ -83,31 +112,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-
-// Load a float from CTA `rank`'s shared memory at the address `local` has in this CTA.
-__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
 struct SageLaunch {
-  WsView ws;  // same fields as SageLaunchArgs, with cap in place of max_kv_len
+  CUtensorMap tm_kv;   // K8 (score pass) or V8 (value pass) pool, box {128, 32, HG}
+  CUtensorMap tm_s;    // score rows [B * Hq][score_pitch] fp32, box {32, HG * G}
+  CUtensorMap tm_sfk;  // score pass, HG >= 4: sfK [num_slots / 64][Hkv] fp32, box {HG, 1}
+  WsView ws;
   const int8_t* q8;
   const float* sf_q;
-  const int8_t* k8;
-  const uint8_t* v8;
   const float* sf_k;
   const float* sf_v;
   const float* v_mean;
@@ -115,246 +126,620 @@ struct SageLaunch {
   const int32_t* page_table;
   int64_t pt_pitch;
   uint16_t* out;
-  int batch, hq, hkv, cap;        // cap: score capacity per CTA per head (keys, multiple of 64)
+  int batch, hq, hkv;
 };
 
-template <int G>
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
-sage_decode_kernel(SageLaunch a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* ring = smem;                                             // [kStages][64 keys][128 B]
-  float* S = reinterpret_cast<float*>(smem + kStages * kTileBytes);  // [G][cap]
-  float* red = S + G * a.cap;                                       // [4 warps][8] maxima
-  float* cta_max = red + 32;                                        // [8]
-  float* part_l = cta_max + 8;                                      // [8]
-  float* part_o = part_l + 8;                                       // [G][128]
-  int32_t* tile_page = reinterpret_cast<int32_t*>(part_o + G * kHeadDim);   // [cap / 64] page of each tile
-  float* tile_sfk = reinterpret_cast<float*>(tile_page + a.cap / kTileKeys);  // [cap / 64] its K scale
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const float NEG_INF = -__int_as_float(0x7f800000);
-  PlanHeader* hdr = a.ws.hdr;
-  const bool ok = hdr->magic == kMagic && hdr->mode == PA_MODE_SAGE_DECODE;
-  const int cluster = blockIdx.x / kClusterCtas;
-  const uint32_t rank = cluster_ctarank();
-  const int item = cluster / a.hkv, h_kv = cluster % a.hkv;
-  // Every CTA of a cluster takes the same branch here, so the cluster barriers below always pair up.
-  if (!ok || item >= hdr->num_items) {
-    if (!ok && tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
-    return;
-  }
-  const int4 it = a.ws.items[item];
-  const int r = it.x, L = it.w;
-  const int C = ((L + kClusterCtas - 1) / kClusterCtas + kTileKeys - 1) / kTileKeys * kTileKeys;
-  const int k0 = min((int)rank * C, L), k1 = min(k0 + C, L);
-  const int n_tiles = (k1 - k0 + kTileKeys - 1) / kTileKeys;
-  const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
-  const size_t slot_stride = (size_t)a.hkv * kRowBytes;
-  const uint32_t ring_base = smem_u32(ring);
-
-  // Tile t covers keys k0 + 64 t .. +63, all in one page (k0 is a multiple of 64).  The page
-  // ids and K scales of all this CTA's tiles are read once, up front, so no copy ever waits
-  // on a table read.
-  for (int t = tid; t < n_tiles; t += kThreads) {
-    const int page = __ldg(table + ((k0 + t * kTileKeys) >> 6));
-    const bool good = page >= 0 && ((long long)page + 1) * kTileKeys <= a.num_slots;
-    if (!good) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-    tile_page[t] = good ? page : -1;
-    tile_sfk[t] = good ? __ldg(a.sf_k + (size_t)page * a.hkv + h_kv) : 0.f;
-  }
-  __syncthreads();
-  // 64 rows x 128 B: thread -> chunk (tid % 8) of rows tid / 8 + 16 i
-  auto issue = [&](const uint8_t* pool, int t) {
-    const int stage = t % kStages;
-    const int page = tile_page[t];
-    const uint32_t dst0 = ring_base + stage * kTileBytes;
-    const int c = tid & 7;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = (tid >> 3) + 16 * i;
-      const int j = k0 + t * kTileKeys + row;
-      const bool valid = page >= 0 && j < k1;   // keys past the range read as zero
-      const size_t off = valid ? ((size_t)page * kTileKeys + row) * slot_stride + (size_t)h_kv * kRowBytes + c * 16 : 0;
-      cp_async_16(dst0 + row * kRowBytes + ((c ^ (row & 7)) << 4), pool + off, valid ? 16 : 0);
-    }
-  };
-
-  // ---------------- phase 1: scores into shared memory, per-head maxima
-  uint32_t qb0[4], qb1[4];
-  {
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(a.q8 + ((size_t)r * a.hq + (size_t)h_kv * G + gid) * kHeadDim);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      qb0[ks] = gid < G ? __ldg(qrow + 8 * ks + tig) : 0u;
-      qb1[ks] = gid < G ? __ldg(qrow + 8 * ks + 4 + tig) : 0u;
-    }
-  }
-  const int col0 = 2 * tig, col1 = 2 * tig + 1;           // this thread's head columns of S^T
-  const float sfq0 = col0 < G ? __ldg(a.sf_q + (size_t)r * a.hq + h_kv * G + col0) : 0.f;
-  const float sfq1 = col1 < G ? __ldg(a.sf_q + (size_t)r * a.hq + h_kv * G + col1) : 0.f;
-  const int mat = lane >> 3;
-  const int k_row = warp * 16 + (lane & 7) + ((mat & 1) << 3);
-  float mx0 = NEG_INF, mx1 = NEG_INF;
-
-  for (int t = 0; t < kStages - 1; ++t) {
-    if (t < n_tiles) issue(reinterpret_cast<const uint8_t*>(a.k8), t);
-    cp_async_commit();
-  }
-  for (int t = 0; t < n_tiles; ++t) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (t + kStages - 1 < n_tiles) issue(reinterpret_cast<const uint8_t*>(a.k8), t + kStages - 1);
-    cp_async_commit();
-    const int stage = t % kStages;
-    const uint32_t kst = ring_base + stage * kTileBytes;
-    int acc[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t af[4];
-      const int chunk = 2 * ks + (mat >> 1);
-      ldmatrix_x4(af, kst + k_row * kRowBytes + ((chunk ^ (k_row & 7)) << 4));
-      mma_s8_16832(acc, af, qb0[ks], qb1[ks]);
-    }
-    const float sfk = tile_sfk[t];
-    const int jl0 = t * kTileKeys + warp * 16 + gid, jl1 = jl0 + 8;   // key index within this CTA's range
-    const bool v0 = k0 + jl0 < k1, v1 = k0 + jl1 < k1;
-    // S = fp32(fp32(sfQ sfK) fp32(dot)); the int32 dot is exact and |dot| < 2^24
-    const float s00 = v0 ? (sfq0 * sfk) * (float)acc[0] : NEG_INF;
-    const float s01 = v0 ? (sfq1 * sfk) * (float)acc[1] : NEG_INF;
-    const float s10 = v1 ? (sfq0 * sfk) * (float)acc[2] : NEG_INF;
-    const float s11 = v1 ? (sfq1 * sfk) * (float)acc[3] : NEG_INF;
-    if (col0 < G) {
-      S[col0 * a.cap + jl0] = s00;
-      S[col0 * a.cap + jl1] = s10;
-      mx0 = fmaxf(mx0, fmaxf(s00, s10));
-    }
-    if (col1 < G) {
-      S[col1 * a.cap + jl0] = s01;
-      S[col1 * a.cap + jl1] = s11;
-      mx1 = fmaxf(mx1, fmaxf(s01, s11));
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();                                             // every warp is done with the K8 ring
-  // the first V8 tiles do not depend on the maximum: start them before the exchange
-  for (int t = 0; t < kStages - 1; ++t) {
-    if (t < n_tiles) issue(a.v8, t);
-    cp_async_commit();
-  }
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-  }
-  if (gid == 0) {
-    red[warp * 8 + col0] = mx0;
-    red[warp * 8 + col1] = mx1;
-  }
-  __syncthreads();
-  if (tid < 8) cta_max[tid] = fmaxf(fmaxf(red[tid], red[8 + tid]), fmaxf(red[16 + tid], red[24 + tid]));
-  cluster_sync();                                              // #1: every CTA's maxima are visible
-
-  // ---------------- phase 2: P8 = E4M3(448 exp(S - m)), l, and O = P8 . V8
-  // This thread forms P8 for head gid (gid < G) at the keys {2tig, 2tig+1, 8+2tig, 9+2tig}
-  // (+16) of each 32-key step: the key order the V8 fragments below come in.
-  float m_h = NEG_INF;
-  if (gid < G)
-    for (uint32_t q = 0; q < kClusterCtas; ++q) m_h = fmaxf(m_h, ld_dsmem_f32(cta_max + gid, q));
-  const float m_use = m_h == NEG_INF ? 0.f : m_h;
-  const float* Sh = S + (gid < G ? gid : 0) * a.cap;
-  float lsum = 0.f;
-  float oe[2][4], oo[2][4];          // d-blocks 2 warp and 2 warp + 1: even / odd d columns
-#pragma unroll
-  for (int b = 0; b < 2; ++b)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) oe[b][i] = oo[b][i] = 0.f;
-
-  for (int t = 0; t < n_tiles; ++t) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (t + kStages - 1 < n_tiles) issue(a.v8, t + kStages - 1);
-    cp_async_commit();
-    const uint32_t vst = ring_base + (t % kStages) * kTileBytes;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t pa0 = 0u, pa2 = 0u;
-      if (gid < G) {
-        const int base = t * kTileKeys + 32 * ks;
-        float p[8];
-        const int keys[8] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig,
-                             16 + 2 * tig, 17 + 2 * tig, 24 + 2 * tig, 25 + 2 * tig};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int jl = base + keys[i];
-          const float sv = k0 + jl < k1 ? Sh[jl] : NEG_INF;
-          p[i] = ex2((sv - m_use) * kLog2e);                  // exp(S - m), 0 for masked keys
-          lsum += p[i];
-        }
-        pa0 = e4m3x2(448.f * p[0], 448.f * p[1]) | (e4m3x2(448.f * p[2], 448.f * p[3]) << 16);
-        pa2 = e4m3x2(448.f * p[4], 448.f * p[5]) | (e4m3x2(448.f * p[6], 448.f * p[7]) << 16);
-      }
-#pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const int db = 2 * warp + b;                          // 16-byte d-block of this warp
-        const int vkey = 32 * ks + 8 * mat + (lane & 7);
-        uint32_t vr[4];
-        ldmatrix_x4_trans(vr, vst + vkey * kRowBytes + ((db ^ (vkey & 7)) << 4));
-        const uint32_t be0 = prmt(vr[0], vr[1], 0x6420), bo0 = prmt(vr[0], vr[1], 0x7531);
-        const uint32_t be1 = prmt(vr[2], vr[3], 0x6420), bo1 = prmt(vr[2], vr[3], 0x7531);
-        mma_e4m3_16832(oe[b], pa0, pa2, be0, be1);
-        mma_e4m3_16832(oo[b], pa0, pa2, bo0, bo1);
-      }
-    }
-  }
-  cp_async_wait<0>();
-  // l for head gid: every warp formed the same probabilities; warp 0's sum is used
-  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-  if (warp == 0 && tig == 0 && gid < G) part_l[gid] = lsum;
-  if (gid < G) {
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const int d = 16 * (2 * warp + b) + 4 * tig;
-      float* row = part_o + gid * kHeadDim;
-      row[d] = oe[b][0];
-      row[d + 2] = oe[b][1];
-      row[d + 1] = oo[b][0];
-      row[d + 3] = oo[b][1];
-    }
-  }
-  cluster_sync();                                              // #2: partials are visible
-
-  if (rank == 0) {
-    for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-      const int h = idx / kHeadDim, d = idx % kHeadDim;
-      float acc = 0.f, l = 0.f;
-      for (uint32_t q = 0; q < kClusterCtas; ++q) {
-        acc += ld_dsmem_f32(part_o + idx, q);
-        l += ld_dsmem_f32(part_l + h, q);
-      }
-      const float vm = a.v_mean ? __ldg(a.v_mean + (size_t)h_kv * kHeadDim + d) : 0.f;
-      const float sfv = __ldg(a.sf_v + (size_t)h_kv * kHeadDim + d);
-      const float o = l > 0.f ? sfv * acc / (448.f * l) + vm : vm;
-      a.out[((size_t)r * a.hq + h_kv * G + h) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-    }
-  }
-  cluster_sync();                                              // #3: CTA 0 is done reading the others
+__device__ __forceinline__ bool sage_ws_ok(const PlanHeader* hdr) {
+  return hdr->magic == kMagic && hdr->mode == PA_MODE_SAGE_DECODE;
 }
 
-template <int G>
-cudaError_t launch_sage_g(const SageLaunch& a, size_t smem, cudaStream_t s) {
+// The items of this CTA's slot: [first, last).
+__device__ __forceinline__ bool slot_items(const SageLaunch& a, int groups, int& first, int& last) {
+  const int slot = blockIdx.x / groups;
+  if (slot >= a.ws.hdr->slots) return false;
+  first = a.ws.slot_first[slot];
+  last = min(a.ws.slot_first[slot + 1], a.ws.hdr->num_items);
+  return first < last;
+}
+
+// Item metadata of a slot, 32 items at a time, one item per lane; every warp keeps its own
+// window, so no role waits on a chain of dependent reads at an item boundary.
+struct ItemWindow {
+  int w0 = -1 << 30;
+  int r = 0, kv0 = 0, kv1 = 0, base = 0, splits = 0;   // item w0 + lane
+  __device__ __forceinline__ void load(const SageLaunch& a, int w, int last, bool with_req) {
+    w0 = w;
+    const int i = w + (threadIdx.x & 31);
+    r = kv0 = kv1 = base = splits = 0;
+    if (i < last) {
+      const int4 it = a.ws.items[i];
+      r = it.x;
+      kv0 = it.z;
+      kv1 = it.w;
+      if (with_req) {
+        base = a.ws.req_base[r];
+        splits = min(a.ws.req_splits[r], a.ws.hdr->max_items - base);   // clamped only after a flagged overflow
+      }
+    }
+  }
+  // item i (the same i on every lane): request, key range, first item and item count of its request
+  __device__ __forceinline__ void get(const SageLaunch& a, int i, int last, bool with_req, int& ri, int& k0, int& k1,
+                                      int& bi, int& si) {
+    if (i < w0 || i >= w0 + 32) load(a, i, last, with_req);
+    const int l = i - w0;
+    ri = __shfl_sync(0xffffffffu, r, l);
+    k0 = __shfl_sync(0xffffffffu, kv0, l);
+    k1 = __shfl_sync(0xffffffffu, kv1, l);
+    bi = __shfl_sync(0xffffffffu, base, l);
+    si = __shfl_sync(0xffffffffu, splits, l);
+  }
+};
+
+// Shared-memory handles of one CTA.
+template <int HG, int G, bool VPASS>
+struct Ring {
+  using L = SageSmem<HG, G, VPASS>;
+  uint32_t base;
+  uint8_t* ptr;
+  __device__ __forceinline__ Ring() {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    base = (raw + 1023u) & ~1023u;
+    ptr = smem_raw + (base - raw);
+  }
+  __device__ __forceinline__ uint32_t stage(int s) const { return base + s * L::STAGE; }
+  __device__ __forceinline__ uint32_t full(int s) const { return base + L::OFF_BAR + 8 * s; }
+  __device__ __forceinline__ uint32_t empty(int s) const { return base + L::OFF_BAR + 8 * (kStages + s); }
+  __device__ __forceinline__ StageInfo* info() const { return reinterpret_cast<StageInfo*>(ptr + L::OFF_INFO); }
+  // score pass: sfK of stage s's page for each head of the group (128-byte aligned: a TMA target)
+  __device__ __forceinline__ float* sfk(int s) const { return reinterpret_cast<float*>(ptr + L::OFF_SFK + 128 * s); }
+  __device__ __forceinline__ volatile int* abort_flag() const {
+    return reinterpret_cast<volatile int*>(ptr + L::OFF_FLAG);
+  }
+  __device__ __forceinline__ float* red() const { return reinterpret_cast<float*>(ptr + L::OFF_RED); }
+  __device__ __forceinline__ void init() const {
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(full(s), 1);
+        mbar_init(empty(s), kConsumerWarps);
+      }
+      *abort_flag() = 0;
+      mbar_fence_init();
+    }
+    __syncthreads();
+  }
+  // bounded, warp-uniform wait: every lane observes the phase itself, the warp agrees on
+  // the outcome; false (and the CTA-wide abort flag set) if the phase never completes
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, PlanHeader* hdr) const {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+      const bool done = mbar_try_wait(bar, parity);
+      if (__all_sync(0xffffffffu, done)) return true;
+      if (__any_sync(0xffffffffu, *abort_flag() != 0)) return false;
+    }
+    if ((threadIdx.x & 31) == 0) {
+      *abort_flag() = 1;
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+    }
+    return false;
+  }
+};
+
+// The producer warp: page ids of 32 tiles per round, one per lane, then one TMA box per tile;
+// in the score pass also the page's K scales (one box {HG, 1} when HG >= 4, which keeps a
+// dependent global read off the path to the first copy; else read by the lanes), in the
+// value pass one box of the tile's scores.  The value pass requests the V8 of its first
+// kStages tiles before it waits for the score pass, their scores after.
+template <int HG, int G, bool VPASS>
+__device__ __forceinline__ void produce(const SageLaunch& a, const Ring<HG, G, VPASS>& rg, int first, int last,
+                                        int grp) {
+  using L = SageSmem<HG, G, VPASS>;
+  const int lane = threadIdx.x & 31;
+  PlanHeader* hdr = a.ws.hdr;
+  StageInfo* info = rg.info();
+  uint32_t q = 0;   // ring uses so far
+  bool ok = true;
+  bool waited = !VPASS;
+  int pend_n = 0, pend_x[kStages], pend_y[kStages];   // value pass: deferred score boxes (lane 0)
+  auto flush = [&]() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the score pass has completed
+    if (lane == 0)
+      for (int k = 0; k < pend_n; ++k)
+        tma_load_2d(rg.stage(k) + L::KV, &a.tm_s, pend_x[k], pend_y[k], rg.full(k));
+    waited = true;
+  };
+  ItemWindow win;
+  // raw table entry of tile tb + lane of an item (or -1 past its tiles); checked when used
+  auto entry = [&](int r, int kv0, int n_tiles, int tb) -> int {
+    const int t = tb + lane;
+    return t < n_tiles ? __ldg(a.page_table + (size_t)r * a.pt_pitch + ((kv0 + kTileKeys * t) >> 6)) : -1;
+  };
+  int r = 0, kv0 = 0, kv1 = 0, b_, s_;
+  if (first < last) win.get(a, first, last, false, r, kv0, kv1, b_, s_);
+  int e_pre = entry(r, kv0, (kv1 - kv0 + kTileKeys - 1) / kTileKeys, 0);   // first round of the next item
+  for (int item = first; item < last && ok; ++item) {
+    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    const int srow = r * a.hq + grp * HG * G;
+    int rn = 0, kv0n = 0, kv1n = 0;
+    if (item + 1 < last) win.get(a, item + 1, last, false, rn, kv0n, kv1n, b_, s_);
+    const int n_tiles_n = (kv1n - kv0n + kTileKeys - 1) / kTileKeys;
+    if (n_tiles == 0 && item + 1 < last) e_pre = entry(rn, kv0n, n_tiles_n, 0);   // an empty item has no round
+    for (int tb = 0; tb < n_tiles && ok; tb += 32) {
+      const int e = tb == 0 ? e_pre : entry(r, kv0, n_tiles, tb);
+      // the next item's first page ids, read behind this item's last round
+      if (tb + 32 >= n_tiles && item + 1 < last) e_pre = entry(rn, kv0n, n_tiles_n, 0);
+      int pg = -1;
+      if (tb + lane < n_tiles) {
+        if (e >= 0 && ((long long)e + 1) * kSageBlock <= a.num_slots) pg = e;
+        else set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      }
+      constexpr bool kSfkLanes = !VPASS && HG < 4;   // K scales read by the lanes
+      float sfk[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+        sfk[h] = kSfkLanes && pg >= 0 ? __ldg(a.sf_k + (size_t)pg * a.hkv + grp * HG + h) : 0.f;
+      const int nt = min(32, n_tiles - tb);
+      for (int i = 0; i < nt; ++i, ++q) {
+        const int s = q % kStages;
+        if (VPASS && !waited && q == kStages) flush();
+        if (q >= kStages && !rg.wait(rg.empty(s), ((q / kStages) - 1) & 1, hdr)) {
+          ok = false;
+          break;
+        }
+        const int p = __shfl_sync(0xffffffffu, pg, i);
+        float sf[HG];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) sf[h] = __shfl_sync(0xffffffffu, sfk[h], i);
+        if (lane == 0) {
+          const int ks = kv0 + kTileKeys * (tb + i);
+          StageInfo& in = info[s];
+          in.kstart = ks;
+          in.nvalid = min(kTileKeys, kv1 - ks);
+          in.page = p;
+          if (kSfkLanes) {
+#pragma unroll
+            for (int h = 0; h < HG; ++h) rg.sfk(s)[h] = sf[h];
+          }
+          const bool sfk_box = !VPASS && !kSfkLanes && p >= 0;
+          mbar_expect_tx(rg.full(s), (p >= 0 ? L::KV : 0) + L::SB + (sfk_box ? HG * 4 : 0));
+          if (p >= 0) tma_load_3d(rg.stage(s), &a.tm_kv, 0, p * kSageBlock + (ks & (kSageBlock - 1)), grp * HG, rg.full(s));
+          if (sfk_box) tma_load_2d(smem_u32(rg.sfk(s)), &a.tm_sfk, grp * HG, p, rg.full(s));
+          if (VPASS) {
+            if (waited) {
+              tma_load_2d(rg.stage(s) + L::KV, &a.tm_s, ks, srow, rg.full(s));
+            } else {
+              pend_x[pend_n] = ks;
+              pend_y[pend_n] = srow;
+              ++pend_n;
+            }
+          }
+        }
+      }
+    }
+    r = rn;
+    kv0 = kv0n;
+    kv1 = kv1n;
+  }
+  if (VPASS && !waited) flush();
+  if (!ok && lane == 0) {
+    // drain: wait (bounded) for the copies this warp issued into the last kStages uses
+    const uint32_t q0 = q > (uint32_t)kStages ? q - kStages : 0;
+    for (uint32_t u = q0; u < q; ++u)
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(rg.full(u % kStages), (u / kStages) & 1); ++i) {}
+  }
+}
+
+// ---------------------------------------------------------------- score pass
+template <int HG, int G>
+__global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_constant__ SageLaunch a) {
+  // the value pass (a programmatic dependent) may be scheduled now; it waits for this
+  // whole grid to finish before it reads the scores
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tig = lane & 3, mat = lane >> 3;
+  PlanHeader* hdr = a.ws.hdr;
+  if (!sage_ws_ok(hdr)) {
+    if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
+    return;
+  }
+  const int groups = a.hkv / HG, grp = blockIdx.x % groups;
+  int first = 0, last = 0;
+  if (!slot_items(a, groups, first, last)) return;
+  Ring<HG, G, false> rg;
+  rg.init();
+  if (warp == kConsumerWarps) {
+    produce<HG, G, false>(a, rg, first, last, grp);
+    return;
+  }
+  // consumer warp `warp` owns KV head `warp` of the group (warps HG.. idle when HG < 8)
+  const bool active = warp < HG;
+  const int hl = active ? warp : 0;
+  const int hkv = grp * HG + hl;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const StageInfo* info = rg.info();
+  const int c0 = 2 * tig, c1 = 2 * tig + 1;          // this thread's query-head columns of S^T
+  // Q8^T as the B operand: b0 = Q8[head gid][32 ks + 4 tig .. +3], b1 = the same at +16; the
+  // next item's are read while this item's tiles are processed
+  uint32_t qn0[4], qn1[4];
+  float sfqn0 = 0.f, sfqn1 = 0.f;
+  auto load_q = [&](int rq) {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(a.q8 + ((size_t)rq * a.hq + (size_t)hkv * G + gid) * kHeadDim);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      qn0[ks] = active && gid < G ? __ldg(qrow + 8 * ks + tig) : 0u;
+      qn1[ks] = active && gid < G ? __ldg(qrow + 8 * ks + 4 + tig) : 0u;
+    }
+    sfqn0 = active && c0 < G ? __ldg(a.sf_q + (size_t)rq * a.hq + (size_t)hkv * G + c0) : 0.f;
+    sfqn1 = active && c1 < G ? __ldg(a.sf_q + (size_t)rq * a.hq + (size_t)hkv * G + c1) : 0.f;
+  };
+  ItemWindow win;
+  int rn = 0, kv0n = 0, kv1n = 0, b_, s_;
+  win.get(a, first, last, false, rn, kv0n, kv1n, b_, s_);
+  load_q(rn);
+  uint32_t q = 0;
+  for (int item = first; item < last; ++item) {
+    const int r = rn, kv0 = kv0n, kv1 = kv1n;
+    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    uint32_t qb0[4], qb1[4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      qb0[ks] = qn0[ks];
+      qb1[ks] = qn1[ks];
+    }
+    const float sfq0 = sfqn0, sfq1 = sfqn1;
+    if (item + 1 < last) {
+      win.get(a, item + 1, last, false, rn, kv0n, kv1n, b_, s_);
+      load_q(rn);
+    }
+    float* srow0 = a.ws.scores + ((size_t)r * a.hq + (size_t)hkv * G + (c0 < G ? c0 : 0)) * a.ws.score_pitch;
+    float* srow1 = a.ws.scores + ((size_t)r * a.hq + (size_t)hkv * G + (c1 < G ? c1 : 0)) * a.ws.score_pitch;
+    float mx0 = NEG_INF, mx1 = NEG_INF;
+    for (int t = 0; t < n_tiles; ++t, ++q) {
+      const int s = q % kStages;
+      if (!rg.wait(rg.full(s), (q / kStages) & 1, hdr)) return;
+      const int ks0 = info[s].kstart, page = info[s].page;
+      if (active && page >= 0) {
+        const float sfk = rg.sfk(s)[hl];
+        const float sc0 = sfq0 * sfk, sc1 = sfq1 * sfk;      // fp32(sfQ sfK)
+        const uint32_t kst = rg.stage(s) + hl * kTileKeys * kHeadDim;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          const int row = 16 * kb + (lane & 7) + ((mat & 1) << 3);
+          int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            uint32_t af[4];
+            const int chunk = 2 * kk + (mat >> 1);
+            ldmatrix_x4(af, kst + row * kHeadDim + ((chunk ^ (row & 7)) << 4));
+            mma_s8_16832(acc, af, qb0[kk], qb1[kk]);
+          }
+          const int key0 = ks0 + 16 * kb + gid, key1 = key0 + 8;
+          // S = fp32(fp32(sfQ sfK) fp32(dot)); the int32 dot is exact and |dot| < 2^24
+          const float s00 = sc0 * (float)acc[0], s01 = sc1 * (float)acc[1];
+          const float s10 = sc0 * (float)acc[2], s11 = sc1 * (float)acc[3];
+          if (c0 < G) {
+            if (key0 < kv1) { srow0[key0] = s00; mx0 = fmaxf(mx0, s00); }
+            if (key1 < kv1) { srow0[key1] = s10; mx0 = fmaxf(mx0, s10); }
+          }
+          if (c1 < G) {
+            if (key0 < kv1) { srow1[key0] = s01; mx1 = fmaxf(mx1, s01); }
+            if (key1 < kv1) { srow1[key1] = s11; mx1 = fmaxf(mx1, s11); }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rg.empty(s));
+    }
+    // this head's maxima over the item (the 8 key rows of the fragments)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    if (active && gid == 0) {
+      float* im = a.ws.item_max + (size_t)item * a.hq + (size_t)hkv * G;
+      if (c0 < G) im[c0] = mx0;
+      if (c1 < G) im[c1] = mx1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- value pass
+// two CTAs per SM where their shared memory fits (G = 8 with HG = 8 takes one)
+template <int HG, int G>
+__global__ void __launch_bounds__(kThreads, 2 * SageSmem<HG, G, true>::BYTES <= 227 * 1024 ? 2 : 1)
+    sage_value_kernel(const __grid_constant__ SageLaunch a) {
+  using L = SageSmem<HG, G, true>;
+  constexpr int WPH = kConsumerWarps / HG;   // warps per KV head
+  constexpr int NDB = 8 / WPH;               // 16-byte d-blocks per warp
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");   // lets the merge be scheduled
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  PlanHeader* hdr = a.ws.hdr;
+  if (!sage_ws_ok(hdr)) return;   // the score pass has flagged it
+  const int groups = a.hkv / HG, grp = blockIdx.x % groups;
+  int first = 0, last = 0;
+  if (!slot_items(a, groups, first, last)) return;
+  Ring<HG, G, true> rg;
+  rg.init();
+  if (warp == kConsumerWarps) {
+    produce<HG, G, true>(a, rg, first, last, grp);
+    return;
+  }
+  const int hl = warp % HG, db0 = (warp / HG) * NDB;
+  const int hkv = grp * HG + hl;
+  const bool p_lane = gid < G;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const StageInfo* info = rg.info();
+  float* mw = rg.red() + warp * 8;
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the score pass has completed and its writes are visible
+  // m for the G query heads of this KV head is the maximum of the request's item maxima: each
+  // lane reads those of items base + lane, base + lane + 32, ...; the first 32 of the next
+  // item's request are read while this item's tiles are processed
+  float mv[G];
+  auto load_m = [&](int b, int sp) {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      mv[g] = lane < sp ? __ldcg(a.ws.item_max + (size_t)(b + lane) * a.hq + (size_t)hkv * G + g) : NEG_INF;
+  };
+  ItemWindow win;
+  int rn = 0, kv0n = 0, kv1n = 0, basen = 0, splitsn = 0;
+  win.get(a, first, last, true, rn, kv0n, kv1n, basen, splitsn);
+  load_m(basen, splitsn);
+  uint32_t q = 0;
+  for (int item = first; item < last; ++item) {
+    const int r = rn, kv0 = kv0n, kv1 = kv1n, base = basen, splits = splitsn;
+    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    {
+      float m[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) m[g] = mv[g];
+      for (int sp = lane + 32; sp < splits; sp += 32) {   // requests of more than 32 items
+#pragma unroll
+        for (int g = 0; g < G; ++g) m[g] = fmaxf(m[g], __ldcg(a.ws.item_max + (size_t)(base + sp) * a.hq + (size_t)hkv * G + g));
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m[g] = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], off));
+        if (lane == 0) mw[g] = m[g] == NEG_INF ? 0.f : m[g];
+      }
+    }
+    __syncwarp();
+    if (item + 1 < last) {
+      win.get(a, item + 1, last, true, rn, kv0n, kv1n, basen, splitsn);
+      load_m(basen, splitsn);
+    }
+    const float m_use = p_lane ? mw[gid] : 0.f;
+    float o[NDB][4];
+#pragma unroll
+    for (int b = 0; b < NDB; ++b) o[b][0] = o[b][1] = o[b][2] = o[b][3] = 0.f;
+    float lsum = 0.f;
+    const int srow = hl * G + (p_lane ? gid : 0);   // this lane's row of the stage's score box
+    for (int t = 0; t < n_tiles; ++t, ++q) {
+      const int s = q % kStages;
+      if (!rg.wait(rg.full(s), (q / kStages) & 1, hdr)) return;
+      const uint32_t vst = rg.stage(s) + hl * kTileKeys * kHeadDim;
+      const int nv = info[s].page >= 0 ? info[s].nvalid : 0;   // keys of the item in this tile
+      if (nv < kTileKeys) {
+        // rows past the item (or of a page that was not loaded) become zero in this warp's d-blocks
+        uint8_t* vp = rg.ptr + (vst - rg.base);
+        for (int idx = lane; idx < (kTileKeys - nv) * NDB; idx += 32) {
+          const int row = nv + idx / NDB, chunk = db0 + idx % NDB;
+          *reinterpret_cast<uint4*>(vp + row * kHeadDim + ((chunk ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      // P8 for query head gid at the keys {2tig, 2tig+1, 8+2tig, 9+2tig} (+16): the key order
+      // of the V8 fragments below
+      uint32_t pb0 = 0u, pb1 = 0u;
+      if (p_lane) {
+        const uint8_t* sp = rg.ptr + (rg.stage(s) - rg.base) + L::KV + srow * 128;
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int key = 2 * tig + 8 * i;
+          const float2 sv = *reinterpret_cast<const float2*>(sp + (((key >> 2) ^ (srow & 7)) << 4) + (key & 3) * 4);
+          const float sx = key < nv ? sv.x : NEG_INF;
+          const float sy = key + 1 < nv ? sv.y : NEG_INF;
+          p[2 * i] = ex2((sx - m_use) * kLog2e);      // exp(S - m), 0 for masked keys
+          p[2 * i + 1] = ex2((sy - m_use) * kLog2e);
+          lsum += p[2 * i] + p[2 * i + 1];
+        }
+        pb0 = e4m3x2(448.f * p[0], 448.f * p[1]) | (e4m3x2(448.f * p[2], 448.f * p[3]) << 16);
+        pb1 = e4m3x2(448.f * p[4], 448.f * p[5]) | (e4m3x2(448.f * p[6], 448.f * p[7]) << 16);
+      }
+#pragma unroll
+      for (int b = 0; b < NDB; ++b) {
+        const int db = db0 + b;
+        uint32_t vr[4];
+        ldmatrix_x4_trans(vr, vst + lane * kHeadDim + ((db ^ (lane & 7)) << 4));
+        uint32_t af[4];
+        af[0] = prmt(vr[0], vr[1], 0x6420);   // d = 16 db + 2 gid,     keys 0-15
+        af[1] = prmt(vr[0], vr[1], 0x7531);   // d = 16 db + 2 gid + 1, keys 0-15
+        af[2] = prmt(vr[2], vr[3], 0x6420);   // keys 16-31
+        af[3] = prmt(vr[2], vr[3], 0x7531);
+        mma_e4m3_16832(o[b], af, pb0, pb1);
+      }
+      if (nv < kTileKeys) fence_proxy_async();   // the zeroing writes before the next TMA into this stage
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rg.empty(s));
+    }
+    // l of query head gid (summed over the 4 lanes that split its keys), then per column
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+    const float l0 = __shfl_sync(0xffffffffu, lsum, (2 * tig) * 4);
+    const float l1 = __shfl_sync(0xffffffffu, lsum, (2 * tig + 1) * 4);
+    const int c0 = 2 * tig, c1 = 2 * tig + 1;          // this thread's query-head columns of O^T
+    if (splits == 1) {
+#pragma unroll
+      for (int b = 0; b < NDB; ++b) {
+        const int d = 16 * (db0 + b) + 2 * gid;
+        const float2 sfv = *reinterpret_cast<const float2*>(a.sf_v + (size_t)hkv * kHeadDim + d);
+        const float2 vm = a.v_mean ? *reinterpret_cast<const float2*>(a.v_mean + (size_t)hkv * kHeadDim + d)
+                                   : make_float2(0.f, 0.f);
+        if (c0 < G) {
+          const float inv = l0 > 0.f ? 1.f / (448.f * l0) : 0.f;
+          *reinterpret_cast<uint32_t*>(a.out + ((size_t)r * a.hq + (size_t)hkv * G + c0) * kHeadDim + d) =
+              pack_bf16x2(sfv.x * o[b][0] * inv + vm.x, sfv.y * o[b][2] * inv + vm.y);
+        }
+        if (c1 < G) {
+          const float inv = l1 > 0.f ? 1.f / (448.f * l1) : 0.f;
+          *reinterpret_cast<uint32_t*>(a.out + ((size_t)r * a.hq + (size_t)hkv * G + c1) * kHeadDim + d) =
+              pack_bf16x2(sfv.x * o[b][1] * inv + vm.x, sfv.y * o[b][3] * inv + vm.y);
+        }
+      }
+    } else {
+      const size_t prow = (size_t)item * a.hq + (size_t)hkv * G;
+#pragma unroll
+      for (int b = 0; b < NDB; ++b) {
+        const int d = 16 * (db0 + b) + 2 * gid;
+        if (c0 < G) *reinterpret_cast<float2*>(a.ws.partial_o + (prow + c0) * kHeadDim + d) = make_float2(o[b][0], o[b][2]);
+        if (c1 < G) *reinterpret_cast<float2*>(a.ws.partial_o + (prow + c1) * kHeadDim + d) = make_float2(o[b][1], o[b][3]);
+      }
+      if (db0 == 0 && tig == 0 && p_lane) a.ws.partial_lse[prow + gid] = lsum;
+    }
+  }
+}
+
+// One warp per (request, query head) of a request that was split:
+// O = sfV sum_s acc_s / (448 sum_s l_s) + v_mean.  Each lane owns 4 of the 128 outputs and
+// issues the loads of 8 items before it adds them (in item order).
+__global__ void __launch_bounds__(256) sage_merge_kernel(const __grid_constant__ SageLaunch a) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the value pass has completed
+  PlanHeader* hdr = a.ws.hdr;
+  if (!sage_ws_ok(hdr)) return;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (gw >= a.batch * a.hq) return;
+  const int r = gw / a.hq, h = gw % a.hq;
+  const int splits = a.ws.req_splits[r];
+  if (splits <= 1) return;
+  const int base = a.ws.req_base[r];
+  if (base + splits > hdr->max_items) return;
+  const int h_kv = h / (a.hq / a.hkv);
+  const float4 sfv = __ldg(reinterpret_cast<const float4*>(a.sf_v + (size_t)h_kv * kHeadDim) + lane);
+  const float4 vm = a.v_mean ? __ldg(reinterpret_cast<const float4*>(a.v_mean + (size_t)h_kv * kHeadDim) + lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* po = reinterpret_cast<const float4*>(a.ws.partial_o + ((size_t)base * a.hq + h) * kHeadDim) + lane;
+  const float* pl = a.ws.partial_lse + (size_t)base * a.hq + h;
+  const size_t row4 = (size_t)a.hq * kHeadDim / 4;   // float4s from one item's row to the next
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float l = 0.f;
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float4 v[8];
+    float lv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = s0 + j < splits;
+      v[j] = in ? __ldcg(po + (size_t)(s0 + j) * row4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      lv[j] = in ? __ldcg(pl + (size_t)(s0 + j) * a.hq) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      acc.x += v[j].x;
+      acc.y += v[j].y;
+      acc.z += v[j].z;
+      acc.w += v[j].w;
+      l += lv[j];
+    }
+  }
+  const float inv = l > 0.f ? 1.f / (448.f * l) : 0.f;
+  uint2 packed;
+  packed.x = pack_bf16x2(sfv.x * acc.x * inv + vm.x, sfv.y * acc.y * inv + vm.y);
+  packed.y = pack_bf16x2(sfv.z * acc.z * inv + vm.z, sfv.w * acc.w * inv + vm.w);
+  reinterpret_cast<uint2*>(a.out + ((size_t)r * a.hq + h) * kHeadDim)[lane] = packed;
+}
+
+cudaError_t launch_pdl(void (*kernel)(const SageLaunch), dim3 grid, dim3 block, size_t smem, const SageLaunch& a,
+                       cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// [num_slots][hkv][128] bytes as 3-D {128, slots, heads}; box {128, 32, HG}, 128-byte swizzle
+bool encode_pool(CUtensorMap* tm, const void* ptr, int64_t num_slots, int hkv, int hg) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)num_slots, (cuuint64_t)hkv};
+  const cuuint64_t strides[2] = {(cuuint64_t)hkv * 128, 128};
+  const cuuint32_t box[3] = {128, (cuuint32_t)kTileKeys, (cuuint32_t)hg};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// score rows [rows][pitch] fp32 as 2-D {pitch, rows}; box {32, box_rows}, 128-byte swizzle
+bool encode_scores(CUtensorMap* tm, const float* ptr, int64_t pitch, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)pitch, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)kTileKeys, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// sfK [pages][hkv] fp32 as 2-D {hkv, pages}; box {hg, 1}
+bool encode_sfk(CUtensorMap* tm, const float* ptr, int64_t pages, int hkv, int hg) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)hkv, (cuuint64_t)pages};
+  const cuuint64_t strides[1] = {(cuuint64_t)hkv * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)hg, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HG, int G>
+cudaError_t launch_sage_hg(SageLaunch& a, const int8_t* k8, const uint8_t* v8, int slots, cudaStream_t s) {
+  using LS = SageSmem<HG, G, false>;
+  using LV = SageSmem<HG, G, true>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sage_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sage_smem_bytes_max());
+    cudaError_t e = cudaFuncSetAttribute(sage_score_kernel<HG, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         LS::BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sage_value_kernel<HG, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, LV::BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  sage_decode_kernel<G><<<a.batch * a.hkv * kClusterCtas, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  const dim3 grid(slots * (a.hkv / HG));
+  if (!encode_scores(&a.tm_s, a.ws.scores, a.ws.score_pitch, (int64_t)a.batch * a.hq, HG * G) ||
+      !encode_pool(&a.tm_kv, k8, a.num_slots, a.hkv, HG) ||
+      (HG >= 4 && !encode_sfk(&a.tm_sfk, a.sf_k, a.num_slots / kSageBlock, a.hkv, HG)))
+    return cudaErrorInvalidValue;
+  sage_score_kernel<HG, G><<<grid, kThreads, LS::BYTES, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (!encode_pool(&a.tm_kv, v8, a.num_slots, a.hkv, HG)) return cudaErrorInvalidValue;
+  e = launch_pdl(sage_value_kernel<HG, G>, grid, dim3(kThreads), LV::BYTES, a, s);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(sage_merge_kernel, dim3((a.batch * a.hq + 7) / 8), dim3(256), 0, a, s);
+}
+
+template <int G>
+cudaError_t launch_sage_g(SageLaunch& a, const int8_t* k8, const uint8_t* v8, int slots, cudaStream_t s) {
+  switch (decode_heads_per_cta(a.hkv)) {
+    case 8: return launch_sage_hg<8, G>(a, k8, v8, slots, s);
+    case 4: return launch_sage_hg<4, G>(a, k8, v8, slots, s);
+    case 2: return launch_sage_hg<2, G>(a, k8, v8, slots, s);
+    default: return launch_sage_hg<1, G>(a, k8, v8, slots, s);
+  }
 }
 
 }  // namespace
@@ -364,8 +749,6 @@ cudaError_t launch_sage(const SageLaunchArgs& in, cudaStream_t s) {
   a.ws = in.ws;
   a.q8 = in.q8;
   a.sf_q = in.sf_q;
-  a.k8 = in.k8;
-  a.v8 = in.v8;
   a.sf_k = in.sf_k;
   a.sf_v = in.sf_v;
   a.v_mean = in.v_mean;
@@ -376,14 +759,11 @@ cudaError_t launch_sage(const SageLaunchArgs& in, cudaStream_t s) {
   a.batch = in.batch;
   a.hq = in.hq;
   a.hkv = in.hkv;
-  a.cap = sage_cap(in.max_kv_len);
-  const int G = in.hq / in.hkv;
-  const size_t smem = sage_smem_bytes(G, a.cap);
-  switch (G) {
-    case 1: return launch_sage_g<1>(a, smem, s);
-    case 2: return launch_sage_g<2>(a, smem, s);
-    case 4: return launch_sage_g<4>(a, smem, s);
-    case 8: return launch_sage_g<8>(a, smem, s);
+  switch (in.hq / in.hkv) {
+    case 1: return launch_sage_g<1>(a, in.k8, in.v8, in.slots, s);
+    case 2: return launch_sage_g<2>(a, in.k8, in.v8, in.slots, s);
+    case 4: return launch_sage_g<4>(a, in.k8, in.v8, in.slots, s);
+    case 8: return launch_sage_g<8>(a, in.k8, in.v8, in.slots, s);
     default: return cudaErrorInvalidValue;
   }
 }

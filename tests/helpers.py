@@ -47,7 +47,8 @@ def sage_row_rel_error(gpu_bf16, ref):
     return float(np.max(num / den))
 
 
-def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 128, hkv: int = 8):
+def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 128, hkv: int = 8,
+               max_kv_len: int = 0, slots: int = 0):
     """Byte offsets of the workspace arrays, from the layout documented at attn_plan."""
     off = 64
     o = {}
@@ -59,12 +60,24 @@ def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 1
     o["items"] = off
     off += 16 * max_items
     off = (off + 255) // 256 * 256
-    if mode == 0:
+    if mode == 2:
+        o["slot_first"] = off
+        off += 4 * (slots + 1)
+        off = (off + 255) // 256 * 256
+    if mode in (0, 2):
         o["partial_o"] = off
         off += 4 * max_items * hq * head_dim
         off = (off + 255) // 256 * 256
         o["partial_lse"] = off
         off += 4 * max_items * hq
+        off = (off + 255) // 256 * 256
+    if mode == 2:
+        o["item_max"] = off
+        off += 4 * max_items * hq
+        off = (off + 255) // 256 * 256
+        o["score_pitch"] = (max(max_kv_len, 64) + 63) // 64 * 64
+        o["scores"] = off
+        off += 4 * batch * hq * o["score_pitch"]
         off = (off + 255) // 256 * 256
     o["total"] = off
     return o
@@ -74,8 +87,8 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
     """Parse the plan the GPU wrote into the workspace (host copy)."""
     raw = ws.cpu().numpy().view(np.uint8)
     hdr = raw[:64].view(np.int32)
-    num_items, max_items, hkv = int(hdr[7]), int(hdr[8]), int(hdr[4])
-    o = ws_offsets(mode, batch, hq, max_items, hkv=hkv)
+    num_items, max_items, hkv, slots = int(hdr[7]), int(hdr[8]), int(hdr[4]), int(hdr[14])
+    o = ws_offsets(mode, batch, hq, max_items, hkv=hkv, slots=slots)
 
     def arr(name, n):
         return raw[o[name]:o[name] + 4 * n].view(np.int32).tolist()
@@ -84,7 +97,8 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
     return {"magic": int(hdr[0]), "mode": int(hdr[1]), "tile": int(hdr[9]), "chunk_tiles": int(hdr[10]),
             "error_word": int(hdr[11]), "num_items": num_items, "max_items": max_items,
             "req_splits": arr("req_splits", batch), "req_base": arr("req_base", batch + 1),
-            "req_len": arr("req_len", batch),
+            "req_len": arr("req_len", batch), "slots": slots,
+            "slot_first": arr("slot_first", slots + 1) if mode == 2 else None,
             "items": [tuple(int(x) for x in it) for it in items]}
 
 

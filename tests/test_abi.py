@@ -64,7 +64,10 @@ def P(**kw):
     (dict(sage_k_block=64), pa.PA_ERR_INVALID),
     (dict(mode=1, page_size=4, max_q_tokens=100), pa.PA_ERR_UNSUPPORTED),
     (dict(mode=2, page_size=64, sage_k_block=16), pa.PA_ERR_UNSUPPORTED),
-    (dict(mode=2, page_size=64, sage_k_block=64, max_kv_len=1 << 20), pa.PA_ERR_UNSUPPORTED),  # smem budget
+    (dict(mode=2, page_size=64, sage_k_block=64, max_q_tokens=8), pa.PA_ERR_INVALID),
+    (dict(mode=2, page_size=64, sage_k_block=64, max_splits=4), pa.PA_ERR_INVALID),   # no split cap in SAGE
+    (dict(mode=2, page_size=64, sage_k_block=64, batch=8192, hq=4096, hkv=512, max_kv_len=1 << 30),
+     pa.PA_ERR_UNSUPPORTED),                            # score rows beyond 2^46 bytes
     (dict(num_sms=-1), pa.PA_ERR_INVALID),
 ])
 def test_parameter_validation(lib, kw, status):
@@ -75,13 +78,15 @@ def test_workspace_size_matches_documented_layout(lib):
     for mode, extra in ((0, {}), (1, dict(page_size=16, max_q_tokens=9000)), (2, dict(page_size=64, sage_k_block=64, max_kv_len=4096))):
         p = P(mode=mode, batch=33, hq=32, hkv=8, **extra)
         n = pa.pa_plan_workspace_size(p)
+        slots = 0
         if mode == 0:
-            mi = 148 * 4 + 33          # Hkv 8: one CTA per item
-        elif mode == 1:
-            mi = -(-9000 // 128) + 33
+            mi = 148 * 4 + 33          # Hkv 8: one plan unit per item
+        elif mode == 2:
+            slots = 148 * 2            # Hkv 8: one CTA per slot
+            mi = slots + 33
         else:
-            mi = 33
-        assert n == ws_offsets(mode, 33, 32, mi, hkv=8)["total"]
+            mi = -(-9000 // 128) + 33
+        assert n == ws_offsets(mode, 33, 32, mi, hkv=8, max_kv_len=p.max_kv_len, slots=slots)["total"]
 
 
 def test_host_checks_precede_device_use(lib):

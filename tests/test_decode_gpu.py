@@ -103,6 +103,8 @@ def _assert_same_plan(g, o):
     assert g["req_splits"] == o["req_splits"]
     assert g["req_base"] == o["req_base"]
     assert g["items"] == [tuple(x) for x in o["items"]]
+    if "slot_first" in o:
+        assert g["slot_first"] == o["slot_first"]
 
 
 def test_decode_plan_bit_exact():

@@ -28,6 +28,8 @@ def test_hand_derived_plans(case):
     assert got["req_splits"] == e["req_splits"]
     assert got["req_base"] == e["req_base"]
     assert [list(x) for x in got["items"]] == e["items"]
+    if "slot_first" in e:
+        assert got["slot_first"] == e["slot_first"]
 
 
 def _check_decode_invariants(lens, hkv, P, num_sms, max_splits):
@@ -117,3 +119,38 @@ def test_rejects_negative_lengths():
         op.plan(op.MODE_DECODE, [5, -1], hkv=1, page_size=1, num_sms=1)
     with pytest.raises(ValueError):
         op.plan(op.MODE_EXTEND, [5], [0, 6], hkv=1, page_size=1, num_sms=1)
+
+
+def test_sage_flat_partition_invariants_random():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        B = int(rng.integers(1, 40))
+        lens = [int(x) for x in rng.integers(0, 5000, B)]
+        if rng.random() < 0.2:
+            lens[int(rng.integers(0, B))] = 0
+        hkv = int(rng.choice([1, 2, 8, 16]))
+        num_sms = int(rng.integers(1, 200))
+        pl = op.plan(op.MODE_SAGE_DECODE, lens, hkv=hkv, page_size=64, num_sms=num_sms)
+        C = op.sage_slots(hkv, num_sms)
+        per = pl["chunk_tiles"]
+        sf = pl["slot_first"]
+        assert len(sf) == C + 1 and sf == sorted(sf) and sf[-1] == pl["num_items"]
+        assert pl["num_items"] <= op.max_items(op.MODE_SAGE_DECODE, B, hkv, num_sms)
+        # every request is covered exactly once, in order, by 32-aligned pieces
+        by_req = {}
+        for i, (r, s, a, b) in enumerate(pl["items"]):
+            by_req.setdefault(r, []).append((s, a, b))
+            assert a % 32 == 0 and (a < b or lens[r] == 0)
+            assert i == pl["req_base"][r] + s          # execution order = generation order
+        for r, L in enumerate(lens):
+            parts = by_req[r]
+            assert [s for s, _, _ in parts] == list(range(pl["req_splits"][r]))
+            assert parts[0][1] == 0 and parts[-1][2] == L
+            assert all(b0 == a1 for (_, _, b0), (_, a1, _) in zip(parts, parts[1:]))
+        # each slot holds at most `per` units, and the slots together hold all of them
+        units = 0
+        for c in range(C):
+            u = sum(-(-(b - a) // 32) for (_, _, a, b) in pl["items"][sf[c]:sf[c + 1]])
+            assert u <= per
+            units += u
+        assert units == sum(-(-L // 32) for L in lens)

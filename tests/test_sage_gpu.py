@@ -1,8 +1,10 @@
 """GPU parity of the 8-bit Sage decode against the quantisation-emulating oracle.
 
 The bar: max over output rows (r, h) of ||O_gpu - O_ref||_inf / max(||O_ref||_inf, 1e-6)
-<= 3e-2, on the full Sage workload, scaled variants across head-group sizes,
-ragged and empty rows, and without v_mean.
+<= 3e-2, on the full Sage workload, scaled variants across head-group sizes and
+KV-head counts, ragged and empty rows, rows split into many key ranges (the
+row max is exchanged between the splits), one split per row, and without
+v_mean.
 """
 import os
 
@@ -28,13 +30,13 @@ def _lib():
     pa.lib()
 
 
-def sage_params(spec, batch):
+def sage_params(spec, batch, num_sms=0):
     return pa.make_params(pa.PA_MODE_SAGE_DECODE, spec.batch, spec.hq, spec.hkv, 128, 64,
-                          max_kv_len=batch.page_table.shape[1] * 64, sage_k_block=64)
+                          max_kv_len=batch.page_table.shape[1] * 64, sage_k_block=64, num_sms=num_sms)
 
 
-def run_sage(spec, batch, lay, use_v_mean=True):
-    params = sage_params(spec, batch)
+def run_sage(spec, batch, lay, use_v_mean=True, num_sms=0):
+    params = sage_params(spec, batch, num_sms)
     ws = alloc_ws(params)
     pa.attn_plan(params, batch.seq_lens, None, ws)
     out = torch.full((spec.batch, spec.hq, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
@@ -71,6 +73,45 @@ def test_sage_head_groups_and_ragged_lengths(G, lo, hi):
     out = run_sage(spec, batch, lay)
     ref = oracle_sage(spec, batch, lay)
     assert sage_row_rel_error(out, ref) <= SAGE_REL
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4), (64, 8), (32, 16)])
+def test_sage_kv_head_counts(hq, hkv):
+    spec = wl.Spec("sage_heads", 22, "sage", batch=3, len_lo=1, len_hi=900, hq=hq, hkv=hkv, page_size=64,
+                   spare_pages=0.2)
+    batch = wl.make_batch(spec, DEV)
+    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    out = run_sage(spec, batch, lay)
+    assert sage_row_rel_error(out, oracle_sage(spec, batch, lay)) <= SAGE_REL
+
+
+def test_sage_long_rows_split_many_ways():
+    # rows far longer than one CTA's share: each is split into many key ranges whose maxima
+    # are combined before any probability is quantised, and whose sums are merged
+    spec = wl.Spec("sage_long", 23, "sage", batch=3, len_lo=20000, len_hi=40000, hq=32, hkv=8, page_size=64,
+                   spare_pages=0.05)
+    batch = wl.make_batch(spec, DEV)
+    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    params = sage_params(spec, batch)
+    ws = alloc_ws(params)
+    pa.attn_plan(params, batch.seq_lens, None, ws)
+    from tests.helpers import read_plan
+    assert min(read_plan(ws, 2, spec.batch, spec.hq)["req_splits"]) > 50
+    out = run_sage(spec, batch, lay)
+    assert sage_row_rel_error(out, oracle_sage(spec, batch, lay)) <= SAGE_REL
+
+
+def test_sage_few_slots_match_many():
+    # a plan for one SM (two CTA slots: long pieces) and the device's full plan give the same
+    # quantised probabilities, so both meet the bar
+    spec = wl.CONFIGS[5].scaled(batch=6, len_lo=2000, len_hi=4000)
+    batch = wl.make_batch(spec, DEV)
+    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    ref = oracle_sage(spec, batch, lay)
+    few = run_sage(spec, batch, lay, num_sms=1)
+    many = run_sage(spec, batch, lay)
+    assert sage_row_rel_error(few, ref) <= SAGE_REL
+    assert sage_row_rel_error(many, ref) <= SAGE_REL
 
 
 def test_sage_without_v_mean_and_with_an_empty_row():
