@@ -103,6 +103,17 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# The sources each workload's kernels are built from; profiles/traffic.json is keyed by their hash,
+# so a recorded DRAM traffic figure is reported only for the exact kernels it was taken on.
+KERNEL_SOURCES = {
+    "decode_llama3_8b": ("decode.cu", "common.cuh"),
+    "decode_long_llama3_70b": ("decode.cu", "common.cuh"),
+    "decode_tiny": ("decode.cu", "common.cuh"),
+    "extend_prefix": ("extend.cu", "common.cuh", "tma.cuh"),
+    "sage_decode": ("sage.cu", "common.cuh", "tma.cuh"),
+}
+
+
 def source_hash(*names):
     h = hashlib.sha256()
     for n in names:
@@ -494,8 +505,7 @@ def main():
 
     avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
     achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / scale
-    kernel_src = {"sage_decode": ("sage.cu", "common.cuh"), "extend_prefix": ("extend.cu", "common.cuh")}.get(
-        args.workload, ("decode.cu", "common.cuh"))
+    kernel_src = KERNEL_SOURCES.get(args.workload, KERNEL_SOURCES["decode_llama3_8b"])
     traffic = recorded_traffic(args.workload, source_hash(*kernel_src))
     unit = getattr(work, "unit", "GB/s")
     if unit == "TFLOP/s":
