@@ -300,6 +300,28 @@ pa_status attn_kv_store(const uint16_t* d_k_new, const uint16_t* d_v_new, const 
                         uint16_t* d_v_pool, int64_t num_slots, void* d_ws, pa_stream_t stream);
 
 /*
+ * attn_kv_store_sage - the same cache update for the 8-bit Sage pools, plus their K
+ * scales:
+ *   k8_pool[s][h][:] = k8_new[t][h][:],  v8_pool[s][h][:] = v8_new[t][h][:],
+ *   sf_k[s / 64][h] = sf_k_new[t][h]  only when s % 64 == 0,
+ * s = out_cache_loc[t].  The K scales are per 64-slot block ("FlashInfer PrimTS, Sage
+ * Attention ...", README formula, sfK[blkK]); a block's scale is written by the token
+ * whose slot opens the block, and later tokens of the block are expected to be quantised
+ * (by the caller) with the scale already there.  The pages have no store step for 8-bit
+ * pools; this is that reading.
+ *
+ * d_k8_new int8, d_v8_new E4M3 bytes, both [n_tokens][Hkv][D], device, 16-byte aligned.
+ * d_sf_k_new  fp32 [n_tokens][Hkv] or NULL (the scales are left unchanged).
+ * d_k8_pool, d_v8_pool [num_slots][Hkv][D], 16-byte aligned; d_sf_k fp32 [num_slots/64][Hkv]
+ *             (required with d_sf_k_new; num_slots a multiple of 64 then).
+ * d_ws, races and out-of-range slots as for attn_kv_store.
+ */
+pa_status attn_kv_store_sage(const int8_t* d_k8_new, const uint8_t* d_v8_new, const float* d_sf_k_new,
+                             const int32_t* d_out_cache_loc, int64_t n_tokens, int32_t hkv, int32_t head_dim,
+                             int8_t* d_k8_pool, uint8_t* d_v8_pool, float* d_sf_k, int64_t num_slots,
+                             void* d_ws, pa_stream_t stream);
+
+/*
  * attn_debug_gather - copy, for request r and KV head h_kv, the slot ids and
  * the K rows the kernels gather: d_slots_out int32 [L], d_rows_out bf16 [L][D]
  * for positions 0 .. L-1, L = min(d_seq_lens[r], max_len).  Out-of-range ids

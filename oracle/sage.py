@@ -102,3 +102,28 @@ def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_
             for h in range(hk * G, (hk + 1) * G):
                 out[r, h] = sage_row(q8[r, h], k8, v8, sf_q[r, h], sfk, sf_v[hk], vm, quantize_p)
     return out
+
+
+def kv_store_sage(k8_pool, v8_pool, sf_k, out_cache_loc, k8_new, v8_new, sf_k_new=None, k_block: int = 64):
+    """The 8-bit cache update before a Sage attention call; returns updated copies.
+
+    Each new token t is written to its slot s = out_cache_loc[t] (as in
+    ``oracle.attention.kv_store``: the cache is updated within the forward methods,
+    "Flash Attention Backend in SGLang: Grundlagen und KV Cache optimal nutzen"):
+    k8_pool[s] = k8_new[t], v8_pool[s] = v8_new[t].  The K scales are per 64-key block
+    of slots ("FlashInfer PrimTS, Sage Attention ..." README formula, sfK[blkK]); a block's
+    scale is written by the token whose slot opens the block (s % k_block == 0):
+    sf_k[s // k_block] = sf_k_new[t].  Later tokens of a block are quantised by the caller
+    with the scale already there, so their scale rows are not written.  A slot outside the
+    pool is skipped.  Raw bytes are copied unchanged.
+    """
+    k = np.array(k8_pool, copy=True)
+    v = np.array(v8_pool, copy=True)
+    sf = np.array(sf_k, copy=True)
+    for t, slot in enumerate(np.asarray(out_cache_loc, dtype=np.int64)):
+        if 0 <= slot < k.shape[0]:
+            k[slot] = k8_new[t]
+            v[slot] = v8_new[t]
+            if sf_k_new is not None and slot % k_block == 0:
+                sf[slot // k_block] = sf_k_new[t]
+    return k, v, sf

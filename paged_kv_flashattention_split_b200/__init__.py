@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     attn_decode_paged_sage,
     attn_extend_paged,
     attn_kv_store,
+    attn_kv_store_sage,
     attn_plan,
     lib,
     make_params,

@@ -21,7 +21,8 @@ PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE = 0, 1, 2
 
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
-            "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store")
+            "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store",
+            "attn_kv_store_sage")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -62,6 +63,7 @@ def lib() -> ctypes.CDLL:
                                          _P, _P, _P]),
             "pa_read_device_error": (_I32, [_P, _P]),
             "attn_kv_store": (_I32, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I64, _P, _P]),
+            "attn_kv_store_sage": (_I32, [_P, _P, _P, _P, _I64, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
             "attn_decode_paged_noalloc": (_I32, [PP, _P, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
             "pa_status_string": (ctypes.c_char_p, [_I32]),
             "pa_version": (_I32, []),
@@ -186,6 +188,19 @@ def attn_kv_store(k_new, v_new, out_cache_loc, k_pool, v_pool, ws=None, n_tokens
     st = lib().attn_kv_store(_ptr(k_new), _ptr(v_new), _ptr(out_cache_loc), int(n), int(hkv), int(k_pool.shape[2]),
                              _ptr(k_pool), _ptr(v_pool), int(num_slots), _ptr(ws), _stream(stream))
     return _check(st, "attn_kv_store", raise_on_error)
+
+
+def attn_kv_store_sage(k8_new, v8_new, sf_k_new, out_cache_loc, k8_pool, v8_pool, sf_k, ws=None, n_tokens=None,
+                       num_slots=None, stream=None, raise_on_error=True) -> int:
+    """Scatter new tokens' K8/V8 rows ([n, Hkv, D] bytes) into the 8-bit pools, and the block
+    scales sf_k_new ([n, Hkv] fp32, or None) of the tokens that open a 64-slot block."""
+    n = k8_new.shape[0] if n_tokens is None else n_tokens
+    num_slots = k8_pool.shape[0] if num_slots is None else num_slots
+    hkv = k8_pool.shape[1]
+    st = lib().attn_kv_store_sage(_ptr(k8_new), _ptr(v8_new), _ptr(sf_k_new), _ptr(out_cache_loc), int(n), int(hkv),
+                                  int(k8_pool.shape[2]), _ptr(k8_pool), _ptr(v8_pool), _ptr(sf_k), int(num_slots),
+                                  _ptr(ws), _stream(stream))
+    return _check(st, "attn_kv_store_sage", raise_on_error)
 
 
 def pa_read_device_error(ws, stream=None) -> int:

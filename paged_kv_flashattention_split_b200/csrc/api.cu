@@ -313,9 +313,42 @@ pa_status attn_kv_store(const uint16_t* d_k_new, const uint16_t* d_v_new, const 
   a.loc = d_out_cache_loc;
   a.n_tokens = n_tokens;
   a.hkv = hkv;
+  a.elem_bytes = 2;
   a.k_pool = d_k_pool;
   a.v_pool = d_v_pool;
   a.num_slots = num_slots;
+  a.sf_k_new = nullptr;
+  a.sf_k = nullptr;
+  a.hdr = static_cast<PlanHeader*>(d_ws);
+  return from_cuda(launch_kv_store(a, (cudaStream_t)stream));
+}
+
+pa_status attn_kv_store_sage(const int8_t* d_k8_new, const uint8_t* d_v8_new, const float* d_sf_k_new,
+                             const int32_t* d_out_cache_loc, int64_t n_tokens, int32_t hkv, int32_t head_dim,
+                             int8_t* d_k8_pool, uint8_t* d_v8_pool, float* d_sf_k, int64_t num_slots, void* d_ws,
+                             pa_stream_t stream) {
+  if (n_tokens < 0 || hkv < 1 || num_slots < 1) return PA_ERR_INVALID;
+  if (head_dim != kHeadDim) return PA_ERR_UNSUPPORTED;
+  if (d_sf_k_new && (!d_sf_k || num_slots % kSageBlock != 0)) return PA_ERR_INVALID;
+  if (n_tokens == 0) return PA_OK;
+  if (!d_k8_new || !d_v8_new || !d_out_cache_loc || !d_k8_pool || !d_v8_pool) return PA_ERR_INVALID;
+  if (!aligned16(d_k8_new) || !aligned16(d_v8_new) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) ||
+      (d_ws && !aligned16(d_ws)))
+    return PA_ERR_INVALID;
+  pa_status st = check_arch();
+  if (st != PA_OK) return st;
+  StoreLaunch a;
+  a.k_new = d_k8_new;
+  a.v_new = d_v8_new;
+  a.loc = d_out_cache_loc;
+  a.n_tokens = n_tokens;
+  a.hkv = hkv;
+  a.elem_bytes = 1;
+  a.k_pool = d_k8_pool;
+  a.v_pool = d_v8_pool;
+  a.num_slots = num_slots;
+  a.sf_k_new = d_sf_k_new;
+  a.sf_k = d_sf_k;
   a.hdr = static_cast<PlanHeader*>(d_ws);
   return from_cuda(launch_kv_store(a, (cudaStream_t)stream));
 }

@@ -64,14 +64,17 @@ struct ExtendArgs {
 cudaError_t launch_extend(const ExtendArgs& a, cudaStream_t s);
 
 struct StoreLaunch {
-  const uint16_t* k_new;
-  const uint16_t* v_new;
+  const void* k_new;
+  const void* v_new;
   const int32_t* loc;
   int64_t n_tokens;
   int hkv;
-  uint16_t* k_pool;
-  uint16_t* v_pool;
+  int elem_bytes;      // 2: bf16 pools; 1: Sage K8 / V8 pools
+  void* k_pool;
+  void* v_pool;
   int64_t num_slots;
+  const float* sf_k_new;   // Sage: [n_tokens][hkv] block scales, or NULL
+  float* sf_k;             // Sage: [num_slots / 64][hkv]
   PlanHeader* hdr;     // optional: where to record an out-of-range slot
 };
 cudaError_t launch_kv_store(const StoreLaunch& a, cudaStream_t s);

@@ -148,3 +148,22 @@ def test_scores_use_the_exact_integer_dot():
     q8n = np.full(128, -127, np.int8)
     S = sage.sage_scores_f32(q8n, k8, np.float32(0.5), np.array([0.25], np.float32))
     assert S[0] == -2064512.0 / 8
+
+
+def test_kv_store_sage_rows_and_block_scales():
+    rng = np.random.default_rng(15)
+    k8 = rng.integers(-127, 128, (256, 2, 4)).astype(np.int8)
+    v8 = rng.integers(0, 256, (256, 2, 4)).astype(np.uint8)
+    sf = rng.random((4, 2)).astype(np.float32)
+    kn = rng.integers(-127, 128, (4, 2, 4)).astype(np.int8)
+    vn = rng.integers(0, 256, (4, 2, 4)).astype(np.uint8)
+    sfn = np.array([[9, 8], [7, 6], [5, 4], [3, 2]], dtype=np.float32)
+    # slot 128 opens block 2, slot 70 is inside block 1, 256 is outside the pool, 0 opens block 0
+    k2, v2, sf2 = sage.kv_store_sage(k8, v8, sf, [128, 70, 256, 0], kn, vn, sfn)
+    assert np.array_equal(k2[128], kn[0]) and np.array_equal(v2[70], vn[1]) and np.array_equal(k2[0], kn[3])
+    assert sf2[2].tolist() == [9, 8] and sf2[0].tolist() == [3, 2]
+    assert np.array_equal(sf2[1], sf[1]) and np.array_equal(sf2[3], sf[3])      # mid-block token, outside slot
+    untouched = [s for s in range(256) if s not in (128, 70, 0)]
+    assert np.array_equal(k2[untouched], k8[untouched]) and np.array_equal(v2[untouched], v8[untouched])
+    k3, v3, sf3 = sage.kv_store_sage(k8, v8, sf, [64], kn[:1], vn[:1], None)      # no scales given
+    assert np.array_equal(sf3, sf) and np.array_equal(k3[64], kn[0])

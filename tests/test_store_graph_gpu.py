@@ -1,4 +1,4 @@
-"""GPU tests of the KV-cache store and of a CUDA-graph-captured decode step.
+"""GPU tests of the KV-cache stores (bf16 and 8-bit Sage) and of a CUDA-graph-captured decode step.
 
 The store is compared bit for bit with the oracle's scatter; a decode step that
 stores the new token's K/V and then attends (the order of a forward pass) matches
@@ -126,3 +126,72 @@ def test_decode_step_captured_in_a_cuda_graph_replays_bit_exactly():
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
     del graph
+
+
+def test_sage_store_is_bit_exact_with_block_scales():
+    from oracle import sage as osg
+    g = torch.Generator(device=DEV).manual_seed(6)
+    S, H = 64 * 80, 8
+    k8 = torch.randint(-127, 128, (S, H, 128), device=DEV, generator=g, dtype=torch.int32).to(torch.int8)
+    v8 = torch.randint(0, 256, (S, H, 128), device=DEV, generator=g, dtype=torch.int32).to(torch.uint8)
+    sf = torch.rand(S // 64, H, device=DEV, generator=g)
+    n = 200
+    kn = torch.randint(-127, 128, (n, H, 128), device=DEV, generator=g, dtype=torch.int32).to(torch.int8)
+    vn = torch.randint(0, 256, (n, H, 128), device=DEV, generator=g, dtype=torch.int32).to(torch.uint8)
+    sfn = torch.rand(n, H, device=DEV, generator=g) + 1.0
+    loc = torch.randperm(S, device=DEV, generator=g)[:n].to(torch.int32)
+    loc[:10] = torch.arange(10, device=DEV, dtype=torch.int32) * 64       # tokens that open blocks 0..9
+    loc[50] = -3                                                          # outside the pool: skipped, flagged
+    ref = osg.kv_store_sage(k8.cpu().numpy(), v8.cpu().numpy(), sf.cpu().numpy(), loc.cpu().numpy(),
+                            kn.cpu().numpy(), vn.cpu().numpy(), sfn.cpu().numpy())
+    params = pa.make_params(pa.PA_MODE_DECODE, 1, 8, 8, 128, 1, max_kv_len=1, num_sms=0)
+    ws = alloc_ws(params)
+    pa.attn_kv_store_sage(kn, vn, sfn, loc, k8, v8, sf, ws=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(k8.cpu().numpy(), ref[0]) and np.array_equal(v8.cpu().numpy(), ref[1])
+    assert np.array_equal(sf.cpu().numpy(), ref[2])
+    assert pa.pa_read_device_error(ws) == pa.PA_ERR_DEVICE_INDEX
+
+
+def test_sage_store_then_decode_matches_the_oracle():
+    from oracle import sage as osg
+    spec = wl.CONFIGS[5].scaled(batch=6, len_lo=100, len_hi=1500)
+    batch = wl.make_batch(spec, DEV)
+    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    # every request's decode token goes to the first slot of a spare (unused) page, appended
+    pages_used = set(int(x) for x in batch.page_table.flatten().tolist())
+    spare = [p for p in range(batch.num_slots // 64) if p not in pages_used][: spec.batch]
+    assert len(spare) == spec.batch
+    table = torch.zeros(spec.batch, batch.page_table.shape[1] + 1, dtype=torch.int32, device=DEV)
+    table[:, :-1] = batch.page_table
+    lens = batch.seq_lens.clone()
+    loc = torch.empty(spec.batch, dtype=torch.int32, device=DEV)
+    for r in range(spec.batch):
+        L = int(lens[r])
+        if L % 64 == 0:                          # the next position starts a new page
+            table[r, L // 64] = spare[r]
+            loc[r] = spare[r] * 64
+        else:                                    # the next position is inside the last page
+            loc[r] = int(table[r, L // 64]) * 64 + L % 64
+    lens += 1
+    g = torch.Generator(device=DEV).manual_seed(12)
+    kn = torch.randint(-127, 128, (spec.batch, spec.hkv, 128), device=DEV, generator=g, dtype=torch.int32).to(torch.int8)
+    vn = (16 * torch.randn(spec.batch, spec.hkv, 128, device=DEV, generator=g)).to(torch.float8_e4m3fn).view(torch.uint8)
+    sfn = torch.exp(-4 + 0.5 * torch.randn(spec.batch, spec.hkv, device=DEV, generator=g))
+    k8, v8, sfk = osg.kv_store_sage(lay.k8.cpu().numpy(), lay.v8.cpu().numpy(), lay.sf_k.cpu().numpy(),
+                                    loc.cpu().numpy(), kn.cpu().numpy(), vn.cpu().numpy(), sfn.cpu().numpy())
+    pa.attn_kv_store_sage(kn, vn, sfn, loc, lay.k8, lay.v8, lay.sf_k)
+    b2 = wl.Batch(lens, table, batch.num_slots, batch.used_slot_mask)
+    params = pa.make_params(pa.PA_MODE_SAGE_DECODE, spec.batch, spec.hq, spec.hkv, 128, 64,
+                            max_kv_len=table.shape[1] * 64, sage_k_block=64)
+    ws = alloc_ws(params)
+    pa.attn_plan(params, lens, None, ws)
+    out = torch.empty(spec.batch, spec.hq, 128, dtype=torch.bfloat16, device=DEV)
+    pa.attn_decode_paged_sage(params, ws, lay.q8, lay.sf_q, lay.k8, lay.v8, lay.sf_k, lay.sf_v, lay.v_mean,
+                              table, out)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(ws) == pa.PA_OK
+    ref = osg.sage_decode(lay.q8.cpu().numpy(), lay.sf_q.cpu().numpy(), k8, v8, sfk, lay.sf_v.cpu().numpy(),
+                          lay.v_mean.cpu().numpy(), table.cpu().numpy(), lens.cpu().numpy(), 64)
+    from tests.helpers import SAGE_REL, sage_row_rel_error
+    assert sage_row_rel_error(out, ref) <= SAGE_REL
