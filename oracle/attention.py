@@ -33,7 +33,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .codecs import bf16_bits_to_f64
+from .codecs import bf16_bits_to_f64, e4m3_to_f64
 
 
 def gather_slots(page_table: np.ndarray, seq_len: int, page_size: int, r: int) -> np.ndarray:
@@ -97,6 +97,36 @@ def decode(q_bits, k_pool_bits, v_pool_bits, page_table, seq_lens, page_size, sm
         for hk in range(Hkv):
             k = gather_kv(k_pool_bits, slots, hk)
             v = gather_kv(v_pool_bits, slots, hk)
+            heads = slice(hk * G, (hk + 1) * G)
+            o, ls = softmax_attend(q[r, heads, :], k, v, sm_scale)
+            out[r, heads, :] = o
+            lse[r, heads] = ls
+    return out, lse
+
+
+def decode_fp8(q_bits, k8_pool, v8_pool, k_scale, v_scale, page_table, seq_lens, page_size, sm_scale):
+    """DECODE over an FP8 KV cache: pools of E4M3 codes with one dequantisation scale each.
+
+    The pages list FP8 among the FlashAttention backend's features ("Implement Flash
+    Attention Back End in SGLang - Basics and KV Cache", feature list) without a formula;
+    the reading taken: K = k_scale * E4M3(K8) and V = v_scale * E4M3(V8), decoded exactly
+    (float64), then the standard definition as in ``decode``.  q_bits [B, Hq, D] uint16
+    (bf16), k8_pool / v8_pool [num_slots, Hkv, D] uint8 codes.  Returns (O, lse).
+    """
+    B, Hq, D = q_bits.shape
+    Hkv = k8_pool.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    lse = np.full((B, Hq), -np.inf)
+    q = bf16_bits_to_f64(q_bits)
+    for r in range(B):
+        L = int(seq_lens[r])
+        if L == 0:
+            continue
+        slots = gather_slots(page_table, L, page_size, r)
+        for hk in range(Hkv):
+            k = float(k_scale) * e4m3_to_f64(k8_pool[slots, hk, :])
+            v = float(v_scale) * e4m3_to_f64(v8_pool[slots, hk, :])
             heads = slice(hk * G, (hk + 1) * G)
             o, ls = softmax_attend(q[r, heads, :], k, v, sm_scale)
             out[r, heads, :] = o
