@@ -9,7 +9,7 @@ layer calls of attn_decode_paged, each layer with its own pool (78.6 GB in
 total, so every step reads inputs far larger than L2).  The metric is the
 decode's algorithmic KV bandwidth: K and V rows read once, slot ids, Q and O,
 divided by the device time.  Other workloads (``--workload``):
-decode_long_llama3_70b, extend_prefix, sage_decode, decode_tiny.
+decode_long_llama3_70b, extend_prefix, sage_decode, decode_fp8_llama3_8b, decode_tiny.
 
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
 replica on its own GPU (no collective on the data path); the time is the max
@@ -109,6 +109,7 @@ KERNEL_SOURCES = {
     "decode_llama3_8b": ("decode.cu", "common.cuh"),
     "decode_long_llama3_70b": ("decode.cu", "common.cuh"),
     "decode_tiny": ("decode.cu", "common.cuh"),
+    "decode_fp8_llama3_8b": ("decode_fp8.cu", "decode.cu", "common.cuh"),
     "extend_prefix": ("extend.cu", "common.cuh", "tma.cuh"),
     "sage_decode": ("sage.cu", "common.cuh", "tma.cuh"),
 }
@@ -382,8 +383,54 @@ class ExtendWorkload(DecodeWorkload):
         return flops, time.perf_counter() - t0, f"oracle.attention.extend, one query head at a time, {r * spec.hq + h} (request, head) pairs of layer 0"
 
 
+class Fp8DecodeWorkload(DecodeWorkload):
+    """plan + L layer calls of the FP8-KV decode (E4M3 pools, bf16 Q and O)."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        import paged_kv_flashattention_split_b200 as pa
+        self.pa, self.spec, self.dev = pa, spec, device
+        self.batch = wl.make_batch(spec, device)
+        n_pools = spec.distinct_pools or spec.layers
+        self.pools = [wl.make_fp8_pools(spec, self.batch, l, device) for l in range(n_pools)]
+        self.q = [wl.make_bf16_queries(spec, spec.batch, l, device) for l in range(spec.layers)]
+        self.out = [torch.empty_like(x) for x in self.q]
+        self.params = pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, spec.head_dim,
+                                     spec.page_size, max_kv_len=self.batch.page_table.shape[1] * spec.page_size)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        self.stream = torch.cuda.current_stream()
+        L = self.batch.seq_lens.cpu().tolist()
+        # K8 + V8 rows (1 B per element), page ids, bf16 Q and O
+        self.layer_bytes = wl.decode_kv_bytes(L, spec.hkv, spec.head_dim, 1, spec.page_size, spec.hq, 2, 2)
+        self.step_bytes = self.layer_bytes * spec.layers
+        self.launches_per_step = 1 + 2 * spec.layers
+
+    def layer(self, l):
+        k8, v8 = self.pool(l)
+        self.pa.attn_decode_paged_fp8(self.params, self.ws, self.q[l], k8, v8, wl.FP8_SCALE, wl.FP8_SCALE,
+                                      self.batch.page_table, self.spec.sm_scale, self.out[l])
+
+    def oracle_sample(self, seconds=12.0):
+        from oracle import attention as oa
+        spec = self.spec
+        t0 = time.perf_counter()
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        k8, v8 = (x.cpu().numpy() for x in self.pool(0))
+        qb = self.q[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        prep = time.perf_counter() - t0
+        nbytes, r = 0.0, 0
+        t0 = time.perf_counter()
+        while r < spec.batch and (time.perf_counter() - t0) < seconds:
+            oa.decode_fp8(qb[r:r + 1], k8, v8, wl.FP8_SCALE, wl.FP8_SCALE, table[r:r + 1], lens[r:r + 1],
+                          spec.page_size, spec.sm_scale)
+            nbytes += wl.decode_kv_bytes([int(lens[r])], spec.hkv, spec.head_dim, 1, spec.page_size, spec.hq, 2, 2)
+            r += 1
+        return nbytes, time.perf_counter() - t0, f"oracle.attention.decode_fp8 on requests 0..{r - 1} of layer 0 ({r} of {spec.batch} requests, {int(lens[:r].sum())} keys); host copy {prep:.1f}s untimed"
+
+
 WORKLOADS = {
     "extend_prefix": (3, ExtendWorkload),
+    "decode_fp8_llama3_8b": (6, Fp8DecodeWorkload),
     "sage_decode": (5, SageWorkload),
     "decode_llama3_8b": (2, DecodeWorkload),
     "decode_long_llama3_70b": (4, DecodeWorkload),
@@ -524,7 +571,9 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int8/e4m3 in, fp32 math, bf16 out" if args.workload == "sage_decode" else "bf16",
+        "dtype": {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
+                  "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}.get(
+                      args.workload, "bf16"),
         "data": "synthetic",
         "config": {
             "workload": args.workload,
@@ -532,7 +581,8 @@ def main():
             "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
             "step": "attn_plan + %d x %s" % (spec.layers, {"sage_decode": "attn_decode_paged_sage",
-                                                            "extend_prefix": "attn_extend_paged"}.get(
+                                                            "extend_prefix": "attn_extend_paged",
+                                                            "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}.get(
                                                                args.workload, "attn_decode_paged")),
             "l2": "inputs larger than L2 (each layer reads its own >1 GB pool)",
             "parallelism": f"replicas x{world}",
@@ -541,7 +591,8 @@ def main():
             "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": {"sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
-                       "extend_prefix": "extend_kernel (one launch per attn_extend_paged call)"}.get(
+                       "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
+                       "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}.get(
                            args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
                       + ", per-layer CUDA events",
             "peak_source": peak_note,
@@ -599,6 +650,17 @@ def run_reference(args, spec, cls):
             n = q1 - q0
             return 4.0 * spec.head_dim * (n * (int(lens[r]) - n) + n * (n + 1) // 2)
         per_step, what = 2, "(request, query head) pairs"
+    elif spec.mode == "fp8":
+        k8, v8 = (x.numpy() for x in wl.make_fp8_pools(spec, batch, 0, "cpu"))
+        qb = bits(wl.make_bf16_queries(spec, spec.batch, 0, "cpu"))
+        unit, scale = "GB/s", 1e9
+
+        def one(i):
+            r = i % spec.batch
+            oa.decode_fp8(qb[r:r + 1], k8, v8, wl.FP8_SCALE, wl.FP8_SCALE, table[r:r + 1], lens[r:r + 1],
+                          spec.page_size, spec.sm_scale)
+            return wl.decode_kv_bytes([int(lens[r])], spec.hkv, spec.head_dim, 1, spec.page_size, spec.hq, 2, 2)
+        per_step, what = 2, "requests"
     else:
         k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
         q = wl.make_bf16_queries(spec, spec.batch, 0, "cpu")

@@ -199,6 +199,27 @@ pa_status attn_decode_paged(const pa_plan_params* params, const void* d_ws, size
                             uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
 
 /*
+ * attn_decode_paged_fp8 - DECODE over an FP8 KV cache for one layer.  The FlashAttention
+ * backend lists FP8 among its features ("Implement Flash Attention Back End in SGLang -
+ * Basics and KV Cache", feature list); the operation is the standard decode of
+ * attn_decode_paged on the dequantised cache
+ *     K = k_scale * E4M3(K8),  V = v_scale * E4M3(V8)     (one scale per pool),
+ *     O = softmax(sm_scale * q K^T) V,  lse = log sum_j exp(sm_scale q . K_j).
+ * Same plan (mode PA_MODE_DECODE), work list, split partials and merge as the bf16 decode;
+ * one CTA covers HG = the largest of 8, 4, 2, 1 dividing Hkv heads (1 KB runs per slot at
+ * Hkv = 8).  The tensor cores run in f16 (E4M3 converts to f16 exactly), so |q| must stay
+ * below 65504; q values below 2^-24 flush to zero.  Scales are not checked.
+ *
+ * d_q             bf16 [B][Hq][D];  d_k8_pool, d_v8_pool E4M3 bytes [num_slots][Hkv][D].
+ * Everything else as for attn_decode_paged (any page size 1 .. 256).
+ */
+pa_status attn_decode_paged_fp8(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                                const uint16_t* d_q, const uint8_t* d_k8_pool, const uint8_t* d_v8_pool,
+                                float k_scale, float v_scale, int64_t num_slots,
+                                const int32_t* d_page_table, int64_t pt_pitch, float sm_scale,
+                                uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
+
+/*
  * attn_extend_paged - bf16 causal EXTEND for one layer.  New token i of
  * request r (row cu_seqlens_q[r] + i of Q) sits at absolute position p_r + i
  * and attends to keys j <= p_r + i, whose K/V (prefix and new tokens alike)

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     PagedAttnError,
     attn_debug_gather,
     attn_decode_paged,
+    attn_decode_paged_fp8,
     attn_decode_paged_noalloc,
     attn_decode_paged_sage,
     attn_extend_paged,

@@ -22,7 +22,7 @@ PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE = 0, 1, 2
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
             "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store",
-            "attn_kv_store_sage")
+            "attn_kv_store_sage", "attn_decode_paged_fp8")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
             "attn_plan": (_I32, [PP, _P, _P, _P, _SZ, _P]),
             "attn_decode_paged": (_I32, [PP, _P, _SZ, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
             "attn_extend_paged": (_I32, [PP, _P, _SZ, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
+            "attn_decode_paged_fp8": (_I32, [PP, _P, _SZ, _P, _P, _P, _F32, _F32, _I64, _P, _I64, _F32, _P, _P,
+                                             _P]),
             "attn_decode_paged_sage": (_I32, [PP, _P, _SZ, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64,
                                               _P, _P]),
             "attn_debug_gather": (_I32, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _I64, _P, _I64,
@@ -133,6 +135,18 @@ def attn_decode_paged(params, ws, q, k_pool, v_pool, page_table, sm_scale, out, 
                                  int(pt_pitch), float(sm_scale), _ptr(out), _ptr(lse_out),
                                  _stream(stream))
     return _check(st, "attn_decode_paged", raise_on_error)
+
+
+def attn_decode_paged_fp8(params, ws, q, k8_pool, v8_pool, k_scale, v_scale, page_table, sm_scale, out,
+                          lse_out=None, num_slots=None, pt_pitch=None, stream=None, raise_on_error=True) -> int:
+    """DECODE over E4M3 pools (uint8 codes) dequantised by k_scale / v_scale; q and out bf16."""
+    num_slots = k8_pool.shape[0] if num_slots is None else num_slots
+    pt_pitch = page_table.shape[-1] if pt_pitch is None else pt_pitch
+    st = lib().attn_decode_paged_fp8(ctypes.byref(params), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _ptr(q), _ptr(k8_pool), _ptr(v8_pool), float(k_scale), float(v_scale),
+                                     int(num_slots), _ptr(page_table), int(pt_pitch), float(sm_scale), _ptr(out),
+                                     _ptr(lse_out), _stream(stream))
+    return _check(st, "attn_decode_paged_fp8", raise_on_error)
 
 
 def attn_extend_paged(params, ws, q, k_pool, v_pool, page_table, sm_scale, out, lse_out=None,

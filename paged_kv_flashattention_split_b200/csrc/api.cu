@@ -217,6 +217,45 @@ pa_status attn_decode_paged(const pa_plan_params* params, const void* d_ws, size
   return from_cuda(launch_decode(a, (cudaStream_t)stream));
 }
 
+pa_status attn_decode_paged_fp8(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                                const uint16_t* d_q, const uint8_t* d_k8_pool, const uint8_t* d_v8_pool,
+                                float k_scale, float v_scale, int64_t num_slots, const int32_t* d_page_table,
+                                int64_t pt_pitch, float sm_scale, uint16_t* d_out, float* d_lse_out,
+                                pa_stream_t stream) {
+  Derived d;
+  pa_status st = derive(params, &d);
+  if (st != PA_OK) return st;
+  if (params->mode != PA_MODE_DECODE) return PA_ERR_WORKSPACE;
+  if (!d_ws || !d_q || !d_k8_pool || !d_v8_pool || !d_page_table || !d_out) return PA_ERR_INVALID;
+  if (!aligned16(d_ws) || !aligned16(d_q) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) ||
+      !aligned16(d_out))
+    return PA_ERR_INVALID;
+  if (d_lse_out && (reinterpret_cast<uintptr_t>(d_lse_out) & 3u)) return PA_ERR_INVALID;
+  if (num_slots < 1 || pt_pitch < 1) return PA_ERR_INVALID;
+  const long long need_pitch = ((long long)params->max_kv_len + params->page_size - 1) / params->page_size;
+  if (pt_pitch < need_pitch) return PA_ERR_INVALID;
+  if (ws_bytes < d.layout.total) return PA_ERR_WORKSPACE;
+  if ((st = check_arch()) != PA_OK) return st;
+  Fp8DecodeLaunch a;
+  a.ws = ws_view(const_cast<void*>(d_ws), d.layout);
+  a.q = d_q;
+  a.k8_pool = d_k8_pool;
+  a.v8_pool = d_v8_pool;
+  a.num_slots = num_slots;
+  a.page_table = d_page_table;
+  a.pt_pitch = pt_pitch;
+  a.scale_log2 = sm_scale * k_scale * 1.4426950408889634f;
+  a.v_scale = v_scale;
+  a.out = d_out;
+  a.lse_out = d_lse_out;
+  a.batch = params->batch;
+  a.hq = params->hq;
+  a.hkv = params->hkv;
+  a.page_shift = d.page_shift;
+  a.max_items = d.max_items;
+  return from_cuda(launch_decode_fp8(a, (cudaStream_t)stream));
+}
+
 pa_status attn_extend_paged(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
                             const uint16_t* d_q, const uint16_t* d_k_pool, const uint16_t* d_v_pool,
                             int64_t num_slots, const int32_t* d_page_table, int64_t pt_pitch,

@@ -350,7 +350,14 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   decode_splitkv_kernel<HG, G><<<a.max_items * groups, kThreads, kDecodeSmem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // the merge is a programmatic dependent of the decode grid: its launch overlaps the decode's tail
+  return launch_decode_merge(a, s);
+}
+
+}  // namespace
+
+// The merge is a programmatic dependent of the decode grid just launched on `s` (that grid
+// executes griddepcontrol.launch_dependents): its launch overlaps the decode's tail.
+cudaError_t launch_decode_merge(const DecodeLaunch& a, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.batch * a.hq + 7) / 8);
   cfg.blockDim = dim3(256);
@@ -363,6 +370,8 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, merge_kernel, a);
 }
+
+namespace {
 
 // A plan item covers decode_heads_per_cta(Hkv) <= 8 KV heads; a CTA of four warps takes at
 // most four of them, so an item of eight heads is two CTAs.

@@ -29,6 +29,23 @@ struct DecodeLaunch {
   int batch, hq, hkv, page_shift, max_items;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s);
+cudaError_t launch_decode_merge(const DecodeLaunch& a, cudaStream_t s);   // the split merge alone
+
+struct Fp8DecodeLaunch {
+  WsView ws;
+  const uint16_t* q;       // bf16 [B][Hq][D]
+  const uint8_t* k8_pool;  // E4M3 [num_slots][Hkv][D]
+  const uint8_t* v8_pool;
+  int64_t num_slots;
+  const int32_t* page_table;
+  int64_t pt_pitch;
+  float scale_log2;        // sm_scale * k_scale * log2(e)
+  float v_scale;
+  uint16_t* out;
+  float* lse_out;
+  int batch, hq, hkv, page_shift, max_items;
+};
+cudaError_t launch_decode_fp8(const Fp8DecodeLaunch& a, cudaStream_t s);
 
 struct SageLaunchArgs {
   WsView ws;

@@ -23,6 +23,9 @@ Recipe (all draws from ``torch.Generator``; integers uniform and inclusive):
 * Sage: Q8, K8 uniform in [-127, 127]; V8 = E4M3(16 N(0, 1)); sfQ, sfK, sfV
   lognormal(mu=-4, sigma=0.5); v_mean ~ N(0, 0.1^2) (0.1 read as the standard
   deviation).
+* FP8 KV cache: K8, V8 = E4M3(16 N(0, 1)) (clamped to +-448, nearest-even) with
+  k_scale = v_scale = 1/16, so the dequantised K, V are N(0, 1) like the bf16 pools;
+  Q ~ N(0, 1) in bf16.
 """
 from __future__ import annotations
 
@@ -42,7 +45,7 @@ class Spec:
     the new tokens)."""
     name: str
     cfg: int
-    mode: str                 # "decode" | "extend" | "sage"
+    mode: str                 # "decode" | "extend" | "sage" | "fp8"
     batch: int
     len_lo: int
     len_hi: int
@@ -78,7 +81,11 @@ CONFIGS = {
             hkv=8, page_size=64, layers=80, distinct_pools=8, peaked_frac=0.01, peaked_scale=8.0),
     5: Spec("sage_decode", 5, "sage", batch=32, len_lo=1024, len_hi=4096, hq=32, hkv=8,
             page_size=64, spare_pages=0.10, layers=32),
+    6: Spec("decode_fp8_llama3_8b", 6, "fp8", batch=64, len_lo=512, len_hi=8192, hq=32, hkv=8,
+            page_size=16, spare_pages=0.10, layers=32),
 }
+
+FP8_SCALE = 1.0 / 16.0   # k_scale = v_scale of the FP8 pools
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -157,6 +164,20 @@ def make_bf16_pools(spec: Spec, batch: Batch, layer: int, device="cpu", seed: in
     for t in (k, v):
         t.view(torch.int16)[unused] = BF16_NAN
     return k, v
+
+
+def make_fp8_pools(spec: Spec, batch: Batch, layer: int, device="cpu", seed: int | None = None):
+    """K8 and V8 pools [num_slots, Hkv, D] of E4M3 codes (uint8) for one layer, unused rows NaN;
+    dequantised by FP8_SCALE."""
+    g = _gen(1000 + 100 * spec.cfg + layer if seed is None else seed, device)
+    shape = (batch.num_slots, spec.hkv, spec.head_dim)
+    out = []
+    for _ in range(2):
+        x = (16.0 * torch.randn(shape, generator=g, device=device, dtype=torch.float32)).clamp(-448, 448)
+        c = x.to(torch.float8_e4m3fn).view(torch.uint8)
+        c[~batch.used_slot_mask.to(device)] = E4M3_NAN
+        out.append(c)
+    return out[0], out[1]
 
 
 def make_bf16_queries(spec: Spec, rows: int, layer: int, device="cpu", seed: int | None = None):
