@@ -55,10 +55,20 @@ SAGE_DECODE (flat, balanced partition over CTA slots)
   items slot_first[c] .. slot_first[c+1] - 1.  req_base as for DECODE; every
   slot has at most per units, so the slots finish together.
   Bound: num_items <= C + B.
+
+SAGE_SPARSE (the same partition over the selected blocks' units)
+  A mask[r][b] (b < ceil(L_r / 64)) selects request r's 64-key blocks; sel_r is the
+  ascending list of selected blocks, sel_base its exclusive prefix sum over requests
+  (sel_block concatenates the lists).  A selected block holds 2 units, except a last
+  block of L_r - 64 b <= 32 keys, which holds 1; U_r = the units of sel_r, in order.
+  The SAGE_DECODE partition runs over the U_r, with items (r, s, u0, u1) in unit
+  indices of request r (unit u is key positions 64 sel_r[u // 2] + 32 (u % 2) onward,
+  up to 32 keys and not past L_r).  A request with no selected unit is one item
+  (r, 0, 0, 0).  Bound: num_items <= C + B.
 """
 from __future__ import annotations
 
-MODE_DECODE, MODE_EXTEND, MODE_SAGE_DECODE = 0, 1, 2
+MODE_DECODE, MODE_EXTEND, MODE_SAGE_DECODE, MODE_SAGE_SPARSE = 0, 1, 2, 3
 DECODE_MIN_TILE = 64
 DECODE_CTAS_PER_SM = 4
 SAGE_UNIT = 32
@@ -92,7 +102,7 @@ def max_items(mode: int, batch: int, hkv: int, num_sms: int, max_q_tokens: int =
     """The host-side bound on the number of work items for a plan of this shape."""
     if mode == MODE_DECODE:
         return _cdiv(num_sms * DECODE_CTAS_PER_SM, decode_head_groups(hkv)) + batch
-    if mode == MODE_SAGE_DECODE:
+    if mode in (MODE_SAGE_DECODE, MODE_SAGE_SPARSE):
         return sage_slots(hkv, num_sms) + batch
     if mode == MODE_EXTEND:
         return _cdiv(max_q_tokens, EXTEND_Q_TILE) + batch
@@ -100,13 +110,14 @@ def max_items(mode: int, batch: int, hkv: int, num_sms: int, max_q_tokens: int =
 
 
 def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, num_sms: int,
-         max_splits: int = 1 << 30, max_q_tokens: int = 0):
+         max_splits: int = 1 << 30, max_q_tokens: int = 0, block_mask=None):
     """Return the plan as a dict of plain Python ints and lists.
 
     Keys: ``tile``, ``chunk_tiles`` (DECODE: tiles per split; SAGE_DECODE:
     units per slot; 0 otherwise), ``req_splits``, ``req_base`` (length B + 1),
     ``items`` (list of 4-tuples, in execution order), ``num_items`` and, for
-    SAGE_DECODE, ``slot_first`` (length C + 1).
+    SAGE_DECODE and SAGE_SPARSE, ``slot_first`` (length C + 1); for SAGE_SPARSE also
+    ``sel_base`` (length B + 1) and ``sel_block``.
     """
     L = [int(x) for x in seq_lens]
     B = len(L)
@@ -118,6 +129,8 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
     tile = 0
     if mode == MODE_SAGE_DECODE:
         return _sage_plan(L, hkv, num_sms)
+    if mode == MODE_SAGE_SPARSE:
+        return _sage_plan(L, hkv, num_sms, block_mask)
     if mode == MODE_DECODE:
         tile = decode_tile(page_size)
         tiles = [_cdiv(x, tile) for x in L]
@@ -164,10 +177,19 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
             "items": items, "num_items": len(items)}
 
 
-def _sage_plan(L, hkv: int, num_sms: int):
-    """The flat partition of SAGE_DECODE (module docstring), written out unit by unit."""
+def _sage_plan(L, hkv: int, num_sms: int, block_mask=None):
+    """The flat partition of SAGE_DECODE / SAGE_SPARSE (module docstring), unit by unit."""
     B = len(L)
-    units = [_cdiv(x, SAGE_UNIT) for x in L]
+    sel = None
+    if block_mask is None:
+        units = [_cdiv(x, SAGE_UNIT) for x in L]
+    else:
+        sel, units = [], []
+        for r in range(B):
+            nb = _cdiv(L[r], 2 * SAGE_UNIT)
+            blocks = [b for b in range(nb) if block_mask[r][b]]
+            sel.append(blocks)
+            units.append(sum(1 if L[r] - 2 * SAGE_UNIT * b <= SAGE_UNIT else 2 for b in blocks))
     C = sage_slots(hkv, num_sms)
     total = sum(units)
     per = max(1, _cdiv(total, C))
@@ -185,7 +207,10 @@ def _sage_plan(L, hkv: int, num_sms: int):
         for s, c in enumerate(range(c_first, c_last + 1)):
             u0 = max(g, c * per) - g
             u1 = min(g + units[r], (c + 1) * per) - g
-            items.append((r, s, SAGE_UNIT * u0, min(SAGE_UNIT * u1, L[r])))
+            if sel is None:
+                items.append((r, s, SAGE_UNIT * u0, min(SAGE_UNIT * u1, L[r])))
+            else:
+                items.append((r, s, u0, u1))
             item_slot.append(c)
         g += units[r]
     slot_first = []
@@ -195,5 +220,12 @@ def _sage_plan(L, hkv: int, num_sms: int):
     base = [0] * (B + 1)
     for r in range(B):
         base[r + 1] = base[r] + splits[r]
-    return {"tile": SAGE_UNIT, "chunk_tiles": per, "req_splits": splits, "req_base": base,
-            "items": items, "num_items": len(items), "slot_first": slot_first}
+    out = {"tile": SAGE_UNIT, "chunk_tiles": per, "req_splits": splits, "req_base": base,
+           "items": items, "num_items": len(items), "slot_first": slot_first}
+    if sel is not None:
+        sb = [0] * (B + 1)
+        for r in range(B):
+            sb[r + 1] = sb[r] + len(sel[r])
+        out["sel_base"] = sb
+        out["sel_block"] = [b for blocks in sel for b in blocks]
+    return out

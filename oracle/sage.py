@@ -78,13 +78,30 @@ def sage_row(q8_row, k8_rows, v8_rows, sf_q, sf_k_rows, sf_v, v_mean, quantize_p
     return np.asarray(sf_v, dtype=np.float64) * acc / (448.0 * l) + vm   # step 6: epilogue
 
 
+def selected_positions(seq_len: int, mask_row, k_block: int = 64) -> np.ndarray:
+    """Key positions 0 .. L-1 of a request whose 64-key block j // k_block is selected.
+
+    Block-sparse mode ("FlashInfer PrimTS, Sage Attention ...", README: the decode kernel
+    runs in the dense and block-sparse modes): the reading taken is one mask per
+    (request, logical key block), shared by every head; mask_row[b] != 0 selects block b.
+    """
+    j = np.arange(int(seq_len), dtype=np.int64)
+    if mask_row is None:
+        return j
+    m = np.asarray(mask_row)
+    return j[m[j // k_block] != 0]
+
+
 def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_lens,
-                page_size: int, k_block: int = 64, quantize_p: bool = True) -> np.ndarray:
+                page_size: int, k_block: int = 64, quantize_p: bool = True, block_mask=None) -> np.ndarray:
     """Sage DECODE over the paged cache; returns O [B, Hq, D] float64.
 
     Keys are gathered through the page table exactly as in the bf16 path
     (``oracle.attention.gather_slots``); key c's K scale is
     sf_k[slot(c) // k_block][h_kv]; query head h reads KV head h // (Hq // Hkv).
+    With ``block_mask`` [B][n_blocks] (block-sparse mode), row r attends only to the keys
+    of its selected blocks (``selected_positions``): the Sage formula, row max and row
+    sum included, over that subset; a row with no selected key gives v_mean.
     """
     B, Hq, D = q8.shape
     Hkv = k8_pool.shape[1]
@@ -93,6 +110,8 @@ def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_
     for r in range(B):
         L = int(seq_lens[r])
         slots = gather_slots(page_table, L, page_size, r)
+        if block_mask is not None:
+            slots = slots[selected_positions(L, block_mask[r], k_block)]
         blocks = slots // k_block
         for hk in range(Hkv):
             k8 = k8_pool[slots, hk, :]

@@ -21,7 +21,7 @@ GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "plan_
 def test_hand_derived_plans(case):
     got = op.plan(case["mode"], case["seq_lens"], case.get("cu_seqlens_q"), hkv=case["hkv"],
                   page_size=case["page_size"], num_sms=case["num_sms"], max_splits=case["max_splits"],
-                  max_q_tokens=(case.get("cu_seqlens_q") or [0])[-1])
+                  max_q_tokens=(case.get("cu_seqlens_q") or [0])[-1], block_mask=case.get("block_mask"))
     e = case["expect"]
     assert got["tile"] == e["tile"]
     assert got["chunk_tiles"] == e["chunk_tiles"]
@@ -30,6 +30,9 @@ def test_hand_derived_plans(case):
     assert [list(x) for x in got["items"]] == e["items"]
     if "slot_first" in e:
         assert got["slot_first"] == e["slot_first"]
+    for k in ("sel_base", "sel_block"):
+        if k in e:
+            assert got[k] == e[k]
 
 
 def _check_decode_invariants(lens, hkv, P, num_sms, max_splits):
@@ -154,3 +157,31 @@ def test_sage_flat_partition_invariants_random():
             assert u <= per
             units += u
         assert units == sum(-(-L // 32) for L in lens)
+
+
+def test_sage_sparse_units_cover_exactly_the_selected_keys():
+    rng = np.random.default_rng(8)
+    for _ in range(150):
+        B = int(rng.integers(1, 20))
+        lens = [int(x) for x in rng.integers(0, 3000, B)]
+        nbm = max(1, max(-(-L // 64) for L in lens))
+        mask = (rng.random((B, nbm)) < rng.choice([0.0, 0.1, 0.5, 1.0])).astype(int)
+        hkv, num_sms = int(rng.choice([1, 2, 8])), int(rng.integers(1, 100))
+        pl = op.plan(op.MODE_SAGE_SPARSE, lens, hkv=hkv, page_size=64, num_sms=num_sms, block_mask=mask)
+        sb, blk = pl["sel_base"], pl["sel_block"]
+        per = pl["chunk_tiles"]
+        C = op.sage_slots(hkv, num_sms)
+        assert pl["num_items"] <= op.max_items(op.MODE_SAGE_SPARSE, B, hkv, num_sms)
+        for r, L in enumerate(lens):
+            want = [j for j in range(L) if mask[r][j // 64]]
+            got = []
+            for (rr, s, u0, u1) in pl["items"]:
+                if rr != r:
+                    continue
+                for u in range(u0, u1):
+                    k0 = 64 * blk[sb[r] + u // 2] + 32 * (u % 2)
+                    got += list(range(k0, min(k0 + 32, L)))
+            assert got == want
+            assert blk[sb[r]:sb[r + 1]] == sorted(b for b in range(-(-L // 64)) if mask[r][b])
+        for c in range(C):
+            assert sum(u1 - u0 for (_, _, u0, u1) in pl["items"][pl["slot_first"][c]:pl["slot_first"][c + 1]]) <= per

@@ -167,3 +167,53 @@ def test_kv_store_sage_rows_and_block_scales():
     assert np.array_equal(k2[untouched], k8[untouched]) and np.array_equal(v2[untouched], v8[untouched])
     k3, v3, sf3 = sage.kv_store_sage(k8, v8, sf, [64], kn[:1], vn[:1], None)      # no scales given
     assert np.array_equal(sf3, sf) and np.array_equal(k3[64], kn[0])
+
+
+def _sage_case(rng, lens, hq, hkv, spare=2):
+    P = 64
+    need = [(L + P - 1) // P for L in lens]
+    num_pages = sum(need) + spare
+    perm = rng.permutation(num_pages)
+    table = np.zeros((len(lens), max(1, max(need))), dtype=np.int64)
+    off = 0
+    for r, n in enumerate(need):
+        table[r, :n] = perm[off:off + n]
+        off += n
+    S = num_pages * P
+    q8 = rng.integers(-127, 128, (len(lens), hq, 128)).astype(np.int8)
+    k8 = rng.integers(-127, 128, (S, hkv, 128)).astype(np.int8)
+    v8 = f64_to_e4m3(16 * rng.standard_normal((S, hkv, 128)))
+    sfq = np.exp(-4 + 0.5 * rng.standard_normal((len(lens), hq))).astype(np.float32)
+    sfk = np.exp(-4 + 0.5 * rng.standard_normal((num_pages, hkv))).astype(np.float32)
+    sfv = np.exp(-4 + 0.5 * rng.standard_normal((hkv, 128))).astype(np.float32)
+    vm = 0.1 * rng.standard_normal((hkv, 128))
+    return q8, k8, v8, sfq, sfk, sfv, vm, table
+
+
+def test_block_sparse_equals_dense_on_the_compacted_cache():
+    # selecting blocks = a dense call over a page table holding only the selected pages
+    rng = np.random.default_rng(41)
+    lens, hq, hkv = [300, 64, 130, 1], 8, 2
+    q8, k8, v8, sfq, sfk, sfv, vm, table = _sage_case(rng, lens, hq, hkv)
+    mask = np.array([[1, 0, 1, 1, 0], [1, 0, 0, 0, 0], [0, 1, 1, 0, 0], [1, 0, 0, 0, 0]])
+    sparse = sage.sage_decode(q8, sfq, k8, v8, sfk, sfv, vm, table, lens, 64, block_mask=mask)
+    for r, L in enumerate(lens):
+        nb = -(-L // 64)
+        keep = [b for b in range(nb) if mask[r][b]]
+        sub_table = np.array([[table[r][b] for b in keep] or [0]])
+        # keys of a kept block: all 64, or the tail for the last block
+        sub_len = sum(min(64, L - 64 * b) for b in keep)
+        # (only the request's last block can be partial, so it is also last in the compacted row)
+        dense = sage.sage_decode(q8[r:r + 1], sfq[r:r + 1], k8, v8, sfk, sfv, vm, sub_table, [sub_len], 64)
+        assert np.array_equal(sparse[r], dense[0])
+
+
+def test_block_sparse_all_ones_is_dense_and_none_selected_is_v_mean():
+    rng = np.random.default_rng(42)
+    lens, hq, hkv = [200, 70], 4, 1
+    q8, k8, v8, sfq, sfk, sfv, vm, table = _sage_case(rng, lens, hq, hkv)
+    dense = sage.sage_decode(q8, sfq, k8, v8, sfk, sfv, vm, table, lens, 64)
+    ones = sage.sage_decode(q8, sfq, k8, v8, sfk, sfv, vm, table, lens, 64, block_mask=np.ones((2, 4), int))
+    assert np.array_equal(dense, ones)
+    none = sage.sage_decode(q8, sfq, k8, v8, sfk, sfv, vm, table, lens, 64, block_mask=np.zeros((2, 4), int))
+    assert np.array_equal(none, np.repeat(vm[None, :, :], 2, 0).repeat(hq // hkv, 1))
