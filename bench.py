@@ -9,7 +9,8 @@ layer calls of attn_decode_paged, each layer with its own pool (78.6 GB in
 total, so every step reads inputs far larger than L2).  The metric is the
 decode's algorithmic KV bandwidth: K and V rows read once, slot ids, Q and O,
 divided by the device time.  Other workloads (``--workload``):
-decode_long_llama3_70b, extend_prefix, sage_decode, decode_fp8_llama3_8b, decode_tiny.
+decode_long_llama3_70b, extend_prefix, sage_decode, sage_sparse_decode,
+decode_fp8_llama3_8b, decode_tiny.
 
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
 replica on its own GPU (no collective on the data path); the time is the max
@@ -112,6 +113,7 @@ KERNEL_SOURCES = {
     "decode_fp8_llama3_8b": ("decode_fp8.cu", "decode.cu", "common.cuh"),
     "extend_prefix": ("extend.cu", "common.cuh", "tma.cuh"),
     "sage_decode": ("sage.cu", "common.cuh", "tma.cuh"),
+    "sage_sparse_decode": ("sage.cu", "common.cuh", "tma.cuh"),
 }
 
 
@@ -383,6 +385,63 @@ class ExtendWorkload(DecodeWorkload):
         return flops, time.perf_counter() - t0, f"oracle.attention.extend, one query head at a time, {r * spec.hq + h} (request, head) pairs of layer 0"
 
 
+class SageSparseWorkload(SageWorkload):
+    """plan (with the batch's block mask) + L layer calls of the block-sparse Sage decode."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        super().__init__(spec, device)
+        import paged_kv_flashattention_split_b200 as pa
+        self.mask = wl.make_block_mask(spec, self.batch, device)
+        self.params = pa.make_params(pa.PA_MODE_SAGE_SPARSE, spec.batch, spec.hq, spec.hkv, spec.head_dim, 64,
+                                     max_kv_len=self.batch.page_table.shape[1] * 64, sage_k_block=64)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        L = self.batch.seq_lens.cpu().tolist()
+        m = self.mask.cpu().numpy()
+        sel = [sum(min(64, x - 64 * b) for b in range(-(-x // 64)) if m[r][b]) for r, x in enumerate(L)]
+        nsel_blocks = sum(int(m[r][: -(-x // 64)].sum()) for r, x in enumerate(L))
+        # the selected keys' K8 + V8 rows, their blocks' sfK and page ids, Q8 + sfQ, bf16 O
+        self.layer_bytes = float(sum(sel) * spec.hkv * spec.head_dim * 2 + nsel_blocks * (spec.hkv * 4 + 4)
+                                 + spec.batch * spec.hq * (spec.head_dim * 1 + 4 + spec.head_dim * 2))
+        self.step_bytes = self.layer_bytes * spec.layers
+        self.selected_keys = sum(sel)
+
+    def step(self, layer_events=None):
+        self.pa.attn_plan_sage_sparse(self.params, self.batch.seq_lens, self.mask, self.ws)
+        for l in range(self.spec.layers):
+            if layer_events is not None:
+                layer_events[l][0].record()
+            self.layer(l)
+            if layer_events is not None:
+                layer_events[l][1].record()
+
+    def step_e2e(self):
+        self.batch.seq_lens.copy_(self.h_lens, non_blocking=True)
+        self.batch.page_table.copy_(self.h_table, non_blocking=True)
+        self.pa.attn_plan_sage_sparse(self.params, self.batch.seq_lens, self.mask, self.ws)
+        for l in range(self.spec.layers):
+            self.q[l].copy_(self.h_q[l], non_blocking=True)
+            self.layer(l)
+            self.h_out[l].copy_(self.out[l], non_blocking=True)
+
+    def oracle_sample(self, seconds=12.0):
+        from oracle import sage as osg
+        spec = self.spec
+        d = self.layers_data[0]
+        host = {k: getattr(d, k).cpu().numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        m = self.mask.cpu().numpy()
+        t0 = time.perf_counter()
+        nbytes, r = 0.0, 0
+        while r < spec.batch and (time.perf_counter() - t0) < seconds:
+            osg.sage_decode(host["q8"][r:r + 1], host["sf_q"][r:r + 1], host["k8"], host["v8"], host["sf_k"],
+                            host["sf_v"], host["v_mean"], table[r:r + 1], lens[r:r + 1], 64, block_mask=m[r:r + 1])
+            L = int(lens[r])
+            nbytes += sum(min(64, L - 64 * b) for b in range(-(-L // 64)) if m[r][b]) * spec.hkv * spec.head_dim * 2
+            r += 1
+        return nbytes, time.perf_counter() - t0, f"oracle.sage.sage_decode (block mask) on requests 0..{r - 1} of layer 0"
+
+
 class Fp8DecodeWorkload(DecodeWorkload):
     """plan + L layer calls of the FP8-KV decode (E4M3 pools, bf16 Q and O)."""
 
@@ -431,6 +490,7 @@ class Fp8DecodeWorkload(DecodeWorkload):
 WORKLOADS = {
     "extend_prefix": (3, ExtendWorkload),
     "decode_fp8_llama3_8b": (6, Fp8DecodeWorkload),
+    "sage_sparse_decode": (7, SageSparseWorkload),
     "sage_decode": (5, SageWorkload),
     "decode_llama3_8b": (2, DecodeWorkload),
     "decode_long_llama3_70b": (4, DecodeWorkload),
@@ -572,6 +632,7 @@ def main():
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
+                  "sage_sparse_decode": "int8/e4m3 in, fp32 math, bf16 out",
                   "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}.get(
                       args.workload, "bf16"),
         "data": "synthetic",
@@ -581,6 +642,7 @@ def main():
             "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
             "step": "attn_plan + %d x %s" % (spec.layers, {"sage_decode": "attn_decode_paged_sage",
+                                                            "sage_sparse_decode": "attn_decode_paged_sage (block-sparse plan)",
                                                             "extend_prefix": "attn_extend_paged",
                                                             "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}.get(
                                                                args.workload, "attn_decode_paged")),
@@ -591,6 +653,7 @@ def main():
             "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": {"sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
+                       "sage_sparse_decode": "attn_decode_paged_sage call, block-sparse plan (score + value + merge kernels)",
                        "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
                        "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}.get(
                            args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
@@ -628,12 +691,16 @@ def run_reference(args, spec, cls):
         host = {k: getattr(d, k).numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
         unit, scale = "GB/s", 1e9
         per_key = spec.hkv * spec.head_dim * 2 + spec.hkv * 4 / 64
+        mask = wl.make_block_mask(spec, batch, "cpu").numpy() if spec.density < 1.0 else None
 
         def one(i):
             r = i % spec.batch
             osg.sage_decode(host["q8"][r:r + 1], host["sf_q"][r:r + 1], host["k8"], host["v8"], host["sf_k"],
-                            host["sf_v"], host["v_mean"], table[r:r + 1], lens[r:r + 1], 64)
-            return float(lens[r]) * per_key
+                            host["sf_v"], host["v_mean"], table[r:r + 1], lens[r:r + 1], 64,
+                            block_mask=None if mask is None else mask[r:r + 1])
+            L = int(lens[r])
+            keys = L if mask is None else sum(min(64, L - 64 * b) for b in range(-(-L // 64)) if mask[r][b])
+            return float(keys) * per_key
         per_step, what = 2, "requests"
     elif spec.mode == "extend":
         k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")

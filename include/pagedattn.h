@@ -73,7 +73,8 @@ typedef enum {
 typedef enum {
   PA_MODE_DECODE = 0,       /* bf16 split-KV decode + log-sum-exp merge */
   PA_MODE_EXTEND = 1,       /* bf16 causal extend over a cached prefix (tcgen05 / TMEM) */
-  PA_MODE_SAGE_DECODE = 2   /* INT8 Q/K, E4M3 P and V, per-block scales, bf16 output */
+  PA_MODE_SAGE_DECODE = 2,  /* INT8 Q/K, E4M3 P and V, per-block scales, bf16 output */
+  PA_MODE_SAGE_SPARSE = 3   /* SAGE_DECODE over the selected 64-key blocks of each request */
 } pa_mode;
 
 /*
@@ -144,6 +145,11 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  *     listed r-major (which is also slot order, no sort) and slot_first[c],
  *     c = 0 .. C, is the first item of slot c or later (num_items if none).
  *     max_splits must be 0 (the slots are balanced by construction).
+ *   SAGE_SPARSE: the SAGE_DECODE partition over the units of each request's selected
+ *     blocks (attn_plan_sage_sparse): sel_r = the selected blocks in ascending order, a
+ *     selected block holds 2 units except a last block of L_r - 64 b <= 32 keys (1 unit);
+ *     items are (r, s, u0, u1) in unit indices of request r, unit u being keys
+ *     64 sel_r[u / 2] + 32 (u % 2) onward (at most 32, not past L_r).
  * At most ceil(num_sms * 4 / groups) + B items (DECODE), C + B (SAGE) or
  * ceil(max_q_tokens / 128) + B (EXTEND).
  *
@@ -158,7 +164,9 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  *             req_prefix[B] (EXTEND: p_r), padded to 16 B, then the items
  *             int32x4 [max_items] = {r, split, begin, end} in execution order,
  *             256-byte aligned, then (SAGE) slot_first int32 [C + 1], 256-byte
- *             aligned, then (DECODE, SAGE) fp32 partial outputs
+ *             aligned, then (SAGE_SPARSE) sel_base int32 [B + 1] and sel_block int32
+ *             [B * ceil(max_kv_len / 64)], each 256-byte aligned, then (DECODE,
+ *             SAGE) fp32 partial outputs
  *             [max_items][Hq][D] and partial LSEs (DECODE: log2 units; SAGE:
  *             the split's row sum l) [max_items][Hq], then (SAGE) the split
  *             maxima fp32 [max_items][Hq] and the score rows fp32
@@ -174,6 +182,26 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
 pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
                     const int32_t* d_cu_seqlens_q, void* d_ws, size_t ws_bytes,
                     pa_stream_t stream);
+
+/*
+ * attn_plan_sage_sparse - the plan of a block-sparse Sage decode (mode PA_MODE_SAGE_SPARSE):
+ * Sage attention runs in the dense and block-sparse modes ("FlashInfer PrimTS, Sage
+ * Attention ...", README), and, as for the dense plan, the sparsity pattern is fixed when
+ * the plan is made.  The reading taken for decode: one mask per (request, logical 64-key
+ * block), shared by all heads; request r attends to the keys of its selected blocks only,
+ * and the Sage formula (row max and row sum included) runs over that subset.
+ *
+ * d_block_mask   uint8 [B][mask_pitch], device: nonzero selects block b of request r
+ *                (entries at b >= ceil(L_r / 64) are ignored); mask_pitch >=
+ *                ceil(max_kv_len / 64).
+ * The partition (algorithm at attn_plan, SAGE_SPARSE) runs over the selected blocks'
+ * 32-key units, so every CTA slot streams the same number of selected keys; the workspace
+ * holds the selected blocks of each request (sel_base, sel_block).  A request with no
+ * selected block gives O = v_mean.  Other arguments and errors as for attn_plan.
+ */
+pa_status attn_plan_sage_sparse(const pa_plan_params* params, const int32_t* d_seq_lens,
+                                const uint8_t* d_block_mask, int64_t mask_pitch, void* d_ws, size_t ws_bytes,
+                                pa_stream_t stream);
 
 /*
  * attn_decode_paged - bf16 DECODE over the paged cache for one layer.
@@ -251,7 +279,8 @@ pa_status attn_extend_paged(const pa_plan_params* params, const void* d_ws, size
  * sfQ.  Scales must be finite and positive and are NOT checked (same page,
  * item 1).
  *
- * params, d_ws    the plan (mode PA_MODE_SAGE_DECODE, sage_k_block = 64 = page_size).
+ * params, d_ws    the plan (mode PA_MODE_SAGE_DECODE, or PA_MODE_SAGE_SPARSE from
+ *                 attn_plan_sage_sparse; sage_k_block = 64 = page_size).
  * d_q8 int8 [B][Hq][D];  d_sf_q fp32 [B][Hq].
  * d_k8_pool int8, d_v8_pool E4M3 bytes, both [num_slots][Hkv][D].
  * d_sf_k fp32 [num_slots / 64][Hkv];  d_sf_v fp32 [Hkv][D];

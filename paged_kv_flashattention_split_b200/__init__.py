@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     PA_MODE_DECODE,
     PA_MODE_EXTEND,
     PA_MODE_SAGE_DECODE,
+    PA_MODE_SAGE_SPARSE,
     PA_OK,
     PagedAttnError,
     attn_debug_gather,
@@ -28,6 +29,7 @@ from ._binding import (  # noqa: F401
     attn_kv_store,
     attn_kv_store_sage,
     attn_plan,
+    attn_plan_sage_sparse,
     lib,
     make_params,
     pa_plan_params,

@@ -17,12 +17,12 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedatt
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_ARCH = 0, 1, 2, 3
 PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE_INDEX = 4, 5, 6
-PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE = 0, 1, 2
+PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE, PA_MODE_SAGE_SPARSE = 0, 1, 2, 3
 
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
             "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store",
-            "attn_kv_store_sage", "attn_decode_paged_fp8")
+            "attn_kv_store_sage", "attn_decode_paged_fp8", "attn_plan_sage_sparse")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "pa_plan_workspace_size": (_I32, [PP, ctypes.POINTER(_SZ)]),
             "attn_plan": (_I32, [PP, _P, _P, _P, _SZ, _P]),
+            "attn_plan_sage_sparse": (_I32, [PP, _P, _P, _I64, _P, _SZ, _P]),
             "attn_decode_paged": (_I32, [PP, _P, _SZ, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
             "attn_extend_paged": (_I32, [PP, _P, _SZ, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
             "attn_decode_paged_fp8": (_I32, [PP, _P, _SZ, _P, _P, _P, _F32, _F32, _I64, _P, _I64, _F32, _P, _P,
@@ -124,6 +125,14 @@ def attn_plan(params, seq_lens, cu_seqlens_q, ws, stream=None, raise_on_error=Tr
     st = lib().attn_plan(ctypes.byref(params), _ptr(seq_lens), _ptr(cu_seqlens_q), _ptr(ws), nbytes,
                          _stream(stream))
     return _check(st, "attn_plan", raise_on_error)
+
+
+def attn_plan_sage_sparse(params, seq_lens, block_mask, ws, stream=None, raise_on_error=True) -> int:
+    """Plan of the block-sparse Sage decode; block_mask uint8 [B, mask_pitch] (nonzero = attend)."""
+    nbytes = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
+    st = lib().attn_plan_sage_sparse(ctypes.byref(params), _ptr(seq_lens), _ptr(block_mask),
+                                     int(block_mask.shape[-1]), _ptr(ws), nbytes, _stream(stream))
+    return _check(st, "attn_plan_sage_sparse", raise_on_error)
 
 
 def attn_decode_paged(params, ws, q, k_pool, v_pool, page_table, sm_scale, out, lse_out=None,

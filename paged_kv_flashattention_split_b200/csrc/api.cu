@@ -55,7 +55,7 @@ pa_status check_arch() {
 
 pa_status derive(const pa_plan_params* p, Derived* d) {
   if (!p) return PA_ERR_INVALID;
-  if (p->mode < PA_MODE_DECODE || p->mode > PA_MODE_SAGE_DECODE) return PA_ERR_INVALID;
+  if (p->mode < PA_MODE_DECODE || p->mode > PA_MODE_SAGE_SPARSE) return PA_ERR_INVALID;
   if (p->batch < 1 || p->batch > kMaxBatch) return PA_ERR_INVALID;
   if (p->hq < 1 || p->hkv < 1 || p->hq % p->hkv != 0) return PA_ERR_INVALID;
   if (p->max_kv_len < 0 || p->max_q_tokens < 0 || p->num_sms < 0 || p->max_splits < 0) return PA_ERR_INVALID;
@@ -81,6 +81,7 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
       d->tile = kExtendKvTile;
       break;
     case PA_MODE_SAGE_DECODE:
+    case PA_MODE_SAGE_SPARSE:
       // the flat partition balances the slots itself: no split cap
       if (p->max_q_tokens != 0 || p->max_splits != 0) return PA_ERR_INVALID;
       if (p->sage_k_block != kSageBlock || P != kSageBlock) return PA_ERR_UNSUPPORTED;
@@ -104,7 +105,7 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
     const int groups = p->hkv / decode_heads_per_cta(p->hkv);
     mi = ((long long)sms * kDecodeCtasPerSm + groups - 1) / groups + p->batch;
   }
-  else if (p->mode == PA_MODE_SAGE_DECODE)
+  else if (sage_mode(p->mode))
   {
     d->slots = sage_slots(p->hkv, sms);
     mi = (long long)d->slots + p->batch;
@@ -150,8 +151,28 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes) {
   return PA_OK;
 }
 
+static pa_status plan_common(const pa_plan_params* params, const int32_t* d_seq_lens, const int32_t* d_cu_seqlens_q,
+                             const uint8_t* d_block_mask, int64_t mask_pitch, void* d_ws, size_t ws_bytes,
+                             pa_stream_t stream);
+
 pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
                     const int32_t* d_cu_seqlens_q, void* d_ws, size_t ws_bytes, pa_stream_t stream) {
+  if (params && params->mode == PA_MODE_SAGE_SPARSE) return PA_ERR_INVALID;   // needs attn_plan_sage_sparse
+  return plan_common(params, d_seq_lens, d_cu_seqlens_q, nullptr, 0, d_ws, ws_bytes, stream);
+}
+
+pa_status attn_plan_sage_sparse(const pa_plan_params* params, const int32_t* d_seq_lens,
+                                const uint8_t* d_block_mask, int64_t mask_pitch, void* d_ws, size_t ws_bytes,
+                                pa_stream_t stream) {
+  if (!params || params->mode != PA_MODE_SAGE_SPARSE || !d_block_mask) return PA_ERR_INVALID;
+  if (mask_pitch < ((int64_t)params->max_kv_len + kSageBlock - 1) / kSageBlock || mask_pitch < 1)
+    return PA_ERR_INVALID;
+  return plan_common(params, d_seq_lens, nullptr, d_block_mask, mask_pitch, d_ws, ws_bytes, stream);
+}
+
+static pa_status plan_common(const pa_plan_params* params, const int32_t* d_seq_lens, const int32_t* d_cu_seqlens_q,
+                             const uint8_t* d_block_mask, int64_t mask_pitch, void* d_ws, size_t ws_bytes,
+                             pa_stream_t stream) {
   Derived d;
   pa_status st = derive(params, &d);
   if (st != PA_OK) return st;
@@ -177,6 +198,8 @@ pa_status attn_plan(const pa_plan_params* params, const int32_t* d_seq_lens,
   a.tile = d.tile;
   a.sort_n = d.sort_n;
   a.slots = d.slots;
+  a.block_mask = d_block_mask;
+  a.mask_pitch = mask_pitch;
   return from_cuda(launch_plan(a, (cudaStream_t)stream));
 }
 
@@ -302,7 +325,7 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
   Derived d;
   pa_status st = derive(params, &d);
   if (st != PA_OK) return st;
-  if (params->mode != PA_MODE_SAGE_DECODE) return PA_ERR_WORKSPACE;
+  if (!sage_mode(params->mode)) return PA_ERR_WORKSPACE;
   if (!d_ws || !d_q8 || !d_sf_q || !d_k8_pool || !d_v8_pool || !d_sf_k || !d_sf_v || !d_page_table || !d_out)
     return PA_ERR_INVALID;
   if (!aligned16(d_ws) || !aligned16(d_q8) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) || !aligned16(d_out) ||

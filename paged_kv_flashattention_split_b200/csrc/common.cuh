@@ -35,8 +35,8 @@ static_assert(sizeof(PlanHeader) == 64, "header is 64 bytes");
 
 // Byte offsets of the workspace arrays.
 struct WsLayout {
-  size_t req_splits, req_base, req_len, req_aux, req_prefix, items, slot_first, partial_o, partial_lse, item_max,
-      scores, total;
+  size_t req_splits, req_base, req_len, req_aux, req_prefix, items, slot_first, sel_base, sel_block, partial_o,
+      partial_lse, item_max, scores, total;
   int64_t score_pitch;   // SAGE: keys per (request, head) row of the score scratch
 };
 
@@ -47,9 +47,14 @@ __host__ __device__ inline int decode_heads_per_cta(int hkv) {
   return hkv % 8 == 0 ? 8 : hkv % 4 == 0 ? 4 : hkv % 2 == 0 ? 2 : 1;
 }
 
+// The Sage modes (dense and block-sparse) share the flat partition and the run kernels.
+__host__ __device__ inline bool sage_mode(int mode) {
+  return mode == PA_MODE_SAGE_DECODE || mode == PA_MODE_SAGE_SPARSE;
+}
+
 // Modes whose run kernels write split partials for a merge.
 __host__ __device__ inline bool splitkv_mode(int mode) {
-  return mode == PA_MODE_DECODE || mode == PA_MODE_SAGE_DECODE;
+  return mode == PA_MODE_DECODE || sage_mode(mode);
 }
 
 // CTA slots of a Sage plan: max(1, floor(num_sms * 2 / groups)).
@@ -71,8 +76,15 @@ inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, in
   off = align_up(off, 16);
   w.items = off;      off += 16 * (size_t)max_items;
   off = align_up(off, 256);
-  if (mode == PA_MODE_SAGE_DECODE) {
+  if (sage_mode(mode)) {
     w.slot_first = off; off += 4 * (size_t)(slots + 1);
+    off = align_up(off, 256);
+  }
+  if (mode == PA_MODE_SAGE_SPARSE) {
+    const size_t max_blocks = ((size_t)max_kv_len + kSageBlock - 1) / kSageBlock;
+    w.sel_base = off;  off += 4 * (size_t)(batch + 1);
+    off = align_up(off, 256);
+    w.sel_block = off; off += 4 * (size_t)batch * max_blocks;
     off = align_up(off, 256);
   }
   if (splitkv_mode(mode)) {
@@ -81,7 +93,7 @@ inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, in
     w.partial_lse = off; off += 4 * (size_t)max_items * hq;
     off = align_up(off, 256);
   }
-  if (mode == PA_MODE_SAGE_DECODE) {
+  if (sage_mode(mode)) {
     w.item_max = off;    off += 4 * (size_t)max_items * hq;
     off = align_up(off, 256);
     w.score_pitch = (int64_t)align_up((size_t)(max_kv_len > kSageBlock ? max_kv_len : kSageBlock), kSageBlock);
@@ -102,6 +114,8 @@ struct WsView {
   int32_t* req_prefix;
   int4* items;
   int32_t* slot_first;  // SAGE: [slots + 1] first item of each CTA slot
+  int32_t* sel_base;    // SAGE_SPARSE: [B + 1] first selected block of each request in sel_block
+  int32_t* sel_block;   // SAGE_SPARSE: the selected 64-key blocks, request by request
   float* partial_o;
   float* partial_lse;   // DECODE: split LSE (log2); SAGE: split row sum l
   float* item_max;      // SAGE: [max_items][Hq] maximum score of each split
@@ -120,6 +134,8 @@ inline WsView ws_view(void* ws, const WsLayout& w) {
   v.req_prefix = reinterpret_cast<int32_t*>(b + w.req_prefix);
   v.items = reinterpret_cast<int4*>(b + w.items);
   v.slot_first = w.slot_first ? reinterpret_cast<int32_t*>(b + w.slot_first) : nullptr;
+  v.sel_base = w.sel_base ? reinterpret_cast<int32_t*>(b + w.sel_base) : nullptr;
+  v.sel_block = w.sel_block ? reinterpret_cast<int32_t*>(b + w.sel_block) : nullptr;
   v.partial_o = w.partial_o ? reinterpret_cast<float*>(b + w.partial_o) : nullptr;
   v.partial_lse = w.partial_lse ? reinterpret_cast<float*>(b + w.partial_lse) : nullptr;
   v.item_max = w.item_max ? reinterpret_cast<float*>(b + w.item_max) : nullptr;

@@ -12,6 +12,8 @@ struct PlanLaunch {
   int mode, batch, hq, hkv, head_dim, page_size, max_kv_len, num_sms, max_splits, max_items, tile;
   int sort_n;  // power of two >= max_items
   int slots;   // SAGE: CTA slots
+  const uint8_t* block_mask;   // SAGE_SPARSE: [B][mask_pitch], nonzero = the 64-key block is attended
+  int64_t mask_pitch;
 };
 cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s);
 

@@ -62,14 +62,17 @@ __device__ __forceinline__ int item_work(int mode, int s, int L, int chunk_r, in
   return (int)cdiv_ll(prefix + q1, kExtendKvTile);
 }
 
-// SAGE_DECODE: the flat partition of the requests' 32-key units over CTA slots (the
-// algorithm at attn_plan).  Items come out r-major, which is also slot order, so no sort.
+// SAGE_DECODE / SAGE_SPARSE: the flat partition of the requests' 32-key units (of the
+// selected 64-key blocks only, for SAGE_SPARSE) over CTA slots (the algorithm at attn_plan).
+// Items come out r-major, which is also slot order, so no sort.
 __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* chunk_out, int* n_out) {
   const int tid = threadIdx.x, nt = blockDim.x;
   WsView ws = a.ws;
   PlanHeader* hdr = ws.hdr;
   const int B = a.batch;
-  // 1. lengths (clamped and flagged when out of range)
+  const bool sparse = a.mode == PA_MODE_SAGE_SPARSE;
+  // 1. lengths (clamped and flagged when out of range); the units of each request
+  //    (req_prefix holds them during the plan), and its selected block count (SAGE_SPARSE)
   for (int r = tid; r < B; r += nt) {
     int L = a.seq_lens[r];
     if (L < 0 || L > a.max_kv_len) {
@@ -77,27 +80,59 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
       L = max(0, min(L, a.max_kv_len));
     }
     ws.req_len[r] = L;
+    int units = (int)cdiv_ll(L, kSageUnit), nsel = 0;
+    if (sparse) {
+      const int nb = (int)cdiv_ll(L, kSageBlock);
+      const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
+      units = 0;
+      for (int b = 0; b < nb; ++b)
+        if (m[b]) {
+          ++nsel;
+          units += L - kSageBlock * b <= kSageUnit ? 1 : 2;
+        }
+    }
+    ws.req_prefix[r] = units;
+    ws.req_splits[r] = nsel;   // scratch until step 3
   }
   __syncthreads();
-  // 2. g_r = exclusive prefix sum of the units (kept in req_aux), total
   const int per_t = (B + nt - 1) / nt;
   const int r0 = min(B, tid * per_t), r1 = min(B, r0 + per_t);
+  if (sparse) {
+    // sel_base = exclusive prefix sum of the selected block counts; the block lists
+    int local_b = 0;
+    for (int r = r0; r < r1; ++r) local_b += ws.req_splits[r];
+    int total_b = 0;
+    int run_b = block_exclusive_scan(local_b, scan, &total_b);
+    for (int r = r0; r < r1; ++r) {
+      ws.sel_base[r] = run_b;
+      run_b += ws.req_splits[r];
+    }
+    if (tid == 0) ws.sel_base[B] = total_b;
+    __syncthreads();
+    for (int r = tid; r < B; r += nt) {
+      const int L = ws.req_len[r], nb = (int)cdiv_ll(L, kSageBlock);
+      const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
+      int k = ws.sel_base[r];
+      for (int b = 0; b < nb; ++b)
+        if (m[b]) ws.sel_block[k++] = b;
+    }
+  }
+  // 2. g_r = exclusive prefix sum of the units (kept in req_aux), total
   long long local = 0;
-  for (int r = r0; r < r1; ++r) local += cdiv_ll(ws.req_len[r], kSageUnit);
+  for (int r = r0; r < r1; ++r) local += ws.req_prefix[r];
   int total = 0;
   int run = block_exclusive_scan((int)local, scan, &total);
   for (int r = r0; r < r1; ++r) {
     ws.req_aux[r] = run;
-    run += (int)cdiv_ll(ws.req_len[r], kSageUnit);
+    run += ws.req_prefix[r];
   }
   const int per = (int)max(1LL, cdiv_ll(total, a.slots));
   const int used = (int)cdiv_ll(total, per);
   __syncthreads();
   // 3. pieces per request, then req_base
   for (int r = tid; r < B; r += nt) {
-    const int u = (int)cdiv_ll(ws.req_len[r], kSageUnit), g = ws.req_aux[r];
+    const int u = ws.req_prefix[r], g = ws.req_aux[r];
     ws.req_splits[r] = u > 0 ? (g + u - 1) / per - g / per + 1 : 1;
-    ws.req_prefix[r] = 0;
   }
   __syncthreads();
   int local_s = 0;
@@ -114,9 +149,9 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
     n_items = a.max_items;
   }
   __syncthreads();
-  // 4. the items and the slot of each
+  // 4. the items (key ranges; SAGE_SPARSE: unit ranges) and the slot of each
   for (int r = tid; r < B; r += nt) {
-    const int L = ws.req_len[r], u = (int)cdiv_ll(L, kSageUnit), g = ws.req_aux[r], base = ws.req_base[r];
+    const int L = ws.req_len[r], u = ws.req_prefix[r], g = ws.req_aux[r], base = ws.req_base[r];
     if (u == 0) {
       if (base < n_items) {
         ws.items[base] = make_int4(r, 0, 0, 0);
@@ -129,7 +164,8 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
       const int i = base + (c - c_first);
       if (i >= n_items) break;
       const int u0 = max(g, c * per) - g, u1 = min(g + u, (c + 1) * per) - g;
-      ws.items[i] = make_int4(r, c - c_first, u0 * kSageUnit, min(u1 * kSageUnit, L));
+      ws.items[i] = sparse ? make_int4(r, c - c_first, u0, u1)
+                           : make_int4(r, c - c_first, u0 * kSageUnit, min(u1 * kSageUnit, L));
       item_slot[i] = c;
     }
   }
@@ -140,6 +176,8 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
     const int c_prev = i > 0 ? item_slot[i - 1] : -1;
     for (int c = c_prev + 1; c <= item_slot[i]; ++c) ws.slot_first[c] = i;
   }
+  __syncthreads();
+  for (int r = tid; r < B; r += nt) ws.req_prefix[r] = 0;
   *chunk_out = per;
   *n_out = n_items;
 }
@@ -155,7 +193,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
   if (tid == 0) hdr->error_word = 0;  // every new plan starts with a clean error word
   __syncthreads();
   int chunk = 0, n_items = 0;
-  if (a.mode == PA_MODE_SAGE_DECODE) {
+  if (sage_mode(a.mode)) {
     sage_plan(a, reinterpret_cast<int*>(keys), scan, &chunk, &n_items);
   } else {
 
@@ -305,7 +343,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     hdr->chunk_tiles = chunk;
     hdr->num_sms = a.num_sms;
     hdr->max_splits = a.max_splits;
-    hdr->slots = a.mode == PA_MODE_SAGE_DECODE ? a.slots : 0;
+    hdr->slots = sage_mode(a.mode) ? a.slots : 0;
     hdr->reserved1 = 0;
   }
 }

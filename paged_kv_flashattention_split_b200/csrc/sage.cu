@@ -130,7 +130,38 @@ struct SageLaunch {
 };
 
 __device__ __forceinline__ bool sage_ws_ok(const PlanHeader* hdr) {
-  return hdr->magic == kMagic && hdr->mode == PA_MODE_SAGE_DECODE;
+  return hdr->magic == kMagic && sage_mode(hdr->mode);
+}
+
+// Tiles of an item: SAGE_DECODE items are key ranges [a0, a1), SAGE_SPARSE items unit
+// ranges [a0, a1) of the request's selected blocks (one 32-key tile per unit).
+__device__ __forceinline__ int item_tiles(bool sparse, int a0, int a1) {
+  return sparse ? a1 - a0 : (a1 - a0 + kTileKeys - 1) / kTileKeys;
+}
+
+// Tile t of an item: its first key, its key count (0 past the item) and the raw table entry
+// of its page (checked where it is used).
+struct TileRef {
+  int ks, nv, e;
+};
+__device__ __forceinline__ TileRef tile_ref(const SageLaunch& a, bool sparse, int r, int a0, int a1, int len,
+                                            int selb, int t) {
+  TileRef x{0, 0, -1};
+  const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
+  if (!sparse) {
+    x.ks = a0 + kTileKeys * t;
+    if (x.ks < a1) {
+      x.nv = min(kTileKeys, a1 - x.ks);
+      x.e = __ldg(table + (x.ks >> 6));
+    }
+  } else if (a0 + t < a1) {
+    const int u = a0 + t;
+    const int blk = __ldg(a.ws.sel_block + selb + (u >> 1));
+    x.ks = blk * kSageBlock + (u & 1) * kTileKeys;
+    x.nv = min(kTileKeys, len - x.ks);
+    x.e = __ldg(table + blk);
+  }
+  return x;
 }
 
 // The items of this CTA's slot: [first, last).
@@ -147,10 +178,11 @@ __device__ __forceinline__ bool slot_items(const SageLaunch& a, int groups, int&
 struct ItemWindow {
   int w0 = -1 << 30;
   int r = 0, kv0 = 0, kv1 = 0, base = 0, splits = 0;   // item w0 + lane
-  __device__ __forceinline__ void load(const SageLaunch& a, int w, int last, bool with_req) {
+  int len = 0, selb = 0;                                // SAGE_SPARSE producer: L_r and sel_base[r]
+  __device__ __forceinline__ void load(const SageLaunch& a, int w, int last, bool with_req, bool with_sel = false) {
     w0 = w;
     const int i = w + (threadIdx.x & 31);
-    r = kv0 = kv1 = base = splits = 0;
+    r = kv0 = kv1 = base = splits = len = selb = 0;
     if (i < last) {
       const int4 it = a.ws.items[i];
       r = it.x;
@@ -160,7 +192,22 @@ struct ItemWindow {
         base = a.ws.req_base[r];
         splits = min(a.ws.req_splits[r], a.ws.hdr->max_items - base);   // clamped only after a flagged overflow
       }
+      if (with_sel) {
+        len = a.ws.req_len[r];
+        selb = a.ws.sel_base[r];
+      }
     }
+  }
+  // item i for the producer: request, item bounds, L_r and sel_base[r]
+  __device__ __forceinline__ void get_sel(const SageLaunch& a, int i, int last, bool with_sel, int& ri, int& k0,
+                                          int& k1, int& li, int& sbi) {
+    if (i < w0 || i >= w0 + 32) load(a, i, last, false, with_sel);
+    const int l = i - w0;
+    ri = __shfl_sync(0xffffffffu, r, l);
+    k0 = __shfl_sync(0xffffffffu, kv0, l);
+    k1 = __shfl_sync(0xffffffffu, kv1, l);
+    li = __shfl_sync(0xffffffffu, len, l);
+    sbi = __shfl_sync(0xffffffffu, selb, l);
   }
   // item i (the same i on every lane): request, key range, first item and item count of its request
   __device__ __forceinline__ void get(const SageLaunch& a, int i, int last, bool with_req, int& ri, int& k0, int& k1,
@@ -248,28 +295,23 @@ __device__ __forceinline__ void produce(const SageLaunch& a, const Ring<HG, G, V
     waited = true;
   };
   ItemWindow win;
-  // raw table entry of tile tb + lane of an item (or -1 past its tiles); checked when used
-  auto entry = [&](int r, int kv0, int n_tiles, int tb) -> int {
-    const int t = tb + lane;
-    return t < n_tiles ? __ldg(a.page_table + (size_t)r * a.pt_pitch + ((kv0 + kTileKeys * t) >> 6)) : -1;
-  };
-  int r = 0, kv0 = 0, kv1 = 0, b_, s_;
-  if (first < last) win.get(a, first, last, false, r, kv0, kv1, b_, s_);
-  int e_pre = entry(r, kv0, (kv1 - kv0 + kTileKeys - 1) / kTileKeys, 0);   // first round of the next item
+  const bool sparse = hdr->mode == PA_MODE_SAGE_SPARSE;
+  int r = 0, a0 = 0, a1 = 0, len = 0, selb = 0;
+  if (first < last) win.get_sel(a, first, last, sparse, r, a0, a1, len, selb);
+  TileRef pre = tile_ref(a, sparse, r, a0, a1, len, selb, lane);   // first round of the next item
   for (int item = first; item < last && ok; ++item) {
-    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    const int n_tiles = item_tiles(sparse, a0, a1);
     const int srow = r * a.hq + grp * HG * G;
-    int rn = 0, kv0n = 0, kv1n = 0;
-    if (item + 1 < last) win.get(a, item + 1, last, false, rn, kv0n, kv1n, b_, s_);
-    const int n_tiles_n = (kv1n - kv0n + kTileKeys - 1) / kTileKeys;
-    if (n_tiles == 0 && item + 1 < last) e_pre = entry(rn, kv0n, n_tiles_n, 0);   // an empty item has no round
+    int rn = 0, a0n = 0, a1n = 0, lenn = 0, selbn = 0;
+    if (item + 1 < last) win.get_sel(a, item + 1, last, sparse, rn, a0n, a1n, lenn, selbn);
+    if (n_tiles == 0 && item + 1 < last) pre = tile_ref(a, sparse, rn, a0n, a1n, lenn, selbn, lane);   // no round
     for (int tb = 0; tb < n_tiles && ok; tb += 32) {
-      const int e = tb == 0 ? e_pre : entry(r, kv0, n_tiles, tb);
+      const TileRef tr = tb == 0 ? pre : tile_ref(a, sparse, r, a0, a1, len, selb, tb + lane);
       // the next item's first page ids, read behind this item's last round
-      if (tb + 32 >= n_tiles && item + 1 < last) e_pre = entry(rn, kv0n, n_tiles_n, 0);
+      if (tb + 32 >= n_tiles && item + 1 < last) pre = tile_ref(a, sparse, rn, a0n, a1n, lenn, selbn, lane);
       int pg = -1;
       if (tb + lane < n_tiles) {
-        if (e >= 0 && ((long long)e + 1) * kSageBlock <= a.num_slots) pg = e;
+        if (tr.e >= 0 && ((long long)tr.e + 1) * kSageBlock <= a.num_slots) pg = tr.e;
         else set_device_error(hdr, PA_ERR_DEVICE_INDEX);
       }
       constexpr bool kSfkLanes = !VPASS && HG < 4;   // K scales read by the lanes
@@ -286,14 +328,15 @@ __device__ __forceinline__ void produce(const SageLaunch& a, const Ring<HG, G, V
           break;
         }
         const int p = __shfl_sync(0xffffffffu, pg, i);
+        const int ks = __shfl_sync(0xffffffffu, tr.ks, i);
+        const int nv = __shfl_sync(0xffffffffu, tr.nv, i);
         float sf[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) sf[h] = __shfl_sync(0xffffffffu, sfk[h], i);
         if (lane == 0) {
-          const int ks = kv0 + kTileKeys * (tb + i);
           StageInfo& in = info[s];
           in.kstart = ks;
-          in.nvalid = min(kTileKeys, kv1 - ks);
+          in.nvalid = nv;
           in.page = p;
           if (kSfkLanes) {
 #pragma unroll
@@ -316,8 +359,10 @@ __device__ __forceinline__ void produce(const SageLaunch& a, const Ring<HG, G, V
       }
     }
     r = rn;
-    kv0 = kv0n;
-    kv1 = kv1n;
+    a0 = a0n;
+    a1 = a1n;
+    len = lenn;
+    selb = selbn;
   }
   if (VPASS && !waited) flush();
   if (!ok && lane == 0) {
@@ -356,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_co
   const int hkv = grp * HG + hl;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const StageInfo* info = rg.info();
+  const bool sparse = hdr->mode == PA_MODE_SAGE_SPARSE;
   const int c0 = 2 * tig, c1 = 2 * tig + 1;          // this thread's query-head columns of S^T
   // Q8^T as the B operand: b0 = Q8[head gid][32 ks + 4 tig .. +3], b1 = the same at +16; the
   // next item's are read while this item's tiles are processed
@@ -378,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_co
   uint32_t q = 0;
   for (int item = first; item < last; ++item) {
     const int r = rn, kv0 = kv0n, kv1 = kv1n;
-    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    const int n_tiles = item_tiles(sparse, kv0, kv1);
     uint32_t qb0[4], qb1[4];
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
@@ -396,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_co
     for (int t = 0; t < n_tiles; ++t, ++q) {
       const int s = q % kStages;
       if (!rg.wait(rg.full(s), (q / kStages) & 1, hdr)) return;
-      const int ks0 = info[s].kstart, page = info[s].page;
+      const int ks0 = info[s].kstart, page = info[s].page, nv = info[s].nvalid;
       if (active && page >= 0) {
         const float sfk = rg.sfk(s)[hl];
         const float sc0 = sfq0 * sfk, sc1 = sfq1 * sfk;      // fp32(sfQ sfK)
@@ -412,17 +458,18 @@ __global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_co
             ldmatrix_x4(af, kst + row * kHeadDim + ((chunk ^ (row & 7)) << 4));
             mma_s8_16832(acc, af, qb0[kk], qb1[kk]);
           }
-          const int key0 = ks0 + 16 * kb + gid, key1 = key0 + 8;
+          const int j0 = 16 * kb + gid, j1 = j0 + 8;                 // key offsets in the tile
+          const int key0 = ks0 + j0, key1 = ks0 + j1;
           // S = fp32(fp32(sfQ sfK) fp32(dot)); the int32 dot is exact and |dot| < 2^24
           const float s00 = sc0 * (float)acc[0], s01 = sc1 * (float)acc[1];
           const float s10 = sc0 * (float)acc[2], s11 = sc1 * (float)acc[3];
           if (c0 < G) {
-            if (key0 < kv1) { srow0[key0] = s00; mx0 = fmaxf(mx0, s00); }
-            if (key1 < kv1) { srow0[key1] = s10; mx0 = fmaxf(mx0, s10); }
+            if (j0 < nv) { srow0[key0] = s00; mx0 = fmaxf(mx0, s00); }
+            if (j1 < nv) { srow0[key1] = s10; mx0 = fmaxf(mx0, s10); }
           }
           if (c1 < G) {
-            if (key0 < kv1) { srow1[key0] = s01; mx1 = fmaxf(mx1, s01); }
-            if (key1 < kv1) { srow1[key1] = s11; mx1 = fmaxf(mx1, s11); }
+            if (j0 < nv) { srow1[key0] = s01; mx1 = fmaxf(mx1, s01); }
+            if (j1 < nv) { srow1[key1] = s11; mx1 = fmaxf(mx1, s11); }
           }
         }
       }
@@ -470,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 2 * SageSmem<HG, G, true>::BYTES <= 
   const bool p_lane = gid < G;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const StageInfo* info = rg.info();
+  const bool sparse = hdr->mode == PA_MODE_SAGE_SPARSE;
   float* mw = rg.red() + warp * 8;
   asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the score pass has completed and its writes are visible
   // m for the G query heads of this KV head is the maximum of the request's item maxima: each
@@ -488,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2 * SageSmem<HG, G, true>::BYTES <= 
   uint32_t q = 0;
   for (int item = first; item < last; ++item) {
     const int r = rn, kv0 = kv0n, kv1 = kv1n, base = basen, splits = splitsn;
-    const int n_tiles = (kv1 - kv0 + kTileKeys - 1) / kTileKeys;
+    const int n_tiles = item_tiles(sparse, kv0, kv1);
     {
       float m[G];
 #pragma unroll

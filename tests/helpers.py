@@ -60,18 +60,26 @@ def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 1
     o["items"] = off
     off += 16 * max_items
     off = (off + 255) // 256 * 256
-    if mode == 2:
+    if mode in (2, 3):
         o["slot_first"] = off
         off += 4 * (slots + 1)
         off = (off + 255) // 256 * 256
-    if mode in (0, 2):
+    if mode == 3:
+        mb = (max_kv_len + 63) // 64
+        o["sel_base"] = off
+        off += 4 * (batch + 1)
+        off = (off + 255) // 256 * 256
+        o["sel_block"] = off
+        off += 4 * batch * mb
+        off = (off + 255) // 256 * 256
+    if mode in (0, 2, 3):
         o["partial_o"] = off
         off += 4 * max_items * hq * head_dim
         off = (off + 255) // 256 * 256
         o["partial_lse"] = off
         off += 4 * max_items * hq
         off = (off + 255) // 256 * 256
-    if mode == 2:
+    if mode in (2, 3):
         o["item_max"] = off
         off += 4 * max_items * hq
         off = (off + 255) // 256 * 256
@@ -83,12 +91,12 @@ def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 1
     return o
 
 
-def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
+def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int, max_kv_len: int = 0):
     """Parse the plan the GPU wrote into the workspace (host copy)."""
     raw = ws.cpu().numpy().view(np.uint8)
     hdr = raw[:64].view(np.int32)
     num_items, max_items, hkv, slots = int(hdr[7]), int(hdr[8]), int(hdr[4]), int(hdr[14])
-    o = ws_offsets(mode, batch, hq, max_items, hkv=hkv, slots=slots)
+    o = ws_offsets(mode, batch, hq, max_items, hkv=hkv, slots=slots, max_kv_len=max_kv_len)
 
     def arr(name, n):
         return raw[o[name]:o[name] + 4 * n].view(np.int32).tolist()
@@ -97,8 +105,9 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int):
     return {"magic": int(hdr[0]), "mode": int(hdr[1]), "tile": int(hdr[9]), "chunk_tiles": int(hdr[10]),
             "error_word": int(hdr[11]), "num_items": num_items, "max_items": max_items,
             "req_splits": arr("req_splits", batch), "req_base": arr("req_base", batch + 1),
-            "req_len": arr("req_len", batch), "slots": slots,
-            "slot_first": arr("slot_first", slots + 1) if mode == 2 else None,
+            "req_len": arr("req_len", batch), "slots": slots, "num_sms": int(hdr[12]),
+            "slot_first": arr("slot_first", slots + 1) if mode in (2, 3) else None,
+            "sel_base": arr("sel_base", batch + 1) if mode == 3 else None,
             "items": [tuple(int(x) for x in it) for it in items]}
 
 

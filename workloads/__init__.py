@@ -23,6 +23,8 @@ Recipe (all draws from ``torch.Generator``; integers uniform and inclusive):
 * Sage: Q8, K8 uniform in [-127, 127]; V8 = E4M3(16 N(0, 1)); sfQ, sfK, sfV
   lognormal(mu=-4, sigma=0.5); v_mean ~ N(0, 0.1^2) (0.1 read as the standard
   deviation).
+* block-sparse Sage: one Bernoulli(density) mask per (request, 64-key block), drawn
+  from seed 9_000_000 + cfg (the pages measure density 0.10 and 0.125);
 * FP8 KV cache: K8, V8 = E4M3(16 N(0, 1)) (clamped to +-448, nearest-even) with
   k_scale = v_scale = 1/16, so the dequantised K, V are N(0, 1) like the bf16 pools;
   Q ~ N(0, 1) in bf16.
@@ -61,6 +63,7 @@ class Spec:
     new_hi: int = 0
     peaked_frac: float = 0.0
     peaked_scale: float = 1.0
+    density: float = 1.0      # block-sparse Sage: fraction of 64-key blocks attended
 
     @property
     def sm_scale(self) -> float:
@@ -83,6 +86,8 @@ CONFIGS = {
             page_size=64, spare_pages=0.10, layers=32),
     6: Spec("decode_fp8_llama3_8b", 6, "fp8", batch=64, len_lo=512, len_hi=8192, hq=32, hkv=8,
             page_size=16, spare_pages=0.10, layers=32),
+    7: Spec("sage_sparse_decode", 7, "sage", batch=32, len_lo=8192, len_hi=32768, hq=32, hkv=8,
+            page_size=64, spare_pages=0.05, layers=32, distinct_pools=8, density=0.125),
 }
 
 FP8_SCALE = 1.0 / 16.0   # k_scale = v_scale of the FP8 pools
@@ -164,6 +169,13 @@ def make_bf16_pools(spec: Spec, batch: Batch, layer: int, device="cpu", seed: in
     for t in (k, v):
         t.view(torch.int16)[unused] = BF16_NAN
     return k, v
+
+
+def make_block_mask(spec: Spec, batch: Batch, device="cpu", seed: int | None = None) -> torch.Tensor:
+    """uint8 [B, pitch] (pitch = the page table's, 64-key blocks = pages): 1 = block attended."""
+    g = _gen(9_000_000 + spec.cfg if seed is None else seed, "cpu")
+    m = (torch.rand(batch.page_table.shape, generator=g) < spec.density).to(torch.uint8)
+    return m.to(device)
 
 
 def make_fp8_pools(spec: Spec, batch: Batch, layer: int, device="cpu", seed: int | None = None):
