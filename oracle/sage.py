@@ -146,3 +146,36 @@ def kv_store_sage(k8_pool, v8_pool, sf_k, out_cache_loc, k8_new, v8_new, sf_k_ne
             if sf_k_new is not None and slot % k_block == 0:
                 sf[slot // k_block] = sf_k_new[t]
     return k, v, sf
+
+
+def sage_extend(q8, sf_q, cu_seqlens_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_lens,
+                page_size: int, k_block: int = 64) -> np.ndarray:
+    """Sage EXTEND (prefill over a cached prefix); returns O [T, Hq, D] float64.
+
+    The Sage formula of ``sage_row`` for every new token: row i of request r (Q8 row
+    cu_seqlens_q[r] + i, scale sf_q[row][h], blkQ = one row) sits at absolute position
+    p_r + i, p_r = L_r - n_r, and sees keys 0 .. p_r + i (the bottom-right causal reading
+    of ``oracle.attention.extend``); its row max and row sum run over those keys.  This
+    is the variant the pages measure at S = 10800 ("FlashInfer PrimTS, Sage Attention ...",
+    performance item 2); the kernel for it runs on the prefill path.
+    """
+    T, Hq, D = q8.shape
+    Hkv = k8_pool.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((T, Hq, D))
+    for r in range(len(seq_lens)):
+        q0, q1 = int(cu_seqlens_q[r]), int(cu_seqlens_q[r + 1])
+        L = int(seq_lens[r])
+        p = L - (q1 - q0)
+        slots = gather_slots(page_table, L, page_size, r)
+        blocks = slots // k_block
+        for hk in range(Hkv):
+            vm = None if v_mean is None else v_mean[hk]
+            for i in range(q1 - q0):
+                vis = slots[: p + i + 1]
+                k8 = k8_pool[vis, hk, :]
+                v8 = v8_pool[vis, hk, :]
+                sfk = sf_k[blocks[: p + i + 1], hk]
+                for h in range(hk * G, (hk + 1) * G):
+                    out[q0 + i, h] = sage_row(q8[q0 + i, h], k8, v8, sf_q[q0 + i, h], sfk, sf_v[hk], vm)
+    return out

@@ -217,3 +217,38 @@ def test_block_sparse_all_ones_is_dense_and_none_selected_is_v_mean():
     assert np.array_equal(dense, ones)
     none = sage.sage_decode(q8, sfq, k8, v8, sfk, sfv, vm, table, lens, 64, block_mask=np.zeros((2, 4), int))
     assert np.array_equal(none, np.repeat(vm[None, :, :], 2, 0).repeat(hq // hkv, 1))
+
+
+def test_sage_extend_rows_equal_decodes_of_their_visible_prefix():
+    rng = np.random.default_rng(43)
+    lens_new, prefix, hq, hkv = [3, 1, 2], [130, 0, 64], 4, 2
+    lens = [p + n for p, n in zip(prefix, lens_new)]
+    _, k8, v8, _, sfk, sfv, vm, table = _sage_case(rng, lens, hq, hkv)
+    T = sum(lens_new)
+    q8 = rng.integers(-127, 128, (T, hq, 128)).astype(np.int8)
+    sfq = np.exp(-4 + 0.5 * rng.standard_normal((T, hq))).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(lens_new)])
+    o = sage.sage_extend(q8, sfq, cu, k8, v8, sfk, sfv, vm, table, lens, 64)
+    for r in range(len(lens)):
+        for i in range(lens_new[r]):
+            row = cu[r] + i
+            d = sage.sage_decode(q8[row:row + 1], sfq[row:row + 1], k8, v8, sfk, sfv, vm, table[r:r + 1],
+                                 [prefix[r] + i + 1], 64)
+            assert np.array_equal(o[row], d[0])
+
+
+def test_sage_extend_ignores_keys_after_the_row():
+    rng = np.random.default_rng(44)
+    lens_new, prefix, hq, hkv = [5], [60], 2, 1
+    lens = [65]
+    _, k8, v8, _, sfk, sfv, vm, table = _sage_case(rng, lens, hq, hkv)
+    q8 = rng.integers(-127, 128, (5, hq, 128)).astype(np.int8)
+    sfq = np.exp(-4 + 0.5 * rng.standard_normal((5, hq))).astype(np.float32)
+    cu = np.array([0, 5])
+    o1 = sage.sage_extend(q8, sfq, cu, k8, v8, sfk, sfv, vm, table, lens, 64)
+    k8b, v8b = k8.copy(), v8.copy()
+    last = table[0][1] * 64 + 0                      # key 64 (the last) lives in the second page
+    k8b[last] = 5
+    v8b[last] = 0x38
+    o2 = sage.sage_extend(q8, sfq, cu, k8b, v8b, sfk, sfv, vm, table, lens, 64)
+    assert np.array_equal(o1[:4], o2[:4]) and not np.array_equal(o1[4], o2[4])
