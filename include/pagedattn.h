@@ -303,6 +303,30 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
                                  uint16_t* d_out, pa_stream_t stream);
 
 /*
+ * attn_extend_paged_sage - 8-bit Sage EXTEND (prefill over a cached prefix) for one layer:
+ * the Sage formula of attn_decode_paged_sage for every new token, over the keys it sees
+ * (new token i of request r at absolute position p_r + i sees keys j <= p_r + i, the
+ * bottom-right causal alignment of attn_extend_paged):
+ *   S_j = sfQ[row][h] sfK[slot_j / 64][h_kv] (Q8 . K8_j),  m = max S_j,  l = sum exp(S_j - m),
+ *   O[d] = sfV[h_kv][d] (sum_j E4M3(448 exp(S_j - m)) V8_j[d]) / (448 l) + v_mean[h_kv][d].
+ * The dense Sage variant the pages measure at S = 10800 ("FlashInfer PrimTS, Sage
+ * Attention ...", performance item 2).  Two passes over the key tiles of each query tile
+ * (the row max first, then P8 and O) on the tcgen05 tensor cores; the 8-bit operands are
+ * converted to f16 on chip, which holds them exactly.
+ *
+ * params, d_ws    an EXTEND plan (attn_plan, mode PA_MODE_EXTEND) with page_size 64.
+ * d_q8 int8 [max_q_tokens][Hq][D] (rows cu_seqlens_q[r] .. of request r), d_sf_q fp32
+ *                 [max_q_tokens][Hq] (one scale per token and head).
+ * Pools, sfK, sfV, v_mean and the table as for attn_decode_paged_sage; d_out bf16
+ * [max_q_tokens][Hq][D].  q8, the pools and out 16-byte aligned.
+ */
+pa_status attn_extend_paged_sage(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                                 const int8_t* d_q8, const float* d_sf_q, const int8_t* d_k8_pool,
+                                 const uint8_t* d_v8_pool, const float* d_sf_k, const float* d_sf_v,
+                                 const float* d_v_mean, int64_t num_slots, const int32_t* d_page_table,
+                                 int64_t pt_pitch, uint16_t* d_out, pa_stream_t stream);
+
+/*
  * attn_decode_paged_noalloc - attn_plan followed by attn_decode_paged in one
  * call, for callers that cannot allocate device memory (a host framework that
  * owns every device allocation and offers no allocator, a plugin that must not

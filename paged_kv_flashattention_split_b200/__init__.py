@@ -26,6 +26,7 @@ from ._binding import (  # noqa: F401
     attn_decode_paged_noalloc,
     attn_decode_paged_sage,
     attn_extend_paged,
+    attn_extend_paged_sage,
     attn_kv_store,
     attn_kv_store_sage,
     attn_plan,

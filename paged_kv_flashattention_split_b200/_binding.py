@@ -22,7 +22,7 @@ PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE, PA_MODE_SAGE_SPARSE = 0, 1,
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
             "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store",
-            "attn_kv_store_sage", "attn_decode_paged_fp8", "attn_plan_sage_sparse")
+            "attn_kv_store_sage", "attn_decode_paged_fp8", "attn_plan_sage_sparse", "attn_extend_paged_sage")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
                                              _P]),
             "attn_decode_paged_sage": (_I32, [PP, _P, _SZ, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64,
                                               _P, _P]),
+            "attn_extend_paged_sage": (_I32, [PP, _P, _SZ, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P, _P]),
             "attn_debug_gather": (_I32, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _I64, _P, _I64,
                                          _P, _P, _P]),
             "pa_read_device_error": (_I32, [_P, _P]),
@@ -178,6 +179,18 @@ def attn_decode_paged_sage(params, ws, q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v
                                       _ptr(sf_v), _ptr(v_mean), int(num_slots), _ptr(page_table),
                                       int(pt_pitch), _ptr(out), _stream(stream))
     return _check(st, "attn_decode_paged_sage", raise_on_error)
+
+
+def attn_extend_paged_sage(params, ws, q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, out,
+                           num_slots=None, pt_pitch=None, stream=None, raise_on_error=True) -> int:
+    """8-bit Sage EXTEND over an EXTEND plan with page size 64; q8 int8 [T, Hq, D], out bf16."""
+    num_slots = k8_pool.shape[0] if num_slots is None else num_slots
+    pt_pitch = page_table.shape[-1] if pt_pitch is None else pt_pitch
+    st = lib().attn_extend_paged_sage(ctypes.byref(params), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _ptr(q8), _ptr(sf_q), _ptr(k8_pool), _ptr(v8_pool), _ptr(sf_k),
+                                      _ptr(sf_v), _ptr(v_mean), int(num_slots), _ptr(page_table),
+                                      int(pt_pitch), _ptr(out), _stream(stream))
+    return _check(st, "attn_extend_paged_sage", raise_on_error)
 
 
 def attn_debug_gather(seq_lens, r, h_kv, hkv, page_size, max_len, k_pool, page_table, slots_out,

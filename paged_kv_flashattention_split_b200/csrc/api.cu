@@ -357,6 +357,46 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
   return from_cuda(launch_sage(a, (cudaStream_t)stream));
 }
 
+pa_status attn_extend_paged_sage(const pa_plan_params* params, const void* d_ws, size_t ws_bytes,
+                                 const int8_t* d_q8, const float* d_sf_q, const int8_t* d_k8_pool,
+                                 const uint8_t* d_v8_pool, const float* d_sf_k, const float* d_sf_v,
+                                 const float* d_v_mean, int64_t num_slots, const int32_t* d_page_table,
+                                 int64_t pt_pitch, uint16_t* d_out, pa_stream_t stream) {
+  Derived d;
+  pa_status st = derive(params, &d);
+  if (st != PA_OK) return st;
+  if (params->mode != PA_MODE_EXTEND) return PA_ERR_WORKSPACE;
+  if (params->page_size != kSageBlock) return PA_ERR_UNSUPPORTED;   // a page is one sfK block
+  if (!d_ws || !d_q8 || !d_sf_q || !d_k8_pool || !d_v8_pool || !d_sf_k || !d_sf_v || !d_page_table || !d_out)
+    return PA_ERR_INVALID;
+  if (!aligned16(d_ws) || !aligned16(d_q8) || !aligned16(d_k8_pool) || !aligned16(d_v8_pool) || !aligned16(d_out))
+    return PA_ERR_INVALID;
+  if (num_slots < kSageBlock || num_slots % kSageBlock != 0 || num_slots >= (1LL << 31) || pt_pitch < 1)
+    return PA_ERR_INVALID;
+  const long long need_pitch = ((long long)params->max_kv_len + params->page_size - 1) / params->page_size;
+  if (pt_pitch < need_pitch) return PA_ERR_INVALID;
+  if (ws_bytes < d.layout.total) return PA_ERR_WORKSPACE;
+  if ((st = check_arch()) != PA_OK) return st;
+  SageExtendArgs a;
+  a.ws = ws_view(const_cast<void*>(d_ws), d.layout);
+  a.q8 = d_q8;
+  a.sf_q = d_sf_q;
+  a.k8 = d_k8_pool;
+  a.v8 = d_v8_pool;
+  a.sf_k = d_sf_k;
+  a.sf_v = d_sf_v;
+  a.v_mean = d_v_mean;
+  a.num_slots = num_slots;
+  a.page_table = d_page_table;
+  a.pt_pitch = pt_pitch;
+  a.q_rows = params->max_q_tokens;
+  a.out = d_out;
+  a.hq = params->hq;
+  a.hkv = params->hkv;
+  a.max_items = d.max_items;
+  return from_cuda(launch_sage_extend(a, (cudaStream_t)stream));
+}
+
 pa_status attn_kv_store(const uint16_t* d_k_new, const uint16_t* d_v_new, const int32_t* d_out_cache_loc,
                         int64_t n_tokens, int32_t hkv, int32_t head_dim, uint16_t* d_k_pool, uint16_t* d_v_pool,
                         int64_t num_slots, void* d_ws, pa_stream_t stream) {

@@ -82,6 +82,24 @@ struct ExtendArgs {
 };
 cudaError_t launch_extend(const ExtendArgs& a, cudaStream_t s);
 
+struct SageExtendArgs {
+  WsView ws;
+  const int8_t* q8;        // [q_rows][Hq][D]
+  const float* sf_q;       // [q_rows][Hq]
+  const int8_t* k8;
+  const uint8_t* v8;
+  const float* sf_k;
+  const float* sf_v;
+  const float* v_mean;
+  int64_t num_slots;
+  const int32_t* page_table;
+  int64_t pt_pitch;
+  int64_t q_rows;
+  uint16_t* out;           // bf16 [q_rows][Hq][D]
+  int hq, hkv, max_items;
+};
+cudaError_t launch_sage_extend(const SageExtendArgs& a, cudaStream_t s);
+
 struct StoreLaunch {
   const void* k_new;
   const void* v_new;

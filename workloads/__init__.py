@@ -88,6 +88,8 @@ CONFIGS = {
             page_size=16, spare_pages=0.10, layers=32),
     7: Spec("sage_sparse_decode", 7, "sage", batch=32, len_lo=8192, len_hi=32768, hq=32, hkv=8,
             page_size=64, spare_pages=0.05, layers=32, distinct_pools=8, density=0.125),
+    8: Spec("sage_extend_prefix", 8, "extend", batch=8, len_lo=0, len_hi=4096, hq=32, hkv=8,
+            page_size=64, spare_pages=0.10, new_lo=128, new_hi=2048, layers=32),
 }
 
 FP8_SCALE = 1.0 / 16.0   # k_scale = v_scale of the FP8 pools
@@ -211,10 +213,11 @@ class SageLayer:
 
 
 def make_sage_layer(spec: Spec, batch: Batch, layer: int, device="cpu", k_block: int = 64,
-                    seed: int | None = None) -> SageLayer:
-    """8-bit Q/K/V, their scales and v_mean for one layer (see module docstring)."""
+                    seed: int | None = None, q_rows: int | None = None) -> SageLayer:
+    """8-bit Q/K/V, their scales and v_mean for one layer (see module docstring); q_rows query
+    rows (default: one per request, the decode case; the new tokens for EXTEND)."""
     g = _gen(1000 + 100 * spec.cfg + layer if seed is None else seed, device)
-    B, Hq, Hkv, D = spec.batch, spec.hq, spec.hkv, spec.head_dim
+    B, Hq, Hkv, D = spec.batch if q_rows is None else q_rows, spec.hq, spec.hkv, spec.head_dim
     S = batch.num_slots
 
     def ri(shape):
