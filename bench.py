@@ -10,7 +10,7 @@ total, so every step reads inputs far larger than L2).  The metric is the
 decode's algorithmic KV bandwidth: K and V rows read once, slot ids, Q and O,
 divided by the device time.  Other workloads (``--workload``):
 decode_long_llama3_70b, extend_prefix, sage_decode, sage_sparse_decode,
-decode_fp8_llama3_8b, decode_tiny.
+sage_extend_prefix, decode_fp8_llama3_8b, decode_tiny.
 
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
 replica on its own GPU (no collective on the data path); the time is the max
@@ -114,6 +114,7 @@ KERNEL_SOURCES = {
     "extend_prefix": ("extend.cu", "common.cuh", "tma.cuh"),
     "sage_decode": ("sage.cu", "common.cuh", "tma.cuh"),
     "sage_sparse_decode": ("sage.cu", "common.cuh", "tma.cuh"),
+    "sage_extend_prefix": ("sage_extend.cu", "common.cuh", "tma.cuh"),
 }
 
 
@@ -385,6 +386,73 @@ class ExtendWorkload(DecodeWorkload):
         return flops, time.perf_counter() - t0, f"oracle.attention.extend, one query head at a time, {r * spec.hq + h} (request, head) pairs of layer 0"
 
 
+class SageExtendWorkload(ExtendWorkload):
+    """plan + L layer calls of the 8-bit Sage extend (page size 64), each layer with its own pools."""
+
+    def __init__(self, spec: wl.Spec, device: str):
+        import paged_kv_flashattention_split_b200 as pa
+        self.pa, self.spec, self.dev = pa, spec, device
+        self.batch = wl.make_batch(spec, device)
+        self.total_q = int(self.batch.cu_seqlens_q[-1])
+        n_pools = spec.distinct_pools or spec.layers
+        self.layers_data = [wl.make_sage_layer(spec, self.batch, l, device, q_rows=self.total_q) for l in range(n_pools)]
+        self.q = [self.layers_data[l % n_pools].q8 for l in range(spec.layers)]
+        self.out = [torch.empty((self.total_q, spec.hq, spec.head_dim), dtype=torch.bfloat16, device=device)
+                    for _ in range(spec.layers)]
+        self.params = pa.make_params(pa.PA_MODE_EXTEND, spec.batch, spec.hq, spec.hkv, spec.head_dim, 64,
+                                     max_kv_len=self.batch.page_table.shape[1] * 64, max_q_tokens=self.total_q)
+        self.ws = torch.zeros(pa.pa_plan_workspace_size(self.params), dtype=torch.uint8, device=device)
+        L = self.batch.seq_lens.cpu().tolist()
+        n = self.batch.new_lens.cpu().tolist()
+        pairs = sum(ni * (Li - ni) + ni * (ni + 1) // 2 for Li, ni in zip(L, n))   # unmasked (q, k) pairs
+        # QK and PV over the unmasked pairs (the row-max pass is this design's own extra work)
+        self.layer_flops = 4.0 * spec.head_dim * spec.hq * pairs
+        self.step_flops = self.layer_flops * spec.layers
+        self.layer_bytes = self.layer_flops
+        self.step_bytes = self.step_flops
+        self.unit, self.scale = "TFLOP/s", 1e12
+        self.launches_per_step = 1 + spec.layers
+
+    def layer(self, l):
+        d = self.layers_data[l % len(self.layers_data)]
+        self.pa.attn_extend_paged_sage(self.params, self.ws, d.q8, d.sf_q, d.k8, d.v8, d.sf_k, d.sf_v, d.v_mean,
+                                       self.batch.page_table, self.out[l])
+
+    def setup_e2e(self):
+        self.h_q = [x.cpu().pin_memory() for x in self.q]
+        self.h_lens = self.batch.seq_lens.cpu().pin_memory()
+        self.h_table = self.batch.page_table.cpu().pin_memory()
+        self.h_cu = self.batch.cu_seqlens_q.cpu().pin_memory()
+        self.h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in self.out]
+        self.e2e_h2d = (sum(x.numel() for x in self.h_q) + self.h_lens.numel() * 4 + self.h_table.numel() * 4
+                        + self.h_cu.numel() * 4)
+        self.e2e_d2h = sum(x.numel() * 2 for x in self.h_out)
+
+    def oracle_sample(self, seconds=12.0):
+        from oracle import sage as osg
+        spec = self.spec
+        d = self.layers_data[0]
+        host = {k: getattr(d, k).cpu().numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+        cu = self.batch.cu_seqlens_q.cpu().numpy()
+        table = self.batch.page_table.cpu().numpy()
+        lens = self.batch.seq_lens.cpu().numpy()
+        G = spec.hq // spec.hkv
+        flops, r, h = 0.0, 0, 0
+        t0 = time.perf_counter()
+        while (time.perf_counter() - t0) < seconds and r < spec.batch:
+            q0, q1 = int(cu[r]), int(cu[r + 1])
+            hk = h // G
+            osg.sage_extend(host["q8"][q0:q1, h:h + 1], host["sf_q"][q0:q1, h:h + 1], np.array([0, q1 - q0]),
+                            host["k8"][:, hk:hk + 1], host["v8"][:, hk:hk + 1], host["sf_k"][:, hk:hk + 1],
+                            host["sf_v"][hk:hk + 1], host["v_mean"][hk:hk + 1], table[r:r + 1], lens[r:r + 1], 64)
+            nn = q1 - q0
+            flops += 4.0 * spec.head_dim * (nn * (int(lens[r]) - nn) + nn * (nn + 1) // 2)
+            h += 1
+            if h == spec.hq:
+                h, r = 0, r + 1
+        return flops, time.perf_counter() - t0, f"oracle.sage.sage_extend, one query head at a time, {r * spec.hq + h} (request, head) pairs of layer 0"
+
+
 class SageSparseWorkload(SageWorkload):
     """plan (with the batch's block mask) + L layer calls of the block-sparse Sage decode."""
 
@@ -491,6 +559,7 @@ WORKLOADS = {
     "extend_prefix": (3, ExtendWorkload),
     "decode_fp8_llama3_8b": (6, Fp8DecodeWorkload),
     "sage_sparse_decode": (7, SageSparseWorkload),
+    "sage_extend_prefix": (8, SageExtendWorkload),
     "sage_decode": (5, SageWorkload),
     "decode_llama3_8b": (2, DecodeWorkload),
     "decode_long_llama3_70b": (4, DecodeWorkload),
@@ -633,6 +702,7 @@ def main():
         "vs_baseline": None,
         "dtype": {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
                   "sage_sparse_decode": "int8/e4m3 in, fp32 math, bf16 out",
+                  "sage_extend_prefix": "int8/e4m3 in, f16 tensor-core math (exact), fp32 accumulation, bf16 out",
                   "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}.get(
                       args.workload, "bf16"),
         "data": "synthetic",
@@ -643,6 +713,7 @@ def main():
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
             "step": "attn_plan + %d x %s" % (spec.layers, {"sage_decode": "attn_decode_paged_sage",
                                                             "sage_sparse_decode": "attn_decode_paged_sage (block-sparse plan)",
+                                                            "sage_extend_prefix": "attn_extend_paged_sage",
                                                             "extend_prefix": "attn_extend_paged",
                                                             "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}.get(
                                                                args.workload, "attn_decode_paged")),
@@ -654,6 +725,7 @@ def main():
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": {"sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
                        "sage_sparse_decode": "attn_decode_paged_sage call, block-sparse plan (score + value + merge kernels)",
+                       "sage_extend_prefix": "sage_extend_kernel (one launch per attn_extend_paged_sage call; 3 contractions per tile pair, 2 counted)",
                        "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
                        "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}.get(
                            args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
@@ -702,6 +774,22 @@ def run_reference(args, spec, cls):
             keys = L if mask is None else sum(min(64, L - 64 * b) for b in range(-(-L // 64)) if mask[r][b])
             return float(keys) * per_key
         per_step, what = 2, "requests"
+    elif spec.mode == "extend" and args.workload == "sage_extend_prefix":
+        cu = batch.cu_seqlens_q.numpy()
+        d = wl.make_sage_layer(spec, batch, 0, "cpu", q_rows=int(cu[-1]))
+        host = {k: getattr(d, k).numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+        unit, scale = "TFLOP/s", 1e12
+
+        def one(i):
+            r, h = (i // spec.hq) % spec.batch, i % spec.hq
+            hk = h // G
+            q0, q1 = int(cu[r]), int(cu[r + 1])
+            osg.sage_extend(host["q8"][q0:q1, h:h + 1], host["sf_q"][q0:q1, h:h + 1], np.array([0, q1 - q0]),
+                            host["k8"][:, hk:hk + 1], host["v8"][:, hk:hk + 1], host["sf_k"][:, hk:hk + 1],
+                            host["sf_v"][hk:hk + 1], host["v_mean"][hk:hk + 1], table[r:r + 1], lens[r:r + 1], 64)
+            n = q1 - q0
+            return 4.0 * spec.head_dim * (n * (int(lens[r]) - n) + n * (n + 1) // 2)
+        per_step, what = 1, "(request, query head) pairs"
     elif spec.mode == "extend":
         k, v = wl.make_bf16_pools(spec, batch, 0, "cpu")
         cu = batch.cu_seqlens_q.numpy()
