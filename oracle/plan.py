@@ -9,25 +9,19 @@ SGLang: Grundlagen", the FlashAttentionMetadata paragraph).  They give no
 algorithm, so the algorithm below is this library's own; the CUDA plan kernel
 must reproduce it bit for bit.
 
-DECODE (split-KV work list)
-  T        = max(64, page_size)                  keys per tile
-  HG       = the largest of 8, 4, 2, 1 dividing Hkv   (KV heads one CTA covers)
-  groups   = Hkv / HG                            CTAs per work item
-  tiles_r  = ceil(L_r / T)
-  total    = sum_r tiles_r * groups              units of work
-  slots    = num_sms * 4                         CTAs one decode launch aims for
-  chunk    = max(1, ceil(total / slots))         tiles per split
-  L_r == 0 : one split, the empty range [0, 0)
-  else     : splits_r = ceil(tiles_r / chunk), chunk_r = chunk;
-             if splits_r > max_splits: chunk_r = ceil(tiles_r / max_splits),
-                                       splits_r = ceil(tiles_r / chunk_r)
-             split s covers keys [s*chunk_r*T, min((s+1)*chunk_r*T, L_r))
-  items (r, s, kv_begin, kv_end), generated r-major then s, are sorted by
-  key length descending, ties by generation order (longest first, so that the
-  hardware's in-order block dispatch is a longest-processing-time schedule).
-  req_base = exclusive prefix sum of splits_r (the merge's index of split 0).
-  Bound used to size the grid and the workspace:
-  num_items <= ceil(slots / groups) + B.
+DECODE (split-KV work list: a flat, balanced partition over CTA slots)
+  T        = max(64, page_size)                  keys per unit (a tile)
+  HG       = the largest of 8, 4, 2, 1 dividing Hkv   (KV heads one work item covers)
+  groups   = Hkv / HG
+  C        = max(1, floor(num_sms * 2 / groups)) CTA slots
+  units_r  = ceil(L_r / T)
+  the flat partition below (SAGE_DECODE) with unit T: slot c takes the global
+  units [c per, (c+1) per), per = max(1, ceil(sum_r units_r / C)); each piece of a
+  request inside one slot is an item (r, s, T u0, min(T u1, L_r)); an empty request
+  is one item (r, 0, 0, 0); items r-major then s (slot order); slot_first; req_base.
+  Every slot streams at most per tiles, so the slots finish together, and a request
+  is split only where a slot boundary falls inside it (no split cap is needed).
+  Bound: num_items <= C + B.
 
 EXTEND (query-tile work list)
   n_r = cu[r+1] - cu[r], p_r = L_r - n_r, query tiles of 128 rows:
@@ -38,8 +32,7 @@ EXTEND (query-tile work list)
 
 SAGE_DECODE (flat, balanced partition over CTA slots)
   U        = 32 keys per unit; units_r = ceil(L_r / U)
-  HG, groups as for DECODE (a CTA covers HG KV heads of one slot)
-  C        = max(1, floor(num_sms * 2 / groups))     CTA slots (one wave of
+  HG, groups, C as for DECODE (a CTA covers HG KV heads of one slot; one wave of
                                                    two CTAs per SM)
   g_r      = sum_{r' < r} units_r'                 request r's first unit in
                                                    the concatenated sequence
@@ -70,9 +63,8 @@ from __future__ import annotations
 
 MODE_DECODE, MODE_EXTEND, MODE_SAGE_DECODE, MODE_SAGE_SPARSE = 0, 1, 2, 3
 DECODE_MIN_TILE = 64
-DECODE_CTAS_PER_SM = 4
 SAGE_UNIT = 32
-SAGE_CTAS_PER_SM = 2
+CTAS_PER_SM = 2
 EXTEND_Q_TILE = 128
 EXTEND_KV_TILE = 128
 
@@ -93,31 +85,29 @@ def decode_head_groups(hkv: int) -> int:
     raise ValueError("hkv must be positive")
 
 
-def sage_slots(hkv: int, num_sms: int) -> int:
-    """CTA slots of a Sage plan: max(1, floor(num_sms * 2 / groups))."""
-    return max(1, num_sms * SAGE_CTAS_PER_SM // decode_head_groups(hkv))
+def flat_slots(hkv: int, num_sms: int) -> int:
+    """CTA slots of a flat partition (DECODE, SAGE_DECODE, SAGE_SPARSE): max(1, floor(num_sms * 2 / groups))."""
+    return max(1, num_sms * CTAS_PER_SM // decode_head_groups(hkv))
 
 
 def max_items(mode: int, batch: int, hkv: int, num_sms: int, max_q_tokens: int = 0) -> int:
     """The host-side bound on the number of work items for a plan of this shape."""
-    if mode == MODE_DECODE:
-        return _cdiv(num_sms * DECODE_CTAS_PER_SM, decode_head_groups(hkv)) + batch
-    if mode in (MODE_SAGE_DECODE, MODE_SAGE_SPARSE):
-        return sage_slots(hkv, num_sms) + batch
+    if mode in (MODE_DECODE, MODE_SAGE_DECODE, MODE_SAGE_SPARSE):
+        return flat_slots(hkv, num_sms) + batch
     if mode == MODE_EXTEND:
         return _cdiv(max_q_tokens, EXTEND_Q_TILE) + batch
     raise ValueError("unknown mode")
 
 
 def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, num_sms: int,
-         max_splits: int = 1 << 30, max_q_tokens: int = 0, block_mask=None):
+         max_q_tokens: int = 0, block_mask=None):
     """Return the plan as a dict of plain Python ints and lists.
 
-    Keys: ``tile``, ``chunk_tiles`` (DECODE: tiles per split; SAGE_DECODE:
-    units per slot; 0 otherwise), ``req_splits``, ``req_base`` (length B + 1),
-    ``items`` (list of 4-tuples, in execution order), ``num_items`` and, for
-    SAGE_DECODE and SAGE_SPARSE, ``slot_first`` (length C + 1); for SAGE_SPARSE also
-    ``sel_base`` (length B + 1) and ``sel_block``.
+    Keys: ``tile``, ``chunk_tiles`` (DECODE: tiles per slot; SAGE_DECODE: units per
+    slot; 0 otherwise), ``req_splits``, ``req_base`` (length B + 1), ``items`` (list
+    of 4-tuples, in execution order), ``num_items`` and, for DECODE, SAGE_DECODE and
+    SAGE_SPARSE, ``slot_first`` (length C + 1); for SAGE_SPARSE also ``sel_base``
+    (length B + 1) and ``sel_block``.
     """
     L = [int(x) for x in seq_lens]
     B = len(L)
@@ -127,32 +117,13 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
     splits = [0] * B
     chunk = 0
     tile = 0
-    if mode == MODE_SAGE_DECODE:
-        return _sage_plan(L, hkv, num_sms)
-    if mode == MODE_SAGE_SPARSE:
-        return _sage_plan(L, hkv, num_sms, block_mask)
     if mode == MODE_DECODE:
-        tile = decode_tile(page_size)
-        tiles = [_cdiv(x, tile) for x in L]
-        total = sum(tiles) * decode_head_groups(hkv)
-        slots = num_sms * DECODE_CTAS_PER_SM
-        chunk = max(1, _cdiv(total, slots))
-        for r in range(B):
-            if tiles[r] == 0:
-                splits[r] = 1
-                gen.append((0, (r, 0, 0, 0)))
-                continue
-            chunk_r = chunk
-            s_r = _cdiv(tiles[r], chunk_r)
-            if s_r > max_splits:
-                chunk_r = _cdiv(tiles[r], max_splits)
-                s_r = _cdiv(tiles[r], chunk_r)
-            splits[r] = s_r
-            for s in range(s_r):
-                a = s * chunk_r * tile
-                b = min((s + 1) * chunk_r * tile, L[r])
-                gen.append((b - a, (r, s, a, b)))
-    elif mode == MODE_EXTEND:
+        return _flat_plan(L, decode_tile(page_size), flat_slots(hkv, num_sms))
+    if mode == MODE_SAGE_DECODE:
+        return _flat_plan(L, SAGE_UNIT, flat_slots(hkv, num_sms))
+    if mode == MODE_SAGE_SPARSE:
+        return _flat_plan(L, SAGE_UNIT, flat_slots(hkv, num_sms), block_mask)
+    if mode == MODE_EXTEND:
         tile = EXTEND_KV_TILE
         cu = [int(x) for x in cu_seqlens_q]
         for r in range(B):
@@ -177,12 +148,13 @@ def plan(mode: int, seq_lens, cu_seqlens_q=None, *, hkv: int, page_size: int, nu
             "items": items, "num_items": len(items)}
 
 
-def _sage_plan(L, hkv: int, num_sms: int, block_mask=None):
-    """The flat partition of SAGE_DECODE / SAGE_SPARSE (module docstring), unit by unit."""
+def _flat_plan(L, U: int, C: int, block_mask=None):
+    """The flat partition of DECODE / SAGE_DECODE / SAGE_SPARSE (module docstring) over
+    C slots, with units of U keys, unit by unit."""
     B = len(L)
     sel = None
     if block_mask is None:
-        units = [_cdiv(x, SAGE_UNIT) for x in L]
+        units = [_cdiv(x, U) for x in L]
     else:
         sel, units = [], []
         for r in range(B):
@@ -190,7 +162,6 @@ def _sage_plan(L, hkv: int, num_sms: int, block_mask=None):
             blocks = [b for b in range(nb) if block_mask[r][b]]
             sel.append(blocks)
             units.append(sum(1 if L[r] - 2 * SAGE_UNIT * b <= SAGE_UNIT else 2 for b in blocks))
-    C = sage_slots(hkv, num_sms)
     total = sum(units)
     per = max(1, _cdiv(total, C))
     used = _cdiv(total, per)
@@ -208,7 +179,7 @@ def _sage_plan(L, hkv: int, num_sms: int, block_mask=None):
             u0 = max(g, c * per) - g
             u1 = min(g + units[r], (c + 1) * per) - g
             if sel is None:
-                items.append((r, s, SAGE_UNIT * u0, min(SAGE_UNIT * u1, L[r])))
+                items.append((r, s, U * u0, min(U * u1, L[r])))
             else:
                 items.append((r, s, u0, u1))
             item_slot.append(c)
@@ -220,7 +191,7 @@ def _sage_plan(L, hkv: int, num_sms: int, block_mask=None):
     base = [0] * (B + 1)
     for r in range(B):
         base[r + 1] = base[r] + splits[r]
-    out = {"tile": SAGE_UNIT, "chunk_tiles": per, "req_splits": splits, "req_base": base,
+    out = {"tile": U, "chunk_tiles": per, "req_splits": splits, "req_base": base,
            "items": items, "num_items": len(items), "slot_first": slot_first}
     if sel is not None:
         sb = [0] * (B + 1)
