@@ -92,7 +92,7 @@ typedef struct {
   int32_t max_kv_len;    /* upper bound on every seq_lens[r]; longer lengths are clamped and flagged */
   int32_t max_q_tokens;  /* EXTEND: upper bound on sum of new tokens (sizes the grid); else 0 */
   int32_t num_sms;       /* SMs the plan schedules for; 0 = query the current device */
-  int32_t max_splits;    /* DECODE: cap on splits per request (0 = 128); EXTEND: 0 or 1; SAGE: 0 */
+  int32_t max_splits;    /* DECODE and SAGE: 0 (the flat partition needs no cap); EXTEND: 0 or 1 */
   int32_t sage_k_block;  /* SAGE: keys per sfK block, must be 64; else 0 */
   int32_t reserved;      /* must be 0 */
 } pa_plan_params;
@@ -119,51 +119,43 @@ pa_status pa_plan_workspace_size(const pa_plan_params* params, size_t* bytes);
  * d_ws           device workspace of ws_bytes >= pa_plan_workspace_size().
  *
  * One single-CTA kernel computes, from the lengths alone (integer arithmetic):
- *   DECODE: T = max(64, P) keys per tile, tiles_r = ceil(L_r / T); one CTA
- *     covers HG = the largest of 8, 4, 2, 1 dividing Hkv KV heads, so an item
- *     takes groups = Hkv / HG CTAs; total = sum tiles_r * groups,
- *     slots = num_sms * 4, chunk = max(1, ceil(total / slots)) tiles per split;
- *     L_r == 0 gives one empty split; otherwise splits_r = ceil(tiles_r / chunk)
- *     and, if that exceeds max_splits, chunk_r = ceil(tiles_r / max_splits),
- *     splits_r = ceil(tiles_r / chunk_r); split s covers keys
- *     [s chunk_r T, min((s+1) chunk_r T, L_r)).
+ *   DECODE and SAGE_DECODE: a flat, balanced partition of the requests' units
+ *     over CTA slots.  A unit is U keys: U = T = max(64, P) for DECODE, U = 32
+ *     for SAGE_DECODE; units_r = ceil(L_r / U).  A work item covers HG = the
+ *     largest of 8, 4, 2, 1 dividing Hkv KV heads, groups = Hkv / HG, and
+ *     C = max(1, floor(num_sms * 2 / groups)) CTA slots (two slots per SM),
+ *     g_r = sum of the units of the requests before r, total = sum units_r,
+ *     per = max(1, ceil(total / C)), used = ceil(total / per).  Slot c takes the
+ *     concatenated units [c per, (c+1) per); each maximal piece of that range
+ *     within one request is an item (r, s, U u0, min(U u1, L_r)), u0/u1 relative
+ *     to g_r and s the piece's index within request r; an empty request is one
+ *     item (r, 0, 0, 0) of slot min(floor(g_r / per), max(used - 1, 0)).  Items
+ *     are listed r-major (which is also slot order, no sort) and slot_first[c],
+ *     c = 0 .. C, is the first item of slot c or later (num_items if none).  A
+ *     run CTA walks every item of its slot, so every slot streams at most per
+ *     units and the slots finish together; max_splits must be 0.
  *   EXTEND: query tiles of 128 new tokens; tile t of request r covers new
  *     tokens [128 t, min(128 t + 128, n_r)) and reads key tiles
- *     0 .. ceil((p_r + q_end) / 128) - 1, p_r = L_r - n_r.
- *   DECODE and EXTEND items are ordered by work (key count or key-tile
- *     count) descending, ties by (request, split) order, so the in-order block
- *     dispatch of the run kernels schedules the longest work first.
- *   SAGE_DECODE: a flat, balanced partition.  units_r = ceil(L_r / 32), HG and
- *     groups as for DECODE, C = max(1, floor(num_sms * 2 / groups)) CTA slots
- *     (one wave of two CTAs per SM), g_r = sum of the units of the requests
- *     before r, total = sum units_r, per = max(1, ceil(total / C)),
- *     used = ceil(total / per).  Slot c takes the concatenated units
- *     [c per, (c+1) per); each maximal piece of that range within one request
- *     is an item (r, s, 32 u0, min(32 u1, L_r)), u0/u1 relative to g_r and s
- *     the piece's index within request r; an empty request is one item
- *     (r, 0, 0, 0) of slot min(floor(g_r / per), max(used - 1, 0)).  Items are
- *     listed r-major (which is also slot order, no sort) and slot_first[c],
- *     c = 0 .. C, is the first item of slot c or later (num_items if none).
- *     max_splits must be 0 (the slots are balanced by construction).
+ *     0 .. ceil((p_r + q_end) / 128) - 1, p_r = L_r - n_r.  Items are ordered
+ *     by that key-tile count descending, ties by (request, tile) order, so the
+ *     in-order block dispatch of the run kernel schedules the longest work first.
  *   SAGE_SPARSE: the SAGE_DECODE partition over the units of each request's selected
  *     blocks (attn_plan_sage_sparse): sel_r = the selected blocks in ascending order, a
  *     selected block holds 2 units except a last block of L_r - 64 b <= 32 keys (1 unit);
  *     items are (r, s, u0, u1) in unit indices of request r, unit u being keys
  *     64 sel_r[u / 2] + 32 (u % 2) onward (at most 32, not past L_r).
- * At most ceil(num_sms * 4 / groups) + B items (DECODE), C + B (SAGE) or
- * ceil(max_q_tokens / 128) + B (EXTEND).
+ * At most C + B items (DECODE, SAGE) or ceil(max_q_tokens / 128) + B (EXTEND).
  *
  * Workspace layout (for introspection; all int32, offsets in bytes):
  *   [0, 64)   header: magic 0x4C504150, mode, batch, hq, hkv, head_dim,
  *             page_size, num_items, max_items, tile, chunk_tiles, error word,
- *             num_sms, max_splits, slots (SAGE: C, else 0), reserved
+ *             num_sms, max_splits, slots (DECODE, SAGE: C, else 0), reserved
  *   then      req_splits[B] (items of request r), req_base[B+1] (exclusive
  *             prefix sum of req_splits), req_len[B] (L_r as used), req_aux[B]
- *             (DECODE: chunk_r tiles per split; EXTEND: cu_seqlens_q[r];
- *             SAGE: g_r),
+ *             (DECODE, SAGE: g_r; EXTEND: cu_seqlens_q[r]),
  *             req_prefix[B] (EXTEND: p_r), padded to 16 B, then the items
  *             int32x4 [max_items] = {r, split, begin, end} in execution order,
- *             256-byte aligned, then (SAGE) slot_first int32 [C + 1], 256-byte
+ *             256-byte aligned, then (DECODE, SAGE) slot_first int32 [C + 1], 256-byte
  *             aligned, then (SAGE_SPARSE) sel_base int32 [B + 1] and sel_block int32
  *             [B * ceil(max_kv_len / 64)], each 256-byte aligned, then (DECODE,
  *             SAGE) fp32 partial outputs
@@ -340,7 +332,7 @@ pa_status attn_extend_paged_sage(const pa_plan_params* params, const void* d_ws,
  * loads the library holds until the process exits.  The call allocates and
  * frees nothing.  Plans whose pa_plan_workspace_size() exceeds 16 MiB are
  * rejected with PA_ERR_WORKSPACE (the Llama-3-8B decode shape, batch 64 x
- * Hq 32 on 148 SMs, needs about 11 MB).  The first call on a device looks up
+ * Hq 32 on 148 SMs, needs about 6 MB).  The first call on a device looks up
  * the array's device address (once per device, with that device current); make
  * that first call before any stream capture.  All calls share the array and it
  * keeps the last call's contents: calls that overlap on the GPU (other streams

@@ -69,9 +69,12 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
   d->page_shift = ilog2(P);
   switch (p->mode) {
     case PA_MODE_DECODE:
-      if (p->max_q_tokens != 0 || p->sage_k_block != 0) return PA_ERR_INVALID;
-      d->max_splits = p->max_splits == 0 ? 128 : p->max_splits;
-      if (d->max_splits > 4096) return PA_ERR_INVALID;
+      // the flat partition balances the slots itself: no split cap
+      if (p->max_q_tokens != 0 || p->sage_k_block != 0 || p->max_splits != 0) return PA_ERR_INVALID;
+      d->max_splits = 0;
+      // the plan counts tiles in int32
+      if ((long long)p->batch * ((p->max_kv_len + kDecodeMinTile - 1) / kDecodeMinTile) >= (1LL << 31))
+        return PA_ERR_UNSUPPORTED;
       d->tile = P > kDecodeMinTile ? P : kDecodeMinTile;
       break;
     case PA_MODE_EXTEND:
@@ -100,14 +103,9 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
   }
   d->num_sms = sms;
   long long mi = 0;
-  if (p->mode == PA_MODE_DECODE)
+  if (flat_mode(p->mode))
   {
-    const int groups = p->hkv / decode_heads_per_cta(p->hkv);
-    mi = ((long long)sms * kDecodeCtasPerSm + groups - 1) / groups + p->batch;
-  }
-  else if (sage_mode(p->mode))
-  {
-    d->slots = sage_slots(p->hkv, sms);
+    d->slots = flat_slots(p->hkv, sms);
     mi = (long long)d->slots + p->batch;
   }
   else
@@ -237,6 +235,7 @@ pa_status attn_decode_paged(const pa_plan_params* params, const void* d_ws, size
   a.hkv = params->hkv;
   a.page_shift = d.page_shift;
   a.max_items = d.max_items;
+  a.slots = d.slots;
   return from_cuda(launch_decode(a, (cudaStream_t)stream));
 }
 
@@ -276,6 +275,7 @@ pa_status attn_decode_paged_fp8(const pa_plan_params* params, const void* d_ws, 
   a.hkv = params->hkv;
   a.page_shift = d.page_shift;
   a.max_items = d.max_items;
+  a.slots = d.slots;
   return from_cuda(launch_decode_fp8(a, (cudaStream_t)stream));
 }
 

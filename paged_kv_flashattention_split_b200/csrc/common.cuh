@@ -16,12 +16,11 @@ namespace pa {
 constexpr int32_t kMagic = 0x4C504150;          // "PAPL"
 constexpr int kHeadDim = 128;
 constexpr int kDecodeMinTile = 64;               // keys per decode tile (and split granularity floor)
-constexpr int kDecodeCtasPerSm = 4;              // decode CTAs a plan aims for, per SM
 constexpr int kExtendQTile = 128;
 constexpr int kExtendKvTile = 128;
 constexpr int kSageBlock = 64;
 constexpr int kSageUnit = 32;                    // keys per unit of the Sage partition
-constexpr int kSageCtasPerSm = 2;                // Sage CTAs resident per SM (one wave of slots)
+constexpr int kFlatCtasPerSm = 2;                // CTAs per SM a flat partition's slots are sized for
 constexpr int kMaxBatch = 8192;
 constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capacity
 
@@ -29,7 +28,7 @@ constexpr int kMaxSortItems = 16384;             // single-CTA bitonic sort capa
 struct PlanHeader {
   int32_t magic, mode, batch, hq, hkv, head_dim, page_size, num_items;
   int32_t max_items, tile, chunk_tiles, error_word;
-  int32_t num_sms, max_splits, slots, reserved1;   // slots: SAGE CTA slots, else 0
+  int32_t num_sms, max_splits, slots, reserved1;   // slots: CTA slots of a flat partition, else 0
 };
 static_assert(sizeof(PlanHeader) == 64, "header is 64 bytes");
 
@@ -57,10 +56,13 @@ __host__ __device__ inline bool splitkv_mode(int mode) {
   return mode == PA_MODE_DECODE || sage_mode(mode);
 }
 
-// CTA slots of a Sage plan: max(1, floor(num_sms * 2 / groups)).
-__host__ __device__ inline int sage_slots(int hkv, int num_sms) {
+// Modes planned as a flat partition of the requests' units over CTA slots.
+__host__ __device__ inline bool flat_mode(int mode) { return splitkv_mode(mode); }
+
+// CTA slots of a flat partition: max(1, floor(num_sms * 2 / groups)).
+__host__ __device__ inline int flat_slots(int hkv, int num_sms) {
   const int groups = hkv / decode_heads_per_cta(hkv);
-  const int c = num_sms * kSageCtasPerSm / groups;
+  const int c = num_sms * kFlatCtasPerSm / groups;
   return c > 1 ? c : 1;
 }
 
@@ -76,7 +78,7 @@ inline WsLayout ws_layout(int mode, int batch, int hq, int hkv, int head_dim, in
   off = align_up(off, 16);
   w.items = off;      off += 16 * (size_t)max_items;
   off = align_up(off, 256);
-  if (sage_mode(mode)) {
+  if (flat_mode(mode)) {
     w.slot_first = off; off += 4 * (size_t)(slots + 1);
     off = align_up(off, 256);
   }
@@ -113,7 +115,7 @@ struct WsView {
   int32_t* req_aux;
   int32_t* req_prefix;
   int4* items;
-  int32_t* slot_first;  // SAGE: [slots + 1] first item of each CTA slot
+  int32_t* slot_first;  // DECODE, SAGE: [slots + 1] first item of each CTA slot
   int32_t* sel_base;    // SAGE_SPARSE: [B + 1] first selected block of each request in sel_block
   int32_t* sel_block;   // SAGE_SPARSE: the selected 64-key blocks, request by request
   float* partial_o;

@@ -11,7 +11,7 @@ struct PlanLaunch {
   const int32_t* cu_seqlens_q;
   int mode, batch, hq, hkv, head_dim, page_size, max_kv_len, num_sms, max_splits, max_items, tile;
   int sort_n;  // power of two >= max_items
-  int slots;   // SAGE: CTA slots
+  int slots;   // DECODE, SAGE: CTA slots of the flat partition
   const uint8_t* block_mask;   // SAGE_SPARSE: [B][mask_pitch], nonzero = the 64-key block is attended
   int64_t mask_pitch;
 };
@@ -29,6 +29,7 @@ struct DecodeLaunch {
   uint16_t* out;
   float* lse_out;
   int batch, hq, hkv, page_shift, max_items;
+  int slots;          // CTA slots of the plan's flat partition
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeLaunch& a, cudaStream_t s);   // the split merge alone
@@ -46,6 +47,7 @@ struct Fp8DecodeLaunch {
   uint16_t* out;
   float* lse_out;
   int batch, hq, hkv, page_shift, max_items;
+  int slots;               // CTA slots of the plan's flat partition
 };
 cudaError_t launch_decode_fp8(const Fp8DecodeLaunch& a, cudaStream_t s);
 

@@ -15,24 +15,6 @@ constexpr int kPlanThreads = 1024;
 
 __device__ __forceinline__ long long cdiv_ll(long long a, long long b) { return (a + b - 1) / b; }
 
-// Block-wide sum of one int64 per thread.
-__device__ long long block_sum(long long v, long long* red) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  long long t = 0;
-  if (threadIdx.x < 32) {
-    t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) red[0] = t;
-  }
-  __syncthreads();
-  t = red[0];
-  __syncthreads();
-  return t;
-}
-
 // Block-wide exclusive scan of one int per thread; returns this thread's prefix.
 __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
   const int tid = threadIdx.x;
@@ -50,27 +32,23 @@ __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
   return incl - v;
 }
 
-// Work of item (r, s) for the sort key; items run longest first.
-__device__ __forceinline__ int item_work(int mode, int s, int L, int chunk_r, int tile, int prefix, int n) {
-  if (mode == PA_MODE_DECODE) {
-    if (chunk_r == 0) return 0;
-    const long long a = (long long)s * chunk_r * tile;
-    const long long b = min((long long)(s + 1) * chunk_r * tile, (long long)L);
-    return (int)(b - a);
-  }
+// EXTEND: work of query tile s (key tiles it needs) for the sort key; items run longest first.
+__device__ __forceinline__ int item_work(int s, int prefix, int n) {
   const int q1 = min((s + 1) * kExtendQTile, n);
   return (int)cdiv_ll(prefix + q1, kExtendKvTile);
 }
 
-// SAGE_DECODE / SAGE_SPARSE: the flat partition of the requests' 32-key units (of the
-// selected 64-key blocks only, for SAGE_SPARSE) over CTA slots (the algorithm at attn_plan).
-// Items come out r-major, which is also slot order, so no sort.
-__device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* chunk_out, int* n_out) {
+// DECODE, SAGE_DECODE, SAGE_SPARSE: the flat partition of the requests' units (T-key tiles
+// for DECODE, 32-key units for Sage, of the selected 64-key blocks only for SAGE_SPARSE)
+// over CTA slots (the algorithm at attn_plan).  Items come out r-major, which is also slot
+// order, so no sort.
+__device__ void flat_plan(const PlanLaunch& a, int* item_slot, int* scan, int* chunk_out, int* n_out) {
   const int tid = threadIdx.x, nt = blockDim.x;
   WsView ws = a.ws;
   PlanHeader* hdr = ws.hdr;
   const int B = a.batch;
   const bool sparse = a.mode == PA_MODE_SAGE_SPARSE;
+  const int U = a.mode == PA_MODE_DECODE ? a.tile : kSageUnit;   // keys per unit
   // 1. lengths (clamped and flagged when out of range); the units of each request
   //    (req_prefix holds them during the plan), and its selected block count (SAGE_SPARSE)
   for (int r = tid; r < B; r += nt) {
@@ -80,7 +58,7 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
       L = max(0, min(L, a.max_kv_len));
     }
     ws.req_len[r] = L;
-    int units = (int)cdiv_ll(L, kSageUnit), nsel = 0;
+    int units = (int)cdiv_ll(L, U), nsel = 0;
     if (sparse) {
       const int nb = (int)cdiv_ll(L, kSageBlock);
       const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
@@ -165,7 +143,7 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
       if (i >= n_items) break;
       const int u0 = max(g, c * per) - g, u1 = min(g + u, (c + 1) * per) - g;
       ws.items[i] = sparse ? make_int4(r, c - c_first, u0, u1)
-                           : make_int4(r, c - c_first, u0 * kSageUnit, min(u1 * kSageUnit, L));
+                           : make_int4(r, c - c_first, u0 * U, (int)min((long long)u1 * U, (long long)L));
       item_slot[i] = c;
     }
   }
@@ -184,7 +162,6 @@ __device__ void sage_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
   extern __shared__ unsigned long long keys[];
-  __shared__ long long red[32];
   __shared__ int scan[kPlanThreads];
   const int tid = threadIdx.x, nt = blockDim.x;
   WsView ws = a.ws;
@@ -193,12 +170,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
   if (tid == 0) hdr->error_word = 0;  // every new plan starts with a clean error word
   __syncthreads();
   int chunk = 0, n_items = 0;
-  if (sage_mode(a.mode)) {
-    sage_plan(a, reinterpret_cast<int*>(keys), scan, &chunk, &n_items);
+  if (flat_mode(a.mode)) {
+    flat_plan(a, reinterpret_cast<int*>(keys), scan, &chunk, &n_items);
   } else {
 
-  // 1. lengths (clamped and flagged when out of range), tiles per request
-  long long my_tiles = 0;
+  // 1. lengths (clamped and flagged when out of range), query tiles per request
   for (int r = tid; r < B; r += nt) {
     int L = a.seq_lens[r];
     if (L < 0 || L > a.max_kv_len) {
@@ -206,51 +182,19 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
       L = max(0, min(L, a.max_kv_len));
     }
     ws.req_len[r] = L;
-    if (a.mode == PA_MODE_DECODE) my_tiles += cdiv_ll(L, a.tile);
-  }
-  const long long total = block_sum(my_tiles, red) * (a.hkv / decode_heads_per_cta(a.hkv));
-  if (a.mode == PA_MODE_DECODE) {
-    const long long slots = (long long)a.num_sms * kDecodeCtasPerSm;
-    chunk = (int)max(1LL, cdiv_ll(total, slots));
-  }
-
-  // 2. splits (DECODE, SAGE) or query tiles (EXTEND) per request
-  for (int r = tid; r < B; r += nt) {
-    const int L = ws.req_len[r];
-    int splits = 1, aux = 0, prefix = 0;
-    if (a.mode == PA_MODE_DECODE) {
-      const int tiles = (int)cdiv_ll(L, a.tile);
-      if (tiles == 0) {
-        splits = 1;
-        aux = 0;
-      } else {
-        int chunk_r = chunk;
-        int s = (int)cdiv_ll(tiles, chunk_r);
-        if (s > a.max_splits) {
-          chunk_r = (int)cdiv_ll(tiles, a.max_splits);
-          s = (int)cdiv_ll(tiles, chunk_r);
-        }
-        splits = s;
-        aux = chunk_r;
-      }
-    } else if (a.mode == PA_MODE_EXTEND) {
-      const int q0 = a.cu_seqlens_q[r], q1 = a.cu_seqlens_q[r + 1];
-      int n = q1 - q0;
-      if (n < 0 || n > L) {
-        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-        n = max(0, min(n, L));
-      }
-      splits = (int)cdiv_ll(n, kExtendQTile);
-      aux = q0;
-      prefix = L - n;
+    const int q0 = a.cu_seqlens_q[r], q1 = a.cu_seqlens_q[r + 1];
+    int n = q1 - q0;
+    if (n < 0 || n > L) {
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      n = max(0, min(n, L));
     }
-    ws.req_splits[r] = splits;
-    ws.req_aux[r] = aux;
-    ws.req_prefix[r] = prefix;
+    ws.req_splits[r] = (int)cdiv_ll(n, kExtendQTile);
+    ws.req_aux[r] = q0;
+    ws.req_prefix[r] = L - n;
   }
   __syncthreads();
 
-  // 3. req_base = exclusive prefix sum of the per-request item counts
+  // 2. req_base = exclusive prefix sum of the per-request item counts
   const int per = (B + nt - 1) / nt;
   const int r0 = min(B, tid * per), r1 = min(B, r0 + per);
   int local = 0;
@@ -270,21 +214,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
   for (int i = tid; i < a.sort_n; i += nt) keys[i] = ~0ull;
   __syncthreads();
 
-  // 4. sort keys: (0x7FFFFFFF - work) in the high word, generation index in the low word
+  // 3. sort keys: (0x7FFFFFFF - work) in the high word, generation index in the low word
   for (int r = tid; r < B; r += nt) {
     const int base = ws.req_base[r], splits = ws.req_splits[r];
-    const int L = ws.req_len[r], aux = ws.req_aux[r], prefix = ws.req_prefix[r];
+    const int L = ws.req_len[r], prefix = ws.req_prefix[r];
     const int n = L - prefix;
     for (int s = 0; s < splits; ++s) {
       const int g = base + s;
       if (g >= n_items) break;
-      const unsigned work = (unsigned)item_work(a.mode, s, L, aux, a.tile, prefix, n);
+      const unsigned work = (unsigned)item_work(s, prefix, n);
       keys[g] = ((unsigned long long)(0x7FFFFFFFu - work) << 32) | (unsigned)g;
     }
   }
   __syncthreads();
 
-  // 5. bitonic sort, ascending (unique keys, so the order is fully determined)
+  // 4. bitonic sort, ascending (unique keys, so the order is fully determined)
   for (int k = 2; k <= a.sort_n; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int i = tid; i < a.sort_n; i += nt) {
@@ -302,7 +246,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     }
   }
 
-  // 6. items in execution order
+  // 5. items in execution order
   for (int i = tid; i < n_items; i += nt) {
     const int g = (int)(keys[i] & 0xFFFFFFFFu);
     int lo = 0, hi = B;  // find r with req_base[r] <= g < req_base[r+1]
@@ -311,24 +255,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
       if (ws.req_base[mid] <= g) lo = mid; else hi = mid;
     }
     const int r = lo, s = g - ws.req_base[r];
-    const int L = ws.req_len[r], aux = ws.req_aux[r], prefix = ws.req_prefix[r];
-    int4 it;
-    it.x = r;
-    it.y = s;
-    if (a.mode == PA_MODE_DECODE) {
-      const long long b0 = (long long)s * aux * a.tile;
-      it.z = (int)min(b0, (long long)L);
-      it.w = (int)min((long long)(s + 1) * aux * a.tile, (long long)L);
-    } else {
-      const int n = L - prefix;
-      it.z = s * kExtendQTile;
-      it.w = min((s + 1) * kExtendQTile, n);
-    }
-    ws.items[i] = it;
+    const int L = ws.req_len[r], prefix = ws.req_prefix[r];
+    const int n = L - prefix;
+    ws.items[i] = make_int4(r, s, s * kExtendQTile, min((s + 1) * kExtendQTile, n));
   }
-  }  // DECODE, EXTEND
+  }  // EXTEND
 
-  // 7. header
+  // 6. header
   if (tid == 0) {
     hdr->magic = kMagic;
     hdr->mode = a.mode;
@@ -343,7 +276,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
     hdr->chunk_tiles = chunk;
     hdr->num_sms = a.num_sms;
     hdr->max_splits = a.max_splits;
-    hdr->slots = sage_mode(a.mode) ? a.slots : 0;
+    hdr->slots = flat_mode(a.mode) ? a.slots : 0;
     hdr->reserved1 = 0;
   }
 }

@@ -60,7 +60,7 @@ def ws_offsets(mode: int, batch: int, hq: int, max_items: int, head_dim: int = 1
     o["items"] = off
     off += 16 * max_items
     off = (off + 255) // 256 * 256
-    if mode in (2, 3):
+    if mode in (0, 2, 3):
         o["slot_first"] = off
         off += 4 * (slots + 1)
         off = (off + 255) // 256 * 256
@@ -106,7 +106,7 @@ def read_plan(ws: torch.Tensor, mode: int, batch: int, hq: int, max_kv_len: int 
             "error_word": int(hdr[11]), "num_items": num_items, "max_items": max_items,
             "req_splits": arr("req_splits", batch), "req_base": arr("req_base", batch + 1),
             "req_len": arr("req_len", batch), "slots": slots, "num_sms": int(hdr[12]),
-            "slot_first": arr("slot_first", slots + 1) if mode in (2, 3) else None,
+            "slot_first": arr("slot_first", slots + 1) if mode in (0, 2, 3) else None,
             "sel_base": arr("sel_base", batch + 1) if mode == 3 else None,
             "items": [tuple(int(x) for x in it) for it in items]}
 

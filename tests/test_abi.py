@@ -62,6 +62,7 @@ def P(**kw):
     (dict(mode=7), pa.PA_ERR_INVALID),
     (dict(max_q_tokens=5), pa.PA_ERR_INVALID),          # decode plan given an extend-only input
     (dict(sage_k_block=64), pa.PA_ERR_INVALID),
+    (dict(max_splits=4), pa.PA_ERR_INVALID),             # no split cap in DECODE (flat partition)
     (dict(mode=1, page_size=4, max_q_tokens=100), pa.PA_ERR_UNSUPPORTED),
     (dict(mode=2, page_size=64, sage_k_block=16), pa.PA_ERR_UNSUPPORTED),
     (dict(mode=2, page_size=64, sage_k_block=64, max_q_tokens=8), pa.PA_ERR_INVALID),
@@ -79,10 +80,8 @@ def test_workspace_size_matches_documented_layout(lib):
         p = P(mode=mode, batch=33, hq=32, hkv=8, **extra)
         n = pa.pa_plan_workspace_size(p)
         slots = 0
-        if mode == 0:
-            mi = 148 * 4 + 33          # Hkv 8: one plan unit per item
-        elif mode == 2:
-            slots = 148 * 2            # Hkv 8: one CTA per slot
+        if mode in (0, 2):
+            slots = 148 * 2            # Hkv 8: one item covers the 8 KV heads, two slots per SM
             mi = slots + 33
         else:
             mi = -(-9000 // 128) + 33

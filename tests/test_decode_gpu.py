@@ -36,14 +36,13 @@ def num_sms():
     return torch.cuda.get_device_properties(0).multi_processor_count
 
 
-def decode_params(spec, batch, max_splits=0):
+def decode_params(spec, batch, plan_sms=0):
     return pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, spec.head_dim, spec.page_size,
-                          max_kv_len=batch.page_table.shape[1] * spec.page_size, num_sms=0,
-                          max_splits=max_splits)
+                          max_kv_len=batch.page_table.shape[1] * spec.page_size, num_sms=plan_sms)
 
 
-def run_decode(spec, batch, q, k, v, max_splits=0, ws=None, plan=True):
-    params = decode_params(spec, batch, max_splits)
+def run_decode(spec, batch, q, k, v, plan_sms=0, ws=None, plan=True):
+    params = decode_params(spec, batch, plan_sms)
     if ws is None:
         ws = alloc_ws(params)
     if plan:
@@ -77,11 +76,11 @@ def device_case(spec, seed_shift=0, layer=0):
 
 # ---------------------------------------------------------------- plan
 
-def _gpu_plan(mode, lens, cu=None, hq=8, hkv=2, page_size=1, max_splits=0, max_kv_len=None, max_q=0):
+def _gpu_plan(mode, lens, cu=None, hq=8, hkv=2, page_size=1, max_kv_len=None, max_q=0, plan_sms=0):
     B = len(lens)
     max_kv_len = max(lens + [1]) if max_kv_len is None else max_kv_len
     params = pa.make_params(mode, B, hq, hkv, 128, page_size, max_kv_len=max_kv_len, max_q_tokens=max_q,
-                            num_sms=0, max_splits=max_splits, sage_k_block=64 if mode == 2 else 0)
+                            num_sms=plan_sms, sage_k_block=64 if mode == 2 else 0)
     ws = alloc_ws(params)
     sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
     cut = None if cu is None else torch.tensor(cu, dtype=torch.int32, device=DEV)
@@ -90,10 +89,8 @@ def _gpu_plan(mode, lens, cu=None, hq=8, hkv=2, page_size=1, max_splits=0, max_k
     return read_plan(ws, mode, B, hq), ws
 
 
-def _oracle_plan(mode, lens, cu=None, hkv=2, page_size=1, max_splits=0, max_q=0):
-    ms = (128 if max_splits == 0 else max_splits) if mode == 0 else 1
-    return op.plan(mode, lens, cu, hkv=hkv, page_size=page_size, num_sms=num_sms(), max_splits=ms,
-                   max_q_tokens=max_q)
+def _oracle_plan(mode, lens, cu=None, hkv=2, page_size=1, max_q=0, plan_sms=0):
+    return op.plan(mode, lens, cu, hkv=hkv, page_size=page_size, num_sms=plan_sms or num_sms(), max_q_tokens=max_q)
 
 
 def _assert_same_plan(g, o):
@@ -109,16 +106,18 @@ def _assert_same_plan(g, o):
 
 def test_decode_plan_bit_exact():
     rng = np.random.default_rng(100)
-    cases = [([300, 17, 0, 129, 64], 2, 1, 3), ([131072] * 8, 8, 64, 0), ([1], 1, 1, 0), ([0, 0], 4, 16, 0)]
+    # (lengths, Hkv, page size, plan SMs: 0 = the device's count)
+    cases = [([300, 17, 0, 129, 64], 2, 1, 1), ([131072] * 8, 8, 64, 0), ([1], 1, 1, 0), ([0, 0], 4, 16, 0),
+             ([200, 0, 300], 8, 1, 2)]
     for _ in range(25):
         B = int(rng.integers(1, 80))
         lens = [int(x) for x in rng.integers(0, 9000, B)]
         cases.append((lens, int(rng.choice([1, 2, 4, 8])), int(rng.choice([1, 2, 16, 64, 128, 256])),
                       int(rng.choice([0, 1, 3, 17]))))
-    cases.append(([int(x) for x in rng.integers(1, 300, 4096)], 8, 1, 0))   # large batch: sort stress
-    for lens, hkv, P, ms in cases:
-        g, _ = _gpu_plan(0, lens, hq=hkv * 2, hkv=hkv, page_size=P, max_splits=ms)
-        _assert_same_plan(g, _oracle_plan(0, lens, hkv=hkv, page_size=P, max_splits=ms))
+    cases.append(([int(x) for x in rng.integers(1, 300, 4096)], 8, 1, 0))   # large batch
+    for lens, hkv, P, sms in cases:
+        g, _ = _gpu_plan(0, lens, hq=hkv * 2, hkv=hkv, page_size=P, plan_sms=sms)
+        _assert_same_plan(g, _oracle_plan(0, lens, hkv=hkv, page_size=P, plan_sms=sms))
 
 
 def test_extend_and_sage_plans_bit_exact():
@@ -218,13 +217,14 @@ def test_decode_tiny_config():
     check_lse(lse, ref_lse)
 
 
-@pytest.mark.parametrize("max_splits", [0, 1, 2])
-def test_decode_llama3_8b_shape_scaled(max_splits):
+@pytest.mark.parametrize("plan_sms", [0, 1, 7])
+def test_decode_llama3_8b_shape_scaled(plan_sms):
+    # plan_sms = 1 gives two slots, so each CTA walks many items of several requests
     spec = wl.CONFIGS[2].scaled(batch=12, pool_slots=120_000)
     batch, q, k, v = device_case(spec)
-    out, lse, _, _ = run_decode(spec, batch, q, k, v, max_splits=max_splits)
+    out, lse, _, _ = run_decode(spec, batch, q, k, v, plan_sms=plan_sms)
     ref, ref_lse = oracle_decode(spec, batch, q, k, v)
-    assert_bf16_close(out, ref, f"decode_8b max_splits={max_splits}")
+    assert_bf16_close(out, ref, f"decode_8b plan_sms={plan_sms}")
     check_lse(lse, ref_lse)
 
 
