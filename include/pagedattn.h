@@ -303,8 +303,8 @@ pa_status attn_decode_paged_sage(const pa_plan_params* params, const void* d_ws,
  *   O[d] = sfV[h_kv][d] (sum_j E4M3(448 exp(S_j - m)) V8_j[d]) / (448 l) + v_mean[h_kv][d].
  * The dense Sage variant the pages measure at S = 10800 ("FlashInfer PrimTS, Sage
  * Attention ...", performance item 2).  Two passes over the key tiles of each query tile
- * (the row max first, then P8 and O) on the tcgen05 tensor cores; the 8-bit operands are
- * converted to f16 on chip, which holds them exactly.
+ * (the row max first, then P8 and O) on the tcgen05 tensor cores in their 8-bit kinds:
+ * Q8 . K8 on int8 (exact int32 dots), P8 . V8 on E4M3 with fp32 accumulation.
  *
  * params, d_ws    an EXTEND plan (attn_plan, mode PA_MODE_EXTEND) with page_size 64.
  * d_q8 int8 [max_q_tokens][Hq][D] (rows cu_seqlens_q[r] .. of request r), d_sf_q fp32

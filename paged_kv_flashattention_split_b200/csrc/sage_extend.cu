@@ -1,5 +1,5 @@
 // sage_extend.cu - 8-bit "Sage" EXTEND (prefill over a cached prefix) on the 5th-generation
-// tensor cores.
+// tensor cores, in their native 8-bit kinds.
 //
 // The formula ("FlashInfer PrimTS, Sage Attention 도입으로 8비트 양자화 및 성능 최적화
 // 달성", 코드 분석 item 1, README "Sage attention") for every new token: row i of request r
@@ -11,72 +11,64 @@
 //
 // P8 needs the exact row max before any probability is formed, so a CTA (one query tile
 // of 128 new tokens, one head) makes two passes over its key tiles: pass 1 computes
-// S = Q K^T and each row's maximum, pass 2 computes S again, P8 and O += P8 V.  The 8-bit
-// operands enter the tensor cores as f16, which holds every int8 and every E4M3 value
-// exactly; the int8 dot (|dot| < 2^21) and the P8 V8 products accumulate exactly in fp32,
-// so kind::f16 MMAs reproduce the integer and FP8 contractions.  Roles (10 warps):
-//   warp 0      producer: TMA boxes of 64 slots (one page) x 128 bytes into a 3-stage
-//               ring of 8-bit staging tiles, in the order the converters consume them:
-//               Q8, pass 1: K8(0..n-1), pass 2: K8(0), V8(0), K8(1), V8(1), ...;
-//   warps 6-9   converters: 8-bit staging tile -> f16 operand tile in the MMA's 128-byte
-//               swizzled K-major layout (Q, K) or the same rows read MN-major (V); V rows
-//               past the request's last key are written as zero;
-//   warp 1      MMA issuer: S(g) = Q K16(g)^T into TMEM buffer g % 3 (g = 0 .. 2n-1 over
-//               both passes, the K16 use of S(g) is g), and in pass 2 O += P V(j) with
-//               P (f16) read from TMEM;
+// S = Q K^T and each row's maximum, pass 2 computes S again, P8 and O += P8 V.  Both
+// contractions run on the 8-bit tensor cores: S on tcgen05.mma kind::i8 (int8 x int8 into
+// int32, exact), P8 V on kind::f8f6f4 (E4M3 x E4M3 into fp32), with P8 taken from TMEM
+// (four E4M3 codes per 32-bit column) and V8 read in place as an MN-major operand.  The
+// 8-bit tiles land from TMA in the operands' 128-byte-swizzled layouts, so nothing is
+// converted on chip.  Roles (6 warps):
+//   warp 0      producer: Q8 once, then TMA boxes of 64 slots (one page) x 128 bytes into an
+//               8-stage ring of 16 KB tiles, in the order K8(0..n-1) (pass 1), then K8(0),
+//               V8(0), K8(1), V8(1), ... (pass 2);
+//   warp 1      MMA issuer: S(g) = Q K(g)^T into TMEM buffer g % 3 (g = 0 .. 2n-1 over both
+//               passes), and in pass 2 O += P8 V(j) with P8 from TMEM; a stage is released
+//               when the MMA that read it completes;
 //   warps 2-5   softmax: thread i owns query row i (TMEM lane i); pass 1 reduces the row
-//               maximum of the causally masked scores, pass 2 writes P8 (as f16) over the
-//               scores in TMEM and sums l; at the end it applies the epilogue.
-// Every wait on an mbarrier is bounded and every barrier phase is waited once, in order:
-// on timeout the CTA records PA_ERR_DEVICE_INDEX, its roles stop, the producer waits for
-// its copies, the MMA issuer drains the tensor cores, and TMEM is freed before exit.
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
-
+//               maximum of the causally masked scores, pass 2 writes P8 over the scores in
+//               TMEM and sums l; at the end it applies the epilogue.  V8 rows past the
+//               request's last key inside the last 32-key step are zeroed before PV reads
+//               them (0 x NaN would poison O).
+// Every wait on an mbarrier is bounded: on timeout the CTA records PA_ERR_DEVICE_INDEX,
+// its roles stop, the producer waits for its copies, the MMA issuer drains the tensor
+// cores, and TMEM is freed before exit.
 #include "kernels.h"
 #include "tma.cuh"
 
 namespace pa {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 192;
 constexpr int kTileRows = 128;                     // query rows and keys per tile
-constexpr int kHalf = 128 * 128;                   // one 64-d half of a 128 x 128 f16 tile (16 KB)
-constexpr int kF16Tile = 2 * kHalf;                // 32 KB
-constexpr int kStgTile = 128 * 128;                // 128 rows x 128 bytes of 8-bit data (16 KB)
-constexpr int kStg = 3;                            // staging stages
-constexpr uint32_t kTmemCols = 512;                // S0, S1, S2, O
+constexpr int kTile8 = 128 * 128;                  // 128 rows x 128 bytes of 8-bit data (16 KB)
+constexpr int kStg = 8;                            // ring stages
+constexpr uint32_t kTmemCols = 512;                // S0, S1, S2 (int32), O (fp32)
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kF16Tile;            // [2]
-constexpr int kOffV = kOffK + 2 * kF16Tile;        // [2]
-constexpr int kOffStg = kOffV + 2 * kF16Tile;      // [kStg]
-constexpr int kOffBar = kOffStg + kStg * kStgTile;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;
+constexpr int kOffStg = kOffQ + kTile8;            // [kStg]
+constexpr int kOffBar = kOffStg + kStg * kTile8;
+constexpr int kSmemBytes = kOffBar + 512 + 1024;
 
 enum Bar {
-  B_STG_FULL = 0,                  // [3] staging tile landed (TMA)
-  B_STG_EMPTY = B_STG_FULL + kStg, // [3] converters done with it (128)
-  B_Q16 = B_STG_EMPTY + kStg,      // f16 Q tile written (128)
-  B_K16_FULL,                      // [2] (128)
-  B_K16_EMPTY = B_K16_FULL + 2,    // [2] S MMA done with it (commit)
-  B_V16_FULL = B_K16_EMPTY + 2,    // [2] (128)
-  B_V16_EMPTY = B_V16_FULL + 2,    // [2] PV MMA done with it (commit)
-  B_S_FULL = B_V16_EMPTY + 2,      // [3] S(g) in TMEM (commit)
+  B_STG_FULL = 0,                  // [kStg] tile landed (TMA)
+  B_STG_EMPTY = B_STG_FULL + kStg, // [kStg] the MMA that read it has completed (commit)
+  B_Q = B_STG_EMPTY + kStg,        // Q8 landed
+  B_S_FULL,                        // [3] S(g) in TMEM (commit)
   B_S_READ = B_S_FULL + 3,         // [3] pass 1: softmax has read S(g) (128)
-  B_P_FULL = B_S_READ + 3,         // [3] pass 2: P(g) written over S(g) (128)
+  B_P_FULL = B_S_READ + 3,         // [3] pass 2: P8(g) written over S(g) (128)
   B_PV_DONE = B_P_FULL + 3,        // [3] pass 2: PV(g) done (commit)
   B_O_DONE = B_PV_DONE + 3,        // every PV done (commit)
   B_DRAIN,
   B_COUNT
 };
-static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
+static_assert(B_COUNT * 8 + 16 <= 512, "barrier area");
 
-// instruction descriptor, kind::f16: f16 A and B, fp32 D, M = 128, N = 128
-constexpr uint32_t kIdescS = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);   // A, B K-major
-constexpr uint32_t kIdescPV = kIdescS | (1u << 16);                                  // B (V) MN-major
+// instruction descriptors, M = 128, N = 128
+//   S:  kind::i8, s32 D, s8 A and B, both K-major
+//   PV: kind::f8f6f4, f32 D, E4M3 A (from TMEM, K-major) and B (V8, MN-major)
+constexpr uint32_t kIdescS = (2u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 struct SageExtendLaunch {
   CUtensorMap tm_q8;    // q8 [rows][Hq][128] bytes as {128, rows, Hq}, box {128, 128, 1}
@@ -98,24 +90,24 @@ struct SageExtendLaunch {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 
-// smem matrix descriptor: 128-byte swizzle, 8-row groups 1024 bytes apart, LBO as given
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes) {
-  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)(lbo_bytes >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         (1ull << 46) | (2ull << 61);
+// smem matrix descriptor: 128-byte swizzle, 8-row groups 1024 bytes apart (SBO); the
+// operands here are 128 bytes wide, one swizzle atom, so the LBO is never used
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
 }
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// D (TMEM, s32) += A (smem, s8) x B (smem, s8)
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdescS), "r"(accumulate)
       : "memory");
 }
-// D (TMEM) += A (TMEM, K-major f16 pairs) x B (shared memory descriptor)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// D (TMEM, f32) += A (TMEM, E4M3, four per column) x B (smem, E4M3)
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(kIdescPV), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -131,46 +123,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
 }
-// stores v[0..15]
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
-      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n"
+               ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-// Four int8 (one word) to two f16 pairs, exactly: s + 128 as the low mantissa bits of 1024,
-// then 1152 subtracted.
-__device__ __forceinline__ void s8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t u = w ^ 0x80808080u;
-  const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480), __ushort_as_half((unsigned short)0x6480));
-  uint32_t a = prmt(u, 0x64646464u, 0x5140), b = prmt(u, 0x64646464u, 0x7362);
-  const __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
-  const __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
-  lo = *reinterpret_cast<const uint32_t*>(&ha);
-  hi = *reinterpret_cast<const uint32_t*>(&hb);
-}
-// Four E4M3 codes (one word) to two f16 pairs, exactly.
-__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  lo = (uint32_t)a.x | ((uint32_t)a.y << 16);
-  hi = (uint32_t)b.x | ((uint32_t)b.y << 16);
-}
-// Two floats to E4M3 (nearest even, saturating) and back to an f16 pair: the P8 values as the MMA sees them.
-__device__ __forceinline__ uint32_t p8_pair_f16(float lo, float hi) {
+// Two floats to E4M3 codes (nearest even, saturating); `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t v;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(v) : "f"(hi), "f"(lo));
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+  return v;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_constant__ SageExtendLaunch a) {
@@ -201,9 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
-      const bool many = (i >= B_STG_EMPTY && i < B_STG_EMPTY + kStg) || i == B_Q16 ||
-                        (i >= B_K16_FULL && i < B_K16_FULL + 2) || (i >= B_V16_FULL && i < B_V16_FULL + 2) ||
-                        (i >= B_S_READ && i < B_S_READ + 3) || (i >= B_P_FULL && i < B_P_FULL + 3);
+      const bool many = (i >= B_S_READ && i < B_S_READ + 3) || (i >= B_P_FULL && i < B_P_FULL + 3);
       mbar_init(bar(i), many ? 128 : 1);
     }
     *abort_flag = 0;
@@ -241,148 +204,88 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
     }
     return e;
   };
-  // staged tile t: 0 = Q8; 1 .. n = K8(t - 1); then K8(j), V8(j) at n + 1 + 2j, n + 2 + 2j
-  const int n_stg = 1 + 3 * n;
+  // ring items: t < n is K8(t) of pass 1; then K8(j) at n + 2j and V8(j) at n + 2j + 1
+  const int n_items = 3 * n;
+  auto stage_of = [](int t) { return t % kStg; };
+  auto full_parity = [](int t) { return (uint32_t)(t / kStg) & 1u; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
+    if (lane == 0) {
+      mbar_expect_tx(bar(B_Q), kTile8);
+      tma_load_3d(base + kOffQ, &a.tm_q8, 0, q_start + q_begin, h, bar(B_Q));
+    }
     int issued = 0;
     int pg_lo = -1, pg_hi = -1;   // this lane's pages for the tile j = tb + lane of the current round
     int round_tb = -1;
-    for (int t = 0; t < n_stg; ++t) {
-      const int s = t % kStg;
-      int j = -1;
-      bool is_v = false;
-      if (t >= 1 && t <= n) j = t - 1;
-      else if (t > n) { j = (t - n - 1) >> 1; is_v = ((t - n - 1) & 1) != 0; }
-      if (j >= 0 && (j >> 5) << 5 != round_tb) {              // page ids of 32 tiles, one per lane
+    for (int t = 0; t < n_items; ++t) {
+      const int s = stage_of(t);
+      const int j = t < n ? t : (t - n) >> 1;
+      const bool is_v = t >= n && ((t - n) & 1);
+      if ((j >> 5) << 5 != round_tb) {                         // page ids of 32 tiles, one per lane
         round_tb = (j >> 5) << 5;
         const int jj = round_tb + lane;
         pg_lo = jj < n ? page_of(2 * jj) : -1;
         pg_hi = jj < n ? page_of(2 * jj + 1) : -1;
       }
-      const int plo = j >= 0 ? __shfl_sync(0xffffffffu, pg_lo, j & 31) : -1;
-      const int phi = j >= 0 ? __shfl_sync(0xffffffffu, pg_hi, j & 31) : -1;
+      const int plo = __shfl_sync(0xffffffffu, pg_lo, j & 31);
+      const int phi = __shfl_sync(0xffffffffu, pg_hi, j & 31);
       bool ok = true;
       if (lane == 0) {
         ok = t < kStg || wait(bar(B_STG_EMPTY + s), (uint32_t)((t / kStg) - 1) & 1u);
         if (ok) {
-          const uint32_t dst = base + kOffStg + s * kStgTile;
-          if (t == 0) {
-            mbar_expect_tx(bar(B_STG_FULL + s), kStgTile);
-            tma_load_3d(dst, &a.tm_q8, 0, q_start + q_begin, h, bar(B_STG_FULL + s));
-          } else {
-            const uint32_t bytes = (plo >= 0 ? kStgTile / 2 : 0) + (phi >= 0 ? kStgTile / 2 : 0);
-            mbar_expect_tx(bar(B_STG_FULL + s), bytes);
-            const CUtensorMap* tm = is_v ? &a.tm_v8 : &a.tm_k8;
-            if (plo >= 0) tma_load_3d(dst, tm, 0, plo * kSageBlock, h_kv, bar(B_STG_FULL + s));
-            if (phi >= 0) tma_load_3d(dst + kStgTile / 2, tm, 0, phi * kSageBlock, h_kv, bar(B_STG_FULL + s));
-          }
+          const uint32_t dst = base + kOffStg + s * kTile8;
+          const uint32_t bytes = (plo >= 0 ? kTile8 / 2 : 0) + (phi >= 0 ? kTile8 / 2 : 0);
+          mbar_expect_tx(bar(B_STG_FULL + s), bytes);
+          const CUtensorMap* tm = is_v ? &a.tm_v8 : &a.tm_k8;
+          if (plo >= 0) tma_load_3d(dst, tm, 0, plo * kSageBlock, h_kv, bar(B_STG_FULL + s));
+          if (phi >= 0) tma_load_3d(dst + kTile8 / 2, tm, 0, phi * kSageBlock, h_kv, bar(B_STG_FULL + s));
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       issued = t + 1;
     }
     if (lane == 0 && *abort_flag) {   // copies still in flight: wait (bounded) until they land
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_Q), 0); ++i) {}
       for (int t = max(0, issued - kStg); t < issued; ++t)
-        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_STG_FULL + t % kStg), (uint32_t)(t / kStg) & 1u); ++i) {}
-    }
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------ converters (warps 6-9)
-    const int ct = tid - 192;                                  // 0 .. 127
-    const int c = ct & 7, r_in = ct >> 3;                      // 16-byte chunk of a row, row within a pass
-    bool ok = true;
-    for (int t = 0; t < n_stg && ok; ++t) {
-      const int s = t % kStg;
-      int j = -1, uk = -1;
-      bool is_v = false;
-      if (t >= 1 && t <= n) { j = t - 1; uk = j; }
-      else if (t > n) { j = (t - n - 1) >> 1; is_v = ((t - n - 1) & 1) != 0; uk = is_v ? -1 : n + j; }
-      if (!(ok = wwait(bar(B_STG_FULL + s), (uint32_t)(t / kStg) & 1u))) break;
-      uint32_t dst_off;
-      if (t == 0) {
-        dst_off = kOffQ;
-      } else if (!is_v) {
-        if (uk >= 2 && !(ok = wwait(bar(B_K16_EMPTY + (uk & 1)), (uint32_t)((uk >> 1) - 1) & 1u))) break;
-        dst_off = kOffK + (uk & 1) * kF16Tile;
-      } else {
-        if (j >= 2 && !(ok = wwait(bar(B_V16_EMPTY + (j & 1)), (uint32_t)((j >> 1) - 1) & 1u))) break;
-        dst_off = kOffV + (j & 1) * kF16Tile;
-      }
-      const uint8_t* src = base_ptr + kOffStg + s * kStgTile;
-      uint8_t* dst = base_ptr + dst_off;
-      // rows of this tile that hold live keys (V rows past L read as zero)
-      const int live = is_v ? min(kTileRows, L - j * kTileRows) : kTileRows;
-#pragma unroll 2
-      for (int pass = 0; pass < 8; ++pass) {
-        const int row = pass * 16 + r_in;
-        const uint4 w = *reinterpret_cast<const uint4*>(src + row * 128 + ((c ^ (row & 7)) << 4));
-        uint32_t f[8];
-        if (is_v) {
-          e4m3x4_to_f16(w.x, f[0], f[1]);
-          e4m3x4_to_f16(w.y, f[2], f[3]);
-          e4m3x4_to_f16(w.z, f[4], f[5]);
-          e4m3x4_to_f16(w.w, f[6], f[7]);
-          if (row >= live) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0u;
-          }
-        } else {
-          s8x4_to_f16(w.x, f[0], f[1]);
-          s8x4_to_f16(w.y, f[2], f[3]);
-          s8x4_to_f16(w.z, f[4], f[5]);
-          s8x4_to_f16(w.w, f[6], f[7]);
-        }
-        // elements d = 16 c .. 16 c + 15 -> half c / 4, 16-byte units 2 (c % 4) and 2 (c % 4) + 1
-        const int half = c >> 2, u0 = 2 * (c & 3);
-        uint8_t* drow = dst + half * kHalf + row * 128;
-        *reinterpret_cast<uint4*>(drow + ((u0 ^ (row & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
-        *reinterpret_cast<uint4*>(drow + (((u0 + 1) ^ (row & 7)) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
-      }
-      fence_proxy_async();                                     // the f16 tile is read by the tensor cores
-      mbar_arrive(bar(B_STG_EMPTY + s));
-      if (t == 0) mbar_arrive(bar(B_Q16));
-      else if (!is_v) mbar_arrive(bar(B_K16_FULL + (uk & 1)));
-      else mbar_arrive(bar(B_V16_FULL + (j & 1)));
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_STG_FULL + stage_of(t)), full_parity(t)); ++i) {}
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = wait(bar(B_Q16), 0);
+      bool ok = wait(bar(B_Q), 0);
       // S(g) into TMEM buffer g % 3 once its previous user (g - 3) is done with it
       auto issue_s = [&](int g) -> bool {
         const int b = g % 3;
-        if (!wait(bar(B_K16_FULL + (g & 1)), (uint32_t)(g >> 1) & 1u)) return false;
+        const int t = g < n ? g : n + 2 * (g - n);
+        if (!wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))) return false;
         if (g >= 3) {
           const int p = g - 3;
           if (p < n) { if (!wait(bar(B_S_READ + b), (uint32_t)(p / 3) & 1u)) return false; }
           else if (!wait(bar(B_PV_DONE + b), (uint32_t)((p - n) / 3) & 1u)) return false;
         }
         tc_fence_after();
-        const uint32_t kb = base + kOffK + (g & 1) * kF16Tile;
+        const uint32_t kb = base + kOffStg + stage_of(t) * kTile8;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // 8 steps of 16 over d
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          tc_mma(tmem + 128 * b, smem_desc(base + kOffQ + off, 16), smem_desc(kb + off, 16), kIdescS, kk > 0);
-        }
+        for (int kk = 0; kk < 4; ++kk)   // 4 steps of 32 bytes over d
+          mma_i8(tmem + 128 * b, smem_desc(base + kOffQ + kk * 32), smem_desc(kb + kk * 32), kk > 0);
         tc_commit(bar(B_S_FULL + b));
-        tc_commit(bar(B_K16_EMPTY + (g & 1)));
+        tc_commit(bar(B_STG_EMPTY + stage_of(t)));
         return true;
       };
       for (int g = 0; ok && g < n; ++g) ok = issue_s(g);                          // pass 1
       for (int g = n; ok && g < min(2 * n, n + 2); ++g) ok = issue_s(g);           // pass 2, two ahead
       for (int j = 0; ok && j < n; ++j) {
-        const int g = n + j, b = g % 3;
-        if (!(ok = wait(bar(B_P_FULL + b), (uint32_t)(j / 3) & 1u) && wait(bar(B_V16_FULL + (j & 1)), (uint32_t)(j >> 1) & 1u)))
+        const int g = n + j, b = g % 3, t = n + 2 * j + 1;
+        if (!(ok = wait(bar(B_P_FULL + b), (uint32_t)(j / 3) & 1u) && wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))))
           break;
         tc_fence_after();
-        const int nsteps = (min(kTileRows, L - j * kTileRows) + 15) / 16;   // 16-key steps that hold live keys
-        const uint32_t vb = base + kOffV + (j & 1) * kF16Tile;
+        const int nsteps = (min(kTileRows, L - j * kTileRows) + 31) / 32;   // 32-key steps that hold live keys
+        const uint32_t vb = base + kOffStg + stage_of(t) * kTile8;
         for (int kk = 0; kk < nsteps; ++kk)
-          tc_mma_ts(tmem_o, tmem + 128 * b + 8 * kk, smem_desc(vb + kk * 16 * 128, kHalf), kIdescPV,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+          mma_f8_ts(tmem_o, tmem + 128 * b + 8 * kk, smem_desc(vb + kk * 32 * 128), (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_PV_DONE + b));
-        tc_commit(bar(B_V16_EMPTY + (j & 1)));
+        tc_commit(bar(B_STG_EMPTY + stage_of(t)));
         if (g + 2 < 2 * n) ok = issue_s(g + 2);
       }
       if (ok) tc_commit(bar(B_O_DONE));
@@ -416,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
     };
     bool ok = true;
     float m = NEG_INF;
-    // pass 1: the row maximum of the visible scores
+    // pass 1: the row maximum of the visible scores, S = fp32(sfQ sfK) fp32(dot) (the dot is exact)
     for (int j = 0; j < n && ok; ++j) {
       const int b = j % 3;
       float s0, s1;
@@ -437,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
       for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float sval = (cc < 2 ? s0 : s1) * __uint_as_float(sv[cc][e]);   // fp32(sfQ sfK) fp32(dot)
+          const float sval = (cc < 2 ? s0 : s1) * (float)(int)sv[cc][e];
           if (key0 + 32 * cc + e <= limit) mxp[e & 7] = fmaxf(mxp[e & 7], sval);
         }
       m = fmaxf(m, fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
@@ -445,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
     }
     const float m_use = m == NEG_INF ? 0.f : m;
     float l = 0.f;
-    // pass 2: P8 = E4M3(448 exp(S - m)) over the scores (as f16 pairs), l of the unquantised p
+    // pass 2: P8 = E4M3(448 exp(S - m)) over the scores, four codes per column; l of the unquantised p
     for (int j = 0; j < n && ok; ++j) {
       const int g = n + j, b = g % 3;
       float s0, s1;
@@ -459,22 +362,38 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
         uint32_t sv[32];
         tmem_ld32(tmem + 128 * b + lane_off + 32 * cc, sv);
         tmem_wait_ld();
-        uint32_t pw[16];
+        const float sc = cc < 2 ? s0 : s1;
+        uint32_t pw[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float sc = cc < 2 ? s0 : s1;
-          const int k = key0 + 32 * cc + e;
-          const float p0 = k <= limit ? ex2((sc * __uint_as_float(sv[e]) - m_use) * kLog2e) : 0.f;
-          const float p1 = k + 1 <= limit ? ex2((sc * __uint_as_float(sv[e + 1]) - m_use) * kLog2e) : 0.f;
-          ltp[(e >> 1) & 3] += p0 + p1;
-          pw[e >> 1] = p8_pair_f16(448.f * p0, 448.f * p1);
+        for (int e = 0; e < 32; e += 4) {
+          float p[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int k = key0 + 32 * cc + e + u;
+            p[u] = k <= limit ? ex2((sc * (float)(int)sv[e + u] - m_use) * kLog2e) : 0.f;
+          }
+          ltp[(e >> 2) & 3] += (p[0] + p[1]) + (p[2] + p[3]);
+          pw[e >> 2] = e4m3x2(448.f * p[0], 448.f * p[1]) | (e4m3x2(448.f * p[2], 448.f * p[3]) << 16);
         }
-        // column 16 cc + i holds keys 32 cc + 2i (low half) and 32 cc + 2i + 1: the scores
-        // of this 32-key block have been read, and the block's pairs land inside it
-        tmem_st16(tmem + 128 * b + lane_off + 16 * cc, pw);
+        // column 8 cc + i holds keys 32 cc + 4i .. +3 (low byte first): every column written
+        // here lies in the first 32, which were read above
+        tmem_st8(tmem + 128 * b + lane_off + 8 * cc, pw);
       }
       tmem_wait_st();
       l += (ltp[0] + ltp[1]) + (ltp[2] + ltp[3]);
+      // the last tile: V8 rows past L inside the last 32-key step must read as zero
+      const int live = min(kTileRows, L - j * kTileRows);
+      if ((live & 31) && warp == 2) {
+        const int t = n + 2 * j + 1;
+        if (!(ok = wwait(bar(B_STG_FULL + stage_of(t)), full_parity(t)))) break;
+        const int z1 = (live + 31) & ~31;
+        uint8_t* vt = base_ptr + kOffStg + stage_of(t) * kTile8;
+        for (int idx = lane; idx < (z1 - live) * 8; idx += 32) {   // 16-byte units of rows live .. z1-1
+          const int rr = live + idx / 8, un = idx & 7;
+          *reinterpret_cast<uint4*>(vt + rr * 128 + un * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+      }
       tc_fence_before();
       mbar_arrive(bar(B_P_FULL + b));
     }
