@@ -9,25 +9,29 @@
 //     O[d] = sfV[h_kv][d] * (sum_j P8_j V8_j[d]) / (448 l) + v_mean[h_kv][d];
 // the dense Sage variant the pages measure at S = 10800 (same page, performance item 2).
 //
-// P8 needs the exact row max before any probability is formed, so a CTA (one query tile
-// of 128 new tokens, one head) makes two passes over its key tiles: pass 1 computes
-// S = Q K^T and each row's maximum, pass 2 computes S again, P8 and O += P8 V.  Both
-// contractions run on the 8-bit tensor cores: S on tcgen05.mma kind::i8 (int8 x int8 into
-// int32, exact), P8 V on kind::f8f6f4 (E4M3 x E4M3 into fp32), with P8 taken from TMEM
-// (four E4M3 codes per 32-bit column) and V8 read in place as an MN-major operand.  The
-// 8-bit tiles land from TMA in the operands' 128-byte-swizzled layouts, so nothing is
-// converted on chip.  Roles (6 warps):
-//   warp 0      producer: Q8 once, then TMA boxes of 64 slots (one page) x 128 bytes into an
-//               8-stage ring of 16 KB tiles, in the order K8(0..n-1) (pass 1), then K8(0),
-//               V8(0), K8(1), V8(1), ... (pass 2);
-//   warp 1      MMA issuer: S(g) = Q K(g)^T into TMEM buffer g % 3 (g = 0 .. 2n-1 over both
-//               passes), and in pass 2 O += P8 V(j) with P8 from TMEM; a stage is released
-//               when the MMA that read it completes;
-//   warps 2-5   softmax: thread i owns query row i (TMEM lane i); pass 1 reduces the row
-//               maximum of the causally masked scores, pass 2 writes P8 over the scores in
-//               TMEM and sums l; at the end it applies the epilogue.  V8 rows past the
-//               request's last key inside the last 32-key step are zeroed before PV reads
-//               them (0 x NaN would poison O).
+// P8 needs the exact row max before any probability is formed, so a CTA makes two passes
+// over its key tiles: pass 1 computes S = Q K^T and each row's maximum, pass 2 computes S
+// again, P8 and O += P8 V.  A CTA owns one query tile of 128 new tokens and NH query heads
+// of one KV group (NH = 2 when the group size is even, else 1): every K8 and V8 tile it
+// loads serves all NH heads, which halves the tile traffic per head against one head per
+// CTA.  Both contractions run on the 8-bit tensor cores: S on tcgen05.mma kind::i8 (int8 x
+// int8 into int32, exact), P8 V on kind::f8f6f4 (E4M3 x E4M3 into fp32) with P8 from a
+// shared-memory tile (K-major, 128-byte swizzle) and V8 read in place as an MN-major
+// operand.  The 8-bit tiles land from TMA in the operands' 128-byte-swizzled layouts, so
+// nothing is converted on chip.  TMEM holds one S buffer and the O accumulator per head.
+// Roles (2 + 4 NH warps):
+//   warp 0      producer: Q8 of the NH heads once, then TMA boxes of 64 slots (one page) x
+//               128 bytes into an 8-stage ring of 16 KB tiles, in the order K8(0..n-1)
+//               (pass 1), then K8(0), V8(0), K8(1), V8(1), ... (pass 2);
+//   warp 1      MMA issuer: S(g) of every head (g = 0 .. 2n-1 over both passes) as soon as
+//               the softmax has taken S(g-1) into registers, so S(j+1) runs while the
+//               softmax works on tile j; in pass 2, O += P8 V(j) per head once P8(j) is
+//               written; a stage is released when the MMAs that read it complete;
+//   warps 2..   softmax, one warpgroup per head: thread i owns query row i (TMEM lane i);
+//               pass 1 reduces the row maximum of the causally masked scores, pass 2
+//               writes P8 into the head's P buffer j % 2 and sums l; at the end it applies
+//               the epilogue.  V8 rows past the request's last key inside the last 32-key
+//               step are zeroed before PV reads them (0 x NaN would poison O).
 // Every wait on an mbarrier is bounded: on timeout the CTA records PA_ERR_DEVICE_INDEX,
 // its roles stop, the producer waits for its copies, the MMA issuer drains the tensor
 // cores, and TMEM is freed before exit.
@@ -37,28 +41,34 @@
 namespace pa {
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kTileRows = 128;                     // query rows and keys per tile
 constexpr int kTile8 = 128 * 128;                  // 128 rows x 128 bytes of 8-bit data (16 KB)
 constexpr int kStg = 8;                            // ring stages
-constexpr uint32_t kTmemCols = 512;                // S0, S1, S2 (int32), O (fp32)
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr int kOffQ = 0;
-constexpr int kOffStg = kOffQ + kTile8;            // [kStg]
-constexpr int kOffBar = kOffStg + kStg * kTile8;
-constexpr int kSmemBytes = kOffBar + 512 + 1024;
+// NH query heads of one KV group per CTA (2 when the group size is even, else 1)
+template <int NH>
+struct Cfg {
+  static constexpr int kThreads = 64 + 128 * NH;           // producer, MMA issuer, NH softmax warpgroups
+  static constexpr uint32_t kTmemCols = 256 * NH;          // S (int32) of each head, then O (fp32) of each head
+  static constexpr int kOffQ = 0;                          // [NH] Q8 tiles
+  static constexpr int kOffP = kOffQ + NH * kTile8;        // [NH][2] P8 tiles
+  static constexpr int kOffStg = kOffP + 2 * NH * kTile8;  // [kStg] K8 / V8 ring
+  static constexpr int kOffBar = kOffStg + kStg * kTile8;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+};
+static_assert(Cfg<2>::kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 enum Bar {
   B_STG_FULL = 0,                  // [kStg] tile landed (TMA)
   B_STG_EMPTY = B_STG_FULL + kStg, // [kStg] the MMA that read it has completed (commit)
-  B_Q = B_STG_EMPTY + kStg,        // Q8 landed
-  B_S_FULL,                        // [3] S(g) in TMEM (commit)
-  B_S_READ = B_S_FULL + 3,         // [3] pass 1: softmax has read S(g) (128)
-  B_P_FULL = B_S_READ + 3,         // [3] pass 2: P8(g) written over S(g) (128)
-  B_PV_DONE = B_P_FULL + 3,        // [3] pass 2: PV(g) done (commit)
-  B_O_DONE = B_PV_DONE + 3,        // every PV done (commit)
+  B_Q = B_STG_EMPTY + kStg,        // Q8 of the NH heads landed
+  B_S_FULL,                        // S(g) of every head in TMEM (commit)
+  B_S_READ,                        // every softmax thread has S(g) in registers (128 NH)
+  B_P_FULL,                        // [2] P8(j) of every head in its shared-memory buffer j % 2 (128 NH)
+  B_PV_DONE = B_P_FULL + 2,        // [2] PV(j) of every head done: buffer j % 2 is free (commit)
+  B_O_DONE = B_PV_DONE + 2,        // every PV done (commit)
   B_DRAIN,
   B_COUNT
 };
@@ -66,7 +76,7 @@ static_assert(B_COUNT * 8 + 16 <= 512, "barrier area");
 
 // instruction descriptors, M = 128, N = 128
 //   S:  kind::i8, s32 D, s8 A and B, both K-major
-//   PV: kind::f8f6f4, f32 D, E4M3 A (from TMEM, K-major) and B (V8, MN-major)
+//   PV: kind::f8f6f4, f32 D, E4M3 A (P8, K-major) and B (V8, MN-major)
 constexpr uint32_t kIdescS = (2u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
@@ -103,11 +113,11 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdescS), "r"(accumulate)
       : "memory");
 }
-// D (TMEM, f32) += A (TMEM, E4M3, four per column) x B (smem, E4M3)
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
+// D (TMEM, f32) += A (smem, E4M3) x B (smem, E4M3)
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(kIdescPV), "r"(accumulate)
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdescPV), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -123,13 +133,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n"
-               ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 // Two floats to E4M3 codes (nearest even, saturating); `lo` in the low byte.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
@@ -138,50 +142,51 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_constant__ SageExtendLaunch a) {
+template <int NH>
+__global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const __grid_constant__ SageExtendLaunch a) {
+  using C = Cfg<NH>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t bars = base + kOffBar;
+  const uint32_t bars = base + C::kOffBar;
   auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffBar + 8 * B_COUNT);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBar + 8 * B_COUNT + 8);
-
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffBar + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffBar + 8 * B_COUNT + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   PlanHeader* hdr = a.ws.hdr;
   if (hdr->magic != kMagic || hdr->mode != PA_MODE_EXTEND || hdr->page_size != kSageBlock) {
     if (tid == 0 && blockIdx.x == 0) set_device_error(hdr, PA_ERR_WORKSPACE);
     return;
   }
-  const int item = blockIdx.x / a.hq, h = blockIdx.x % a.hq;
+  const int ctas_per_item = a.hq / NH;
+  const int item = blockIdx.x / ctas_per_item, h0 = (blockIdx.x % ctas_per_item) * NH;
   if (item >= hdr->num_items) return;
   const int4 it = a.ws.items[item];
   const int r = it.x, q_begin = it.z, q_end = it.w;
   const int L = a.ws.req_len[r], prefix = a.ws.req_prefix[r], q_start = a.ws.req_aux[r];
-  const int h_kv = h / (a.hq / a.hkv);
+  const int h_kv = h0 / (a.hq / a.hkv);                    // shared by the CTA's NH heads
   const int kv_end = prefix + q_end;                         // keys any row of this tile can see
   const int n = (kv_end + kTileRows - 1) / kTileRows;       // key tiles
   const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
-      const bool many = (i >= B_S_READ && i < B_S_READ + 3) || (i >= B_P_FULL && i < B_P_FULL + 3);
-      mbar_init(bar(i), many ? 128 : 1);
+      const bool many = i == B_S_READ || i == B_P_FULL || i == B_P_FULL + 1;
+      mbar_init(bar(i), many ? 128 * NH : 1);
     }
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
-                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+                 ::"r"(smem_u32(tmem_slot)), "r"(C::kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 384;
 
   auto wait = [&](uint32_t b, uint32_t parity) -> bool {
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -212,8 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
     if (lane == 0) {
-      mbar_expect_tx(bar(B_Q), kTile8);
-      tma_load_3d(base + kOffQ, &a.tm_q8, 0, q_start + q_begin, h, bar(B_Q));
+      mbar_expect_tx(bar(B_Q), NH * kTile8);
+      for (int hh = 0; hh < NH; ++hh)
+        tma_load_3d(base + C::kOffQ + hh * kTile8, &a.tm_q8, 0, q_start + q_begin, h0 + hh, bar(B_Q));
     }
     int issued = 0;
     int pg_lo = -1, pg_hi = -1;   // this lane's pages for the tile j = tb + lane of the current round
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
       if (lane == 0) {
         ok = t < kStg || wait(bar(B_STG_EMPTY + s), (uint32_t)((t / kStg) - 1) & 1u);
         if (ok) {
-          const uint32_t dst = base + kOffStg + s * kTile8;
+          const uint32_t dst = base + C::kOffStg + s * kTile8;
           const uint32_t bytes = (plo >= 0 ? kTile8 / 2 : 0) + (phi >= 0 ? kTile8 / 2 : 0);
           mbar_expect_tx(bar(B_STG_FULL + s), bytes);
           const CUtensorMap* tm = is_v ? &a.tm_v8 : &a.tm_k8;
@@ -254,39 +260,41 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = wait(bar(B_Q), 0);
-      // S(g) into TMEM buffer g % 3 once its previous user (g - 3) is done with it
+      // S(g) of every head of the CTA (g = 0 .. 2n-1 over both passes) into its one TMEM
+      // buffer, once every softmax thread has taken S(g-1) into registers
       auto issue_s = [&](int g) -> bool {
-        const int b = g % 3;
         const int t = g < n ? g : n + 2 * (g - n);
         if (!wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))) return false;
-        if (g >= 3) {
-          const int p = g - 3;
-          if (p < n) { if (!wait(bar(B_S_READ + b), (uint32_t)(p / 3) & 1u)) return false; }
-          else if (!wait(bar(B_PV_DONE + b), (uint32_t)((p - n) / 3) & 1u)) return false;
-        }
+        if (g > 0 && !wait(bar(B_S_READ), (uint32_t)(g - 1) & 1u)) return false;
         tc_fence_after();
-        const uint32_t kb = base + kOffStg + stage_of(t) * kTile8;
+        const uint32_t kb = base + C::kOffStg + stage_of(t) * kTile8;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)   // 4 steps of 32 bytes over d
-          mma_i8(tmem + 128 * b, smem_desc(base + kOffQ + kk * 32), smem_desc(kb + kk * 32), kk > 0);
-        tc_commit(bar(B_S_FULL + b));
+        for (int hh = 0; hh < NH; ++hh)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 4 steps of 32 bytes over d
+            mma_i8(tmem + 128 * hh, smem_desc(base + C::kOffQ + hh * kTile8 + kk * 32), smem_desc(kb + kk * 32), kk > 0);
+        tc_commit(bar(B_S_FULL));
         tc_commit(bar(B_STG_EMPTY + stage_of(t)));
         return true;
       };
-      for (int g = 0; ok && g < n; ++g) ok = issue_s(g);                          // pass 1
-      for (int g = n; ok && g < min(2 * n, n + 2); ++g) ok = issue_s(g);           // pass 2, two ahead
+      for (int g = 0; ok && g <= n; ++g) ok = issue_s(g);   // pass 1, then S(0) of pass 2
       for (int j = 0; ok && j < n; ++j) {
-        const int g = n + j, b = g % 3, t = n + 2 * j + 1;
-        if (!(ok = wait(bar(B_P_FULL + b), (uint32_t)(j / 3) & 1u) && wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))))
+        // S(j + 1) runs on the tensor cores while the softmax turns S(j) into P8(j)
+        if (j + 1 < n && !(ok = issue_s(n + j + 1))) break;
+        const int t = n + 2 * j + 1;   // V8(j)
+        if (!(ok = wait(bar(B_P_FULL + (j & 1)), (uint32_t)(j >> 1) & 1u) && wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))))
           break;
         tc_fence_after();
         const int nsteps = (min(kTileRows, L - j * kTileRows) + 31) / 32;   // 32-key steps that hold live keys
-        const uint32_t vb = base + kOffStg + stage_of(t) * kTile8;
-        for (int kk = 0; kk < nsteps; ++kk)
-          mma_f8_ts(tmem_o, tmem + 128 * b + 8 * kk, smem_desc(vb + kk * 32 * 128), (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_PV_DONE + b));
+        const uint32_t vb = base + C::kOffStg + stage_of(t) * kTile8;
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          const uint32_t pb = base + C::kOffP + (2 * hh + (j & 1)) * kTile8;
+          for (int kk = 0; kk < nsteps; ++kk)
+            mma_f8(tmem + 128 * (NH + hh), smem_desc(pb + kk * 32), smem_desc(vb + kk * 32 * 128), (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(B_PV_DONE + (j & 1)));
         tc_commit(bar(B_STG_EMPTY + stage_of(t)));
-        if (g + 2 < 2 * n) ok = issue_s(g + 2);
       }
       if (ok) tc_commit(bar(B_O_DONE));
       // all issued tensor-core work has finished before TMEM is released
@@ -294,9 +302,14 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++i) {}
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 2-5)
+    // ------------------------------------------------------------ softmax (one warpgroup per head)
+    const int wg = (warp - 2) >> 2, h = h0 + wg;
     const int row = 32 * (warp & 3) + lane;                    // TMEM lane = query row of the tile
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tmem_s = tmem + 128 * wg + lane_off, tmem_o = tmem + 128 * (NH + wg) + lane_off;
+    // this row of a P8 tile: K-major, 128-byte swizzle (16-byte chunk c at c ^ (row & 7))
+    const uint32_t p_row = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+    const int sw = row & 7;
     const int q_local = q_begin + row;
     const bool row_valid = q_local < q_end && q_start + q_local < a.q_rows;
     const int limit = row_valid ? prefix + q_local : -1;       // last visible key (inclusive)
@@ -317,21 +330,25 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
       s0 = sfq * __shfl_sync(0xffffffffu, sk_lo, j & 31);
       s1 = sfq * __shfl_sync(0xffffffffu, sk_hi, j & 31);
     };
+    // S(g) into registers; the MMA issuer may then overwrite the buffer with S(g + 1)
+    auto take_s = [&](int g, uint32_t (&sv)[4][32]) -> bool {
+      if (!wwait(bar(B_S_FULL), (uint32_t)g & 1u)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem_s + 32 * cc, sv[cc]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_S_READ));
+      return true;
+    };
     bool ok = true;
     float m = NEG_INF;
     // pass 1: the row maximum of the visible scores, S = fp32(sfQ sfK) fp32(dot) (the dot is exact)
     for (int j = 0; j < n && ok; ++j) {
-      const int b = j % 3;
       float s0, s1;
       scales(j, s0, s1);
-      if (!(ok = wwait(bar(B_S_FULL + b), (uint32_t)(j / 3) & 1u))) break;
-      tc_fence_after();
       uint32_t sv[4][32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + 128 * b + lane_off + 32 * cc, sv[cc]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_S_READ + b));
+      if (!(ok = take_s(j, sv))) break;
       const int key0 = j * kTileRows;
       float mxp[8];
 #pragma unroll
@@ -348,20 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
     }
     const float m_use = m == NEG_INF ? 0.f : m;
     float l = 0.f;
-    // pass 2: P8 = E4M3(448 exp(S - m)) over the scores, four codes per column; l of the unquantised p
+    // pass 2: P8 = E4M3(448 exp(S - m)) into a shared-memory P tile; l of the unquantised p
     for (int j = 0; j < n && ok; ++j) {
-      const int g = n + j, b = g % 3;
       float s0, s1;
       scales(j, s0, s1);
-      if (!(ok = wwait(bar(B_S_FULL + b), (uint32_t)(g / 3) & 1u))) break;
-      tc_fence_after();
+      uint32_t sv[4][32];
+      if (!(ok = take_s(n + j, sv))) break;
+      // the P buffer's previous tile (j - 2) has been multiplied
+      if (j >= 2 && !(ok = wwait(bar(B_PV_DONE + (j & 1)), (uint32_t)((j >> 1) - 1) & 1u))) break;
+      uint8_t* prow = base_ptr + C::kOffP + (2 * wg + (j & 1)) * kTile8 + p_row;
       const int key0 = j * kTileRows;
       float ltp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32];
-        tmem_ld32(tmem + 128 * b + lane_off + 32 * cc, sv);
-        tmem_wait_ld();
         const float sc = cc < 2 ? s0 : s1;
         uint32_t pw[8];
 #pragma unroll
@@ -370,32 +386,31 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int k = key0 + 32 * cc + e + u;
-            p[u] = k <= limit ? ex2((sc * (float)(int)sv[e + u] - m_use) * kLog2e) : 0.f;
+            p[u] = k <= limit ? ex2((sc * (float)(int)sv[cc][e + u] - m_use) * kLog2e) : 0.f;
           }
           ltp[(e >> 2) & 3] += (p[0] + p[1]) + (p[2] + p[3]);
           pw[e >> 2] = e4m3x2(448.f * p[0], 448.f * p[1]) | (e4m3x2(448.f * p[2], 448.f * p[3]) << 16);
         }
-        // column 8 cc + i holds keys 32 cc + 4i .. +3 (low byte first): every column written
-        // here lies in the first 32, which were read above
-        tmem_st8(tmem + 128 * b + lane_off + 8 * cc, pw);
+        // keys 32 cc .. 32 cc + 31 are the 16-byte chunks 2 cc and 2 cc + 1 of the row
+        *reinterpret_cast<uint4*>(prow + (((2 * cc) ^ sw) << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        *reinterpret_cast<uint4*>(prow + (((2 * cc + 1) ^ sw) << 4)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
       }
-      tmem_wait_st();
       l += (ltp[0] + ltp[1]) + (ltp[2] + ltp[3]);
-      // the last tile: V8 rows past L inside the last 32-key step must read as zero
+      // the last tile: V8 rows past L inside the last 32-key step must read as zero (each
+      // warpgroup's first warp writes the same zeros before its own P_FULL arrival)
       const int live = min(kTileRows, L - j * kTileRows);
-      if ((live & 31) && warp == 2) {
+      if ((live & 31) && (warp & 3) == 2) {
         const int t = n + 2 * j + 1;
         if (!(ok = wwait(bar(B_STG_FULL + stage_of(t)), full_parity(t)))) break;
         const int z1 = (live + 31) & ~31;
-        uint8_t* vt = base_ptr + kOffStg + stage_of(t) * kTile8;
+        uint8_t* vt = base_ptr + C::kOffStg + stage_of(t) * kTile8;
         for (int idx = lane; idx < (z1 - live) * 8; idx += 32) {   // 16-byte units of rows live .. z1-1
           const int rr = live + idx / 8, un = idx & 7;
           *reinterpret_cast<uint4*>(vt + rr * 128 + un * 16) = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async();
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_P_FULL + b));
+      fence_proxy_async();   // the P8 stores (and zeroed V8 rows) are read by the tensor cores
+      mbar_arrive(bar(B_P_FULL + (j & 1)));
     }
     if (ok) ok = wwait(bar(B_O_DONE), 0);
     if (ok) {
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t ov[32];
-        tmem_ld32(tmem_o + lane_off + 32 * cc, ov);
+        tmem_ld32(tmem_o + 32 * cc, ov);
         tmem_wait_ld();
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -431,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_extend_kernel(const __grid_c
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(C::kTmemCols) : "memory");
   }
 }
 
@@ -455,7 +470,10 @@ cudaError_t launch_sage_extend(const SageExtendArgs& in, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sage_extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(sage_extend_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<1>::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sage_extend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<2>::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -476,7 +494,10 @@ cudaError_t launch_sage_extend(const SageExtendArgs& in, cudaStream_t s) {
   a.out = in.out;
   a.hq = in.hq;
   a.hkv = in.hkv;
-  sage_extend_kernel<<<in.max_items * in.hq, kThreads, kSmemBytes, s>>>(a);
+  if ((in.hq / in.hkv) % 2 == 0)
+    sage_extend_kernel<2><<<in.max_items * (in.hq / 2), Cfg<2>::kThreads, Cfg<2>::kSmemBytes, s>>>(a);
+  else
+    sage_extend_kernel<1><<<in.max_items * in.hq, Cfg<1>::kThreads, Cfg<1>::kSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 
