@@ -51,7 +51,12 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running."""
+    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running.
+
+    Entering waits (up to 5 s) for the first sample, so that the sampler is live before the
+    timed region starts; each line is stamped on arrival, and `mark_start` / `mark_end`
+    bracket the timed region so that the summary keeps the samples taken during it (the
+    first one after its start when it is shorter than the sampling period)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -60,6 +65,13 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def __enter__(self):
         try:
@@ -68,13 +80,16 @@ class ClockSampler:
                  "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.monotonic() + 5.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -87,7 +102,12 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines = list(self.lines)
+        if self.t0 is not None and self.t1 is not None:
+            inside = [x for x in lines if self.t0 <= x[0] <= self.t1]
+            # a region shorter than the period: the first sample after its start
+            lines = inside or [x for x in lines if x[0] >= self.t0][:1]
+        for _, line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -623,13 +643,13 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        clocks.mark_start()
         start.record()
         for s in range(args.steps):
             work.step(layer_events)
-            if s == args.steps - 1:
-                pass
         end.record()
         torch.cuda.synchronize()
+        clocks.mark_end()
         # per-layer durations of the last step (the events are re-recorded every step)
         layer_ms = [a.elapsed_time(b) for a, b in layer_events]
     total_ms = max_over_ranks(dist, start.elapsed_time(end), dev)

@@ -35,6 +35,8 @@
 // Every wait on an mbarrier is bounded: on timeout the CTA records PA_ERR_DEVICE_INDEX,
 // its roles stop, the producer waits for its copies, the MMA issuer drains the tensor
 // cores, and TMEM is freed before exit.
+#include <climits>
+
 #include "kernels.h"
 #include "tma.cuh"
 
@@ -46,6 +48,12 @@ constexpr int kTile8 = 128 * 128;                  // 128 rows x 128 bytes of 8-
 constexpr int kStg = 8;                            // ring stages
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.8073549220576041f;   // log2(448): 448 e^x = 2^(x log2(e) + log2(448))
+// int32 -> fp32 without the conversion unit: for |v| < 2^22 the bits 0x4B400000 + v are the
+// float 1.5 * 2^23 + v exactly, and subtracting 1.5 * 2^23 leaves fp32(v) exactly (the
+// dots here are at most 128 * 128 * 128 = 2^21 in magnitude)
+constexpr int kCvtBiasBits = 0x4B400000;
+constexpr float kCvtBias = 12582912.f;
 
 // NH query heads of one KV group per CTA (2 when the group size is even, else 1)
 template <int NH>
@@ -343,28 +351,55 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     };
     bool ok = true;
     float m = NEG_INF;
-    // pass 1: the row maximum of the visible scores, S = fp32(sfQ sfK) fp32(dot) (the dot is exact)
+    // pass 1: the row maximum of the visible scores, S = fp32(sfQ sfK) fp32(dot) (the dot is
+    // exact).  Rounding is monotonic, so over one page half (one scale sc) the maximum of
+    // fp32(sc x) is fp32(sc max x) for sc >= 0 and fp32(sc min x) for sc < 0: the reduction
+    // runs on the int32 dots and converts two values per tile.
     for (int j = 0; j < n && ok; ++j) {
       float s0, s1;
       scales(j, s0, s1);
       uint32_t sv[4][32];
       if (!(ok = take_s(j, sv))) break;
       const int key0 = j * kTileRows;
-      float mxp[8];
+      const bool nonneg = __all_sync(0xffffffffu, s0 >= 0.f && s1 >= 0.f);
+      int mx[2] = {INT_MIN, INT_MIN}, mn[2] = {INT_MAX, INT_MAX};
+      if (__all_sync(0xffffffffu, key0 + kTileRows - 1 <= limit)) {   // every key visible to the warp's rows
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mxp[i] = NEG_INF;
+        for (int hf = 0; hf < 2; ++hf) {
+          int a0 = INT_MIN, a1 = INT_MIN, b0 = INT_MAX, b1 = INT_MAX;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float sval = (cc < 2 ? s0 : s1) * (float)(int)sv[cc][e];
-          if (key0 + 32 * cc + e <= limit) mxp[e & 7] = fmaxf(mxp[e & 7], sval);
+          for (int e = 0; e < 64; e += 4) {
+            const int* v = reinterpret_cast<const int*>(sv[2 * hf + (e >> 5)]) + (e & 31);
+            a0 = __vimax3_s32(a0, v[0], v[1]);
+            a1 = __vimax3_s32(a1, v[2], v[3]);
+            if (!nonneg) {
+              b0 = __vimin3_s32(b0, v[0], v[1]);
+              b1 = __vimin3_s32(b1, v[2], v[3]);
+            }
+          }
+          mx[hf] = max(a0, a1);
+          mn[hf] = min(b0, b1);
         }
-      m = fmaxf(m, fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))));
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int v = (int)sv[cc][e];
+            const bool vis = key0 + 32 * cc + e <= limit;
+            mx[cc >> 1] = vis ? max(mx[cc >> 1], v) : mx[cc >> 1];
+            mn[cc >> 1] = vis ? min(mn[cc >> 1], v) : mn[cc >> 1];
+          }
+      }
+      // a dot is at most 2^21 in magnitude, so INT_MIN marks a half with no visible key
+      if (mx[0] != INT_MIN) m = fmaxf(m, s0 * (float)(s0 >= 0.f ? mx[0] : mn[0]));
+      if (mx[1] != INT_MIN) m = fmaxf(m, s1 * (float)(s1 >= 0.f ? mx[1] : mn[1]));
     }
     const float m_use = m == NEG_INF ? 0.f : m;
-    float l = 0.f;
+    // exponent of 448 e^(S - m) as one fused multiply-add of the exact fp32 dot:
+    // x (sc log2 e) + (log2 448 - m log2 e)
+    const float c2 = kLog2_448 - m_use * kLog2e;
+    float2 l2 = make_float2(0.f, 0.f);   // l scaled by 448
     // pass 2: P8 = E4M3(448 exp(S - m)) into a shared-memory P tile; l of the unquantised p
     for (int j = 0; j < n && ok; ++j) {
       float s0, s1;
@@ -375,27 +410,36 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
       if (j >= 2 && !(ok = wwait(bar(B_PV_DONE + (j & 1)), (uint32_t)((j >> 1) - 1) & 1u))) break;
       uint8_t* prow = base_ptr + C::kOffP + (2 * wg + (j & 1)) * kTile8 + p_row;
       const int key0 = j * kTileRows;
-      float ltp[4] = {0.f, 0.f, 0.f, 0.f};
+      const bool full = __all_sync(0xffffffffu, key0 + kTileRows - 1 <= limit);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        const float sc = cc < 2 ? s0 : s1;
+        const float a = (cc < 2 ? s0 : s1) * kLog2e;
+        const float2 a2 = make_float2(a, a), c22 = make_float2(c2, c2), nb = make_float2(-kCvtBias, -kCvtBias);
         uint32_t pw[8];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           float p[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int k = key0 + 32 * cc + e + u;
-            p[u] = k <= limit ? ex2((sc * (float)(int)sv[cc][e + u] - m_use) * kLog2e) : 0.f;
+          for (int u = 0; u < 4; u += 2) {
+            float2 x = make_float2(__int_as_float((int)sv[cc][e + u] + kCvtBiasBits),
+                                   __int_as_float((int)sv[cc][e + u + 1] + kCvtBiasBits));
+            x = __fadd2_rn(x, nb);                    // the exact fp32 dots
+            const float2 t = __ffma2_rn(x, a2, c22);
+            p[u] = ex2(t.x);
+            p[u + 1] = ex2(t.y);
+            if (!full) {
+              const int k = key0 + 32 * cc + e + u;
+              if (k > limit) p[u] = 0.f;
+              if (k + 1 > limit) p[u + 1] = 0.f;
+            }
+            l2 = __fadd2_rn(l2, make_float2(p[u], p[u + 1]));
           }
-          ltp[(e >> 2) & 3] += (p[0] + p[1]) + (p[2] + p[3]);
-          pw[e >> 2] = e4m3x2(448.f * p[0], 448.f * p[1]) | (e4m3x2(448.f * p[2], 448.f * p[3]) << 16);
+          pw[e >> 2] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
         }
         // keys 32 cc .. 32 cc + 31 are the 16-byte chunks 2 cc and 2 cc + 1 of the row
         *reinterpret_cast<uint4*>(prow + (((2 * cc) ^ sw) << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         *reinterpret_cast<uint4*>(prow + (((2 * cc + 1) ^ sw) << 4)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
       }
-      l += (ltp[0] + ltp[1]) + (ltp[2] + ltp[3]);
       // the last tile: V8 rows past L inside the last 32-key step must read as zero (each
       // warpgroup's first warp writes the same zeros before its own P_FULL arrival)
       const int live = min(kTileRows, L - j * kTileRows);
@@ -415,7 +459,8 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     if (ok) ok = wwait(bar(B_O_DONE), 0);
     if (ok) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / (448.f * l) : 0.f;
+      const float l448 = l2.x + l2.y;
+      const float inv = l448 > 0.f ? 1.f / l448 : 0.f;
       uint16_t* orow = a.out + ((size_t)(q_start + q_local) * a.hq + h) * kHeadDim;
       const float* sfv = a.sf_v + (size_t)h_kv * kHeadDim;
       const float* vm = a.v_mean ? a.v_mean + (size_t)h_kv * kHeadDim : nullptr;

@@ -63,3 +63,24 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_summary_keeps_the_timed_region():
+    """The clocks reported beside a number are the samples taken while it was timed."""
+    sys.path.insert(0, ROOT)
+    import bench
+    idle = "0, 1000, 1965, 100, 0x0, Not Active, Not Active, Not Active, Not Active"
+    busy = "0, 1965, 1965, 900, 0x4, Not Active, Not Active, Not Active, Active"
+    hot = "0, 1500, 1965, 950, 0x8, Not Active, Not Active, Active, Not Active"
+    c = bench.ClockSampler(0)
+    c.lines = [(0.9, idle), (1.1, busy), (1.3, hot), (1.5, busy), (1.9, idle)]
+    c.t0, c.t1 = 1.0, 1.6
+    got = c.summary()
+    assert got["samples"] == 3 and got["sm_mhz"] == 1965.0 and got["sm_max_mhz"] == 1965.0
+    assert got["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    # shorter than the sampling period: the first sample after the start stands for it
+    c.t0, c.t1 = 1.12, 1.2
+    got = c.summary()
+    assert got["samples"] == 1 and got["sm_mhz"] == 1500.0 and got["reasons"] == ["sw_thermal_slowdown"]
+    c.lines = []
+    assert c.summary()["reasons"] == ["unsampled"]
