@@ -93,6 +93,11 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            # a timed region shorter than the period: wait (up to 1 s) for the sample after it
+            deadline = time.monotonic() + 1.0
+            while (self.t0 is not None and not any(x[0] >= self.t0 for x in list(self.lines))
+                   and time.monotonic() < deadline and self.proc.poll() is None):
+                time.sleep(0.02)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)

@@ -18,15 +18,17 @@
 // int8 into int32, exact), P8 V on kind::f8f6f4 (E4M3 x E4M3 into fp32) with P8 from a
 // shared-memory tile (K-major, 128-byte swizzle) and V8 read in place as an MN-major
 // operand.  The 8-bit tiles land from TMA in the operands' 128-byte-swizzled layouts, so
-// nothing is converted on chip.  TMEM holds one S buffer and the O accumulator per head.
+// nothing is converted on chip.  TMEM holds one S buffer and the O accumulator per head;
+// pass 1, which has no O yet, uses the O columns as a second S buffer.
 // Roles (2 + 4 NH warps):
 //   warp 0      producer: Q8 of the NH heads once, then TMA boxes of 64 slots (one page) x
 //               128 bytes into an 8-stage ring of 16 KB tiles, in the order K8(0..n-1)
 //               (pass 1), then K8(0), V8(0), K8(1), V8(1), ... (pass 2);
 //   warp 1      MMA issuer: S(g) of every head (g = 0 .. 2n-1 over both passes) as soon as
-//               the softmax has taken S(g-1) into registers, so S(j+1) runs while the
-//               softmax works on tile j; in pass 2, O += P8 V(j) per head once P8(j) is
-//               written; a stage is released when the MMAs that read it complete;
+//               the softmax has taken the previous S of its buffer into registers, so the
+//               next S runs while the softmax works on the current one; in pass 2, O +=
+//               P8 V(j) per head once P8(j) is written; a stage is released when the MMAs
+//               that read it complete;
 //   warps 2..   softmax, one warpgroup per head: thread i owns query row i (TMEM lane i);
 //               pass 1 reduces the row maximum of the causally masked scores, pass 2
 //               writes P8 into the head's P buffer j % 2 and sums l; at the end it applies
@@ -72,9 +74,9 @@ enum Bar {
   B_STG_FULL = 0,                  // [kStg] tile landed (TMA)
   B_STG_EMPTY = B_STG_FULL + kStg, // [kStg] the MMA that read it has completed (commit)
   B_Q = B_STG_EMPTY + kStg,        // Q8 of the NH heads landed
-  B_S_FULL,                        // S(g) of every head in TMEM (commit)
-  B_S_READ,                        // every softmax thread has S(g) in registers (128 NH)
-  B_P_FULL,                        // [2] P8(j) of every head in its shared-memory buffer j % 2 (128 NH)
+  B_S_FULL,                        // [2] S(g) of every head in TMEM buffer b (commit)
+  B_S_READ = B_S_FULL + 2,         // [2] every softmax thread has taken S(g) from buffer b (128 NH)
+  B_P_FULL = B_S_READ + 2,         // [2] P8(j) of every head in its shared-memory buffer j % 2 (128 NH)
   B_PV_DONE = B_P_FULL + 2,        // [2] PV(j) of every head done: buffer j % 2 is free (commit)
   B_O_DONE = B_PV_DONE + 2,        // every PV done (commit)
   B_DRAIN,
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
-      const bool many = i == B_S_READ || i == B_P_FULL || i == B_P_FULL + 1;
+      const bool many = (i >= B_S_READ && i < B_S_READ + 2) || i == B_P_FULL || i == B_P_FULL + 1;
       mbar_init(bar(i), many ? 128 * NH : 1);
     }
     *abort_flag = 0;
@@ -221,6 +223,10 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
   const int n_items = 3 * n;
   auto stage_of = [](int t) { return t % kStg; };
   auto full_parity = [](int t) { return (uint32_t)(t / kStg) & 1u; };
+  // S buffers: pass 1 (g < n, no O yet) alternates between buffer 0 and buffer 1, which is
+  // the O region; pass 2 uses buffer 0.  u = how many earlier S went through the same buffer.
+  auto s_buf = [n](int g) { return g < n ? (g & 1) : 0; };
+  auto s_use = [n](int g) { return g < n ? (g >> 1) : ((n + 1) >> 1) + (g - n); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
@@ -268,20 +274,26 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = wait(bar(B_Q), 0);
-      // S(g) of every head of the CTA (g = 0 .. 2n-1 over both passes) into its one TMEM
-      // buffer, once every softmax thread has taken S(g-1) into registers
+      // descriptors of the first tile of each operand region; a tile or 32-byte step further
+      // on is the same descriptor with its start address (bits 0-13, 16-byte units) advanced
+      const uint64_t d_q = smem_desc(base + C::kOffQ), d_p = smem_desc(base + C::kOffP);
+      const uint64_t d_stg = smem_desc(base + C::kOffStg);
+      // S(g) of every head of the CTA (g = 0 .. 2n-1 over both passes) into its buffer, once
+      // every softmax thread has taken the buffer's previous S into registers
       auto issue_s = [&](int g) -> bool {
         const int t = g < n ? g : n + 2 * (g - n);
+        const int b = s_buf(g), u = s_use(g);
         if (!wait(bar(B_STG_FULL + stage_of(t)), full_parity(t))) return false;
-        if (g > 0 && !wait(bar(B_S_READ), (uint32_t)(g - 1) & 1u)) return false;
+        if (u > 0 && !wait(bar(B_S_READ + b), (uint32_t)(u - 1) & 1u)) return false;
         tc_fence_after();
-        const uint32_t kb = base + C::kOffStg + stage_of(t) * kTile8;
+        const uint64_t d_k = d_stg + (uint64_t)((stage_of(t) * kTile8) >> 4);
+        const uint32_t d_s = tmem + 128 * NH * b;
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 4 steps of 32 bytes over d
-            mma_i8(tmem + 128 * hh, smem_desc(base + C::kOffQ + hh * kTile8 + kk * 32), smem_desc(kb + kk * 32), kk > 0);
-        tc_commit(bar(B_S_FULL));
+            mma_i8(d_s + 128 * hh, d_q + (uint64_t)((hh * kTile8 + kk * 32) >> 4), d_k + (uint64_t)(kk * 2), kk > 0);
+        tc_commit(bar(B_S_FULL + b));
         tc_commit(bar(B_STG_EMPTY + stage_of(t)));
         return true;
       };
@@ -294,13 +306,15 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
           break;
         tc_fence_after();
         const int nsteps = (min(kTileRows, L - j * kTileRows) + 31) / 32;   // 32-key steps that hold live keys
-        const uint32_t vb = base + C::kOffStg + stage_of(t) * kTile8;
+        const uint64_t d_v = d_stg + (uint64_t)((stage_of(t) * kTile8) >> 4);
+        const uint64_t d_pj = d_p + (uint64_t)(((j & 1) * kTile8) >> 4);
 #pragma unroll
-        for (int hh = 0; hh < NH; ++hh) {
-          const uint32_t pb = base + C::kOffP + (2 * hh + (j & 1)) * kTile8;
-          for (int kk = 0; kk < nsteps; ++kk)
-            mma_f8(tmem + 128 * (NH + hh), smem_desc(pb + kk * 32), smem_desc(vb + kk * 32 * 128), (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int hh = 0; hh < NH; ++hh)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys per step: 32 bytes of P8, 32 rows (4 KB) of V8
+            if (kk < nsteps)
+              mma_f8(tmem + 128 * (NH + hh), d_pj + (uint64_t)((2 * hh * kTile8 + kk * 32) >> 4),
+                     d_v + (uint64_t)(kk * 256), (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_PV_DONE + (j & 1)));
         tc_commit(bar(B_STG_EMPTY + stage_of(t)));
       }
@@ -314,7 +328,7 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     const int wg = (warp - 2) >> 2, h = h0 + wg;
     const int row = 32 * (warp & 3) + lane;                    // TMEM lane = query row of the tile
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tmem_s = tmem + 128 * wg + lane_off, tmem_o = tmem + 128 * (NH + wg) + lane_off;
+    const uint32_t tmem_s = tmem + 128 * wg + lane_off, tmem_o = tmem + 128 * (NH + wg) + lane_off;   // buffer 0
     // this row of a P8 tile: K-major, 128-byte swizzle (16-byte chunk c at c ^ (row & 7))
     const uint32_t p_row = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
     const int sw = row & 7;
@@ -340,13 +354,14 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     };
     // S(g) into registers; the MMA issuer may then overwrite the buffer with S(g + 1)
     auto take_s = [&](int g, uint32_t (&sv)[4][32]) -> bool {
-      if (!wwait(bar(B_S_FULL), (uint32_t)g & 1u)) return false;
+      const int b = s_buf(g);
+      if (!wwait(bar(B_S_FULL + b), (uint32_t)s_use(g) & 1u)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem_s + 32 * cc, sv[cc]);
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem_s + 128 * NH * b + 32 * cc, sv[cc]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(B_S_READ));
+      mbar_arrive(bar(B_S_READ + b));
       return true;
     };
     bool ok = true;
