@@ -580,15 +580,15 @@ class Fp8DecodeWorkload(DecodeWorkload):
         return nbytes, time.perf_counter() - t0, f"oracle.attention.decode_fp8 on requests 0..{r - 1} of layer 0 ({r} of {spec.batch} requests, {int(lens[:r].sum())} keys); host copy {prep:.1f}s untimed"
 
 
-WORKLOADS = {
-    "extend_prefix": (3, ExtendWorkload),
-    "decode_fp8_llama3_8b": (6, Fp8DecodeWorkload),
-    "sage_sparse_decode": (7, SageSparseWorkload),
-    "sage_extend_prefix": (8, SageExtendWorkload),
-    "sage_decode": (5, SageWorkload),
-    "decode_llama3_8b": (2, DecodeWorkload),
-    "decode_long_llama3_70b": (4, DecodeWorkload),
-    "decode_tiny": (1, DecodeWorkload),
+WORKLOADS = {   # workload name (workloads.SPECS) -> the step it runs
+    "extend_prefix": ExtendWorkload,
+    "decode_fp8_llama3_8b": Fp8DecodeWorkload,
+    "sage_sparse_decode": SageSparseWorkload,
+    "sage_extend_prefix": SageExtendWorkload,
+    "sage_decode": SageWorkload,
+    "decode_llama3_8b": DecodeWorkload,
+    "decode_long_llama3_70b": DecodeWorkload,
+    "decode_tiny": DecodeWorkload,
 }
 
 
@@ -613,8 +613,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dist = init_ranks(world, local, "gloo" if args.impl == "reference" else "nccl")
 
-    cfg_id, cls = WORKLOADS[args.workload]
-    spec = wl.CONFIGS[cfg_id]
+    cls = WORKLOADS[args.workload]
+    spec = wl.SPECS[args.workload]
     if args.layers:
         spec = spec.scaled(layers=args.layers)
     if args.distinct_pools:

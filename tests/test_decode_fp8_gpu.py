@@ -70,7 +70,7 @@ def check(spec, batch, q, k8, v8, what, **kw):
 
 
 def test_fp8_decode_full_workload():
-    spec = wl.CONFIGS[6]
+    spec = wl.SPECS["decode_fp8_llama3_8b"]
     batch, q, k8, v8 = case(spec)
     check(spec, batch, q, k8, v8, "fp8 full")
 

@@ -136,7 +136,7 @@ def test_extend_and_sage_plans_bit_exact():
 
 
 def test_plan_identical_on_recompute_and_untouched_by_layer_calls():
-    spec = wl.CONFIGS[2].scaled(batch=16, pool_slots=150_000)
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=16, pool_slots=150_000)
     batch, q, k, v = device_case(spec)
     params = decode_params(spec, batch)
     ws = alloc_ws(params)
@@ -182,7 +182,7 @@ def test_gather_bit_exact(P):
 
 
 def test_out_of_range_page_is_skipped_and_reported():
-    spec = wl.CONFIGS[1]
+    spec = wl.SPECS["decode_tiny"]
     batch, q, k, v = device_case(spec)
     params = decode_params(spec, batch)
     ws = alloc_ws(params)
@@ -196,7 +196,7 @@ def test_out_of_range_page_is_skipped_and_reported():
 
 
 def test_wrong_architecture_is_rejected(monkeypatch):
-    spec = wl.CONFIGS[1]
+    spec = wl.SPECS["decode_tiny"]
     batch, q, k, v = device_case(spec)
     params = decode_params(spec, batch)
     ws = alloc_ws(params)
@@ -209,7 +209,7 @@ def test_wrong_architecture_is_rejected(monkeypatch):
 # ---------------------------------------------------------------- decode parity
 
 def test_decode_tiny_config():
-    spec = wl.CONFIGS[1]
+    spec = wl.SPECS["decode_tiny"]
     batch, q, k, v = device_case(spec)
     out, lse, _, _ = run_decode(spec, batch, q, k, v)
     ref, ref_lse = oracle_decode(spec, batch, q, k, v)
@@ -220,7 +220,7 @@ def test_decode_tiny_config():
 @pytest.mark.parametrize("plan_sms", [0, 1, 7])
 def test_decode_llama3_8b_shape_scaled(plan_sms):
     # plan_sms = 1 gives two slots, so each CTA walks many items of several requests
-    spec = wl.CONFIGS[2].scaled(batch=12, pool_slots=120_000)
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=12, pool_slots=120_000)
     batch, q, k, v = device_case(spec)
     out, lse, _, _ = run_decode(spec, batch, q, k, v, plan_sms=plan_sms)
     ref, ref_lse = oracle_decode(spec, batch, q, k, v)
@@ -229,7 +229,7 @@ def test_decode_llama3_8b_shape_scaled(plan_sms):
 
 
 def test_decode_long_context_peaked_scaled():
-    spec = wl.CONFIGS[4].scaled(batch=2, len_lo=20000, len_hi=33000, layers=1, distinct_pools=0)
+    spec = wl.SPECS["decode_long_llama3_70b"].scaled(batch=2, len_lo=20000, len_hi=33000, layers=1, distinct_pools=0)
     batch, q, k, v = device_case(spec)
     out, lse, _, _ = run_decode(spec, batch, q, k, v)
     ref, ref_lse = oracle_decode(spec, batch, q, k, v)
@@ -262,7 +262,7 @@ def test_decode_empty_and_single_key_requests():
 
 
 def test_decode_shuffle_invariance_and_aliased_pages():
-    spec = wl.CONFIGS[2].scaled(batch=4, pool_slots=40_000, len_hi=3000)
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=4, pool_slots=40_000, len_hi=3000)
     batch, q, k, v = device_case(spec)
     out1, lse1, _, _ = run_decode(spec, batch, q, k, v)
     perm = torch.randperm(k.shape[0], generator=torch.Generator().manual_seed(5)).to(DEV)
@@ -284,7 +284,7 @@ def test_decode_shuffle_invariance_and_aliased_pages():
 
 
 def test_decode_full_size_llama3_8b_one_layer():
-    spec = wl.CONFIGS[2]
+    spec = wl.SPECS["decode_llama3_8b"]
     batch, q, k, v = device_case(spec, layer=0)
     out, lse, _, _ = run_decode(spec, batch, q, k, v)
     ref, ref_lse = oracle_decode(spec, batch, q, k, v)
@@ -293,7 +293,7 @@ def test_decode_full_size_llama3_8b_one_layer():
 
 
 def test_decode_full_size_long_context_sampled():
-    spec = wl.CONFIGS[4]
+    spec = wl.SPECS["decode_long_llama3_70b"]
     batch, q, k, v = device_case(spec, layer=0)
     out, lse, _, _ = run_decode(spec, batch, q, k, v)
     # the oracle on a sample of (request, KV head) pairs at full length

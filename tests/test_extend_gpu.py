@@ -138,7 +138,7 @@ def test_extend_with_one_new_token_equals_decode():
 
 
 def test_extend_full_workload_sampled_heads():
-    spec = wl.CONFIGS[3]
+    spec = wl.SPECS["extend_prefix"]
     batch, q, k, v = extend_case(spec)
     out, lse = run_extend(spec, batch, q, k, v)
     heads = [0, 13, 31]

@@ -106,7 +106,7 @@ def test_sage_extend_one_new_token_matches_sage_decode_and_no_v_mean():
 
 
 def test_sage_extend_full_workload_sampled_heads():
-    spec = wl.CONFIGS[8]
+    spec = wl.SPECS["sage_extend_prefix"]
     batch, lay, T = case(spec)
     out = run(spec, batch, lay, T)
     heads = [0, 13, 31]

@@ -55,7 +55,7 @@ def oracle_sage(spec, batch, lay, use_v_mean=True):
 
 
 def test_sage_full_workload():
-    spec = wl.CONFIGS[5]
+    spec = wl.SPECS["sage_decode"]
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     out = run_sage(spec, batch, lay)
@@ -104,7 +104,7 @@ def test_sage_long_rows_split_many_ways():
 def test_sage_few_slots_match_many():
     # a plan for one SM (two CTA slots: long pieces) and the device's full plan give the same
     # quantised probabilities, so both meet the bar
-    spec = wl.CONFIGS[5].scaled(batch=6, len_lo=2000, len_hi=4000)
+    spec = wl.SPECS["sage_decode"].scaled(batch=6, len_lo=2000, len_hi=4000)
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     ref = oracle_sage(spec, batch, lay)
@@ -115,7 +115,7 @@ def test_sage_few_slots_match_many():
 
 
 def test_sage_without_v_mean_and_with_an_empty_row():
-    spec = wl.CONFIGS[5].scaled(batch=5, len_lo=100, len_hi=1500)
+    spec = wl.SPECS["sage_decode"].scaled(batch=5, len_lo=100, len_hi=1500)
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     out = run_sage(spec, batch, lay, use_v_mean=False)
@@ -129,7 +129,7 @@ def test_sage_without_v_mean_and_with_an_empty_row():
 
 
 def test_sage_shuffled_pages_with_their_scales_give_identical_output():
-    spec = wl.CONFIGS[5].scaled(batch=4, len_lo=500, len_hi=2000)
+    spec = wl.SPECS["sage_decode"].scaled(batch=4, len_lo=500, len_hi=2000)
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     out1 = run_sage(spec, batch, lay)
@@ -146,7 +146,7 @@ def test_sage_shuffled_pages_with_their_scales_give_identical_output():
 
 
 def test_sage_requires_sm100(monkeypatch):
-    spec = wl.CONFIGS[5].scaled(batch=2, len_lo=64, len_hi=128)
+    spec = wl.SPECS["sage_decode"].scaled(batch=2, len_lo=64, len_hi=128)
     batch = wl.make_batch(spec, DEV)
     params = sage_params(spec, batch)
     ws = alloc_ws(params)

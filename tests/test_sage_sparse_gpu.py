@@ -89,7 +89,7 @@ def test_sparse_plan_bit_exact():
 
 
 def test_sparse_full_workload_density_0125():
-    spec = wl.CONFIGS[7]
+    spec = wl.SPECS["sage_sparse_decode"]
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     mask = wl.make_block_mask(spec, batch, DEV)
@@ -110,7 +110,7 @@ def test_sparse_small_cases(hq, hkv, lo, hi, density):
 
 
 def test_all_ones_mask_is_bit_identical_to_dense_and_all_zeros_is_v_mean():
-    spec = wl.CONFIGS[5].scaled(batch=8, len_lo=100, len_hi=3000)
+    spec = wl.SPECS["sage_decode"].scaled(batch=8, len_lo=100, len_hi=3000)
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     dense, _, _ = run(spec, batch, lay)

@@ -47,7 +47,7 @@ def test_store_is_bit_exact_and_flags_bad_slots():
 
 
 def _decode_step_case():
-    spec = wl.CONFIGS[2].scaled(batch=8, pool_slots=60_000, len_hi=3000, layers=2)
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=8, pool_slots=60_000, len_hi=3000, layers=2)
     batch = wl.make_batch(spec, DEV)
     pools = [wl.make_bf16_pools(spec, batch, l, DEV) for l in range(spec.layers)]
     # the decode token of every request goes to a fresh (unused, NaN-filled) slot, appended to its row
@@ -155,7 +155,7 @@ def test_sage_store_is_bit_exact_with_block_scales():
 
 def test_sage_store_then_decode_matches_the_oracle():
     from oracle import sage as osg
-    spec = wl.CONFIGS[5].scaled(batch=6, len_lo=100, len_hi=1500)
+    spec = wl.SPECS["sage_decode"].scaled(batch=6, len_lo=100, len_hi=1500)
     batch = wl.make_batch(spec, DEV)
     lay = wl.make_sage_layer(spec, batch, 0, DEV)
     # every request's decode token goes to the first slot of a spare (unused) page, appended

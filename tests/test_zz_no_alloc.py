@@ -43,10 +43,10 @@ def _params(spec, batch):
 
 def test_noalloc_matches_the_workspace_entry_point_on_consecutive_calls():
     cases = []
-    spec = wl.CONFIGS[2].scaled(batch=16, pool_slots=150_000)
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=16, pool_slots=150_000)
     batch = wl.make_batch(spec, DEV)
     cases += [(spec, batch, 0), (spec, batch, 1)]
-    spec2 = wl.CONFIGS[1]                      # a different batch and head layout on the third call
+    spec2 = wl.SPECS["decode_tiny"]                      # a different batch and head layout on the third call
     cases += [(spec2, wl.make_batch(spec2, DEV), 0)]
     for spec, batch, layer in cases:
         params = _params(spec, batch)

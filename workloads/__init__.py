@@ -92,6 +92,9 @@ CONFIGS = {
             page_size=64, spare_pages=0.10, new_lo=128, new_hi=2048, layers=32),
 }
 
+# the workloads by name (the number of each is its seed id)
+SPECS = {s.name: s for s in CONFIGS.values()}
+
 FP8_SCALE = 1.0 / 16.0   # k_scale = v_scale of the FP8 pools
 
 
