@@ -84,3 +84,20 @@ def test_clock_summary_keeps_the_timed_region():
     assert got["samples"] == 1 and got["sm_mhz"] == 1500.0 and got["reasons"] == ["sw_thermal_slowdown"]
     c.lines = []
     assert c.summary()["reasons"] == ["unsampled"]
+
+
+def test_every_bench_workload_is_a_named_spec():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    assert set(bench.WORKLOADS) <= set(wl.SPECS)
+    for name in bench.WORKLOADS:
+        assert wl.SPECS[name].name == name
+    # the seed ids are distinct, so no two workloads draw the same inputs
+    ids = [s.cfg for s in wl.SPECS.values()]
+    assert len(ids) == len(set(ids))
+    # the step class matches the workload's mode
+    modes = {"DecodeWorkload": "decode", "ExtendWorkload": "extend", "SageExtendWorkload": "extend",
+             "SageWorkload": "sage", "SageSparseWorkload": "sage", "Fp8DecodeWorkload": "fp8"}
+    for name, cls in bench.WORKLOADS.items():
+        assert wl.SPECS[name].mode == modes[cls.__name__], name
