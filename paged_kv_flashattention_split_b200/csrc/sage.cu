@@ -176,7 +176,7 @@ __device__ __forceinline__ bool slot_items(const SageLaunch& a, int groups, int&
 // Item metadata of a slot, 32 items at a time, one item per lane; every warp keeps its own
 // window, so no role waits on a chain of dependent reads at an item boundary.
 struct ItemWindow {
-  int w0 = -1 << 30;
+  int w0 = -(1 << 30);
   int r = 0, kv0 = 0, kv1 = 0, base = 0, splits = 0;   // item w0 + lane
   int len = 0, selb = 0;                                // SAGE_SPARSE producer: L_r and sel_base[r]
   __device__ __forceinline__ void load(const SageLaunch& a, int w, int last, bool with_req, bool with_sel = false) {
