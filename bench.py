@@ -51,21 +51,27 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running.
+    """Samples the GPU's SM clock, power and clock-event (throttle) reasons while running.
 
-    Entering waits (up to 5 s) for the first sample, so that the sampler is live before the
-    timed region starts; each line is stamped on arrival, and `mark_start` / `mark_end`
-    bracket the timed region so that the summary keeps the samples taken during it (the
-    first one after its start when it is shorter than the sampling period)."""
+    NVML is polled every 10 ms on a background thread (the GPU found by its UUID, so a
+    CUDA_VISIBLE_DEVICES remapping cannot point it at another board); without NVML,
+    ``nvidia-smi -lms 200`` is the fallback.  `mark_start` / `mark_end` bracket the timed
+    region and the summary keeps only the samples stamped inside it."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []          # (time, sm_mhz, max_mhz, reasons set)
         self.t0 = self.t1 = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
 
     def mark_start(self):
         self.t0 = time.monotonic()
@@ -73,60 +79,91 @@ class ClockSampler:
     def mark_end(self):
         self.t1 = time.monotonic()
 
-    def __enter__(self):
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-            deadline = time.monotonic() + 5.0
-            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
-                time.sleep(0.02)
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
         except Exception:
-            self.proc = None
-        return self
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.monotonic(), line.strip()))
-
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            # a timed region shorter than the period: wait (up to 1 s) for the sample after it
-            deadline = time.monotonic() + 1.0
-            while (self.t0 is not None and not any(x[0] >= self.t0 for x in list(self.lines))
-                   and time.monotonic() < deadline and self.proc.poll() is None):
-                time.sleep(0.02)
-            self.proc.terminate()
+    def _poll_nvml(self, nv, h):
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
             try:
-                self.proc.wait(timeout=5)
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.monotonic(), float(sm), float(mx),
+                                     {n for n, b in self.REASONS if bits & b}))
             except Exception:
-                self.proc.kill()
+                pass
+            time.sleep(self.period)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = list(self.lines)
-        if self.t0 is not None and self.t1 is not None:
-            inside = [x for x in lines if self.t0 <= x[0] <= self.t1]
-            # a region shorter than the period: the first sample after its start
-            lines = inside or [x for x in lines if x[0] >= self.t0][:1]
-        for _, line in lines:
-            parts = [p.strip() for p in line.split(",")]
+    def _poll_smi(self):
+        for line in self._proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            self.samples.append((time.monotonic(), sm, mx,
+                                 {n for (n, _), v in zip(self.REASONS, parts[5:9]) if v.lower() == "active"}))
+
+    def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self._thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml 10 ms"
+        except Exception:
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.cuda_index), "--query-gpu=" + self.FIELDS,
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._thread = threading.Thread(target=self._poll_smi, daemon=True)
+                self.source = "nvidia-smi 200 ms"
+            except Exception:
+                self._thread = None
+        if self._thread is not None:
+            self._thread.start()
+            deadline = time.monotonic() + 5.0
+            while not self.samples and time.monotonic() < deadline:
+                time.sleep(0.005)
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._proc is not None:
+            # a region shorter than the 200 ms period: wait (up to 1 s) for one sample after its start
+            deadline = time.monotonic() + 1.0
+            while (self.t0 is not None and not any(x[0] >= self.t0 for x in list(self.samples))
+                   and time.monotonic() < deadline):
+                time.sleep(0.02)
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self):
+        samples = list(self.samples)
+        where = "in_region"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [x for x in samples if self.t0 <= x[0] <= self.t1]
+            if not inside:
+                inside, where = [x for x in samples if x[0] >= self.t0][:1], "post_region"
+            samples = inside
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
+        reasons = set().union(*(x[3] for x in samples))
+        return {"sm_mhz": statistics.median(x[1] for x in samples), "sm_max_mhz": samples[-1][2],
+                "reasons": sorted(reasons), "samples": len(samples), "window": where, "source": self.source}
 
 
 # The sources each workload's kernels are built from; profiles/traffic.json is keyed by their hash,
@@ -594,45 +631,30 @@ WORKLOADS = {   # workload name (workloads.SPECS) -> the step it runs
 
 # --------------------------------------------------------------------------- main
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_llama3_8b", choices=sorted(WORKLOADS))
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--layers", type=int, default=0,
-                    help="profiling only: fewer layer calls per step than the workload defines")
-    ap.add_argument("--distinct-pools", type=int, default=0,
-                    help="profiling only: allocate fewer pools (layers rotate over them)")
-    args = ap.parse_args()
+DTYPES = {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
+          "sage_sparse_decode": "int8/e4m3 in, fp32 math, bf16 out",
+          "sage_extend_prefix": "int8 x int8 -> int32 (QK) and e4m3 x e4m3 -> fp32 (PV) tensor-core math, bf16 out",
+          "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}
+STEP_CALLS = {"sage_decode": "attn_decode_paged_sage", "sage_sparse_decode": "attn_decode_paged_sage (block-sparse plan)",
+              "sage_extend_prefix": "attn_extend_paged_sage", "extend_prefix": "attn_extend_paged",
+              "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}
+ROOFLINE_KERNELS = {
+    "sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
+    "sage_sparse_decode": "attn_decode_paged_sage call, block-sparse plan (score + value + merge kernels)",
+    "sage_extend_prefix": "sage_extend_kernel (one launch per attn_extend_paged_sage call; 3 contractions per tile pair, 2 counted)",
+    "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
+    "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}
+# workloads measured beside the default decode in the default run (the other halves of the metric)
+DEFAULT_EXTRAS = ("extend_prefix", "sage_decode")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = init_ranks(world, local, "gloo" if args.impl == "reference" else "nccl")
 
-    cls = WORKLOADS[args.workload]
-    spec = wl.SPECS[args.workload]
-    if args.layers:
-        spec = spec.scaled(layers=args.layers)
-    if args.distinct_pools:
-        spec = spec.scaled(distinct_pools=args.distinct_pools)
-    hbm_peak, bf16_peak, bf16_sus, peak_src = load_peaks()
-
-    if args.impl == "reference":
-        if rank != 0:
-            if dist is not None:
-                dist.destroy_process_group()
-            return
-        run_reference(args, spec, cls)
-        if dist is not None:
-            dist.destroy_process_group()
-        return
-
+def measure(name, spec, args, dist, world, local, rank, peaks, cpu_baseline=True):
+    """Run one workload: warm-up, the timed steps (CUDA events, max over ranks), the CUDA-graph replay,
+    the end-to-end run through host buffers, and (rank 0, one GPU) the oracle on a bounded sample.
+    Returns the JSON fields of that workload."""
+    hbm_peak, bf16_peak, bf16_sus, peak_src = peaks
+    cls = WORKLOADS[name]
     dev = f"cuda:{local}"
-    torch.cuda.set_device(dev)
     work = cls(spec, dev)
     torch.cuda.synchronize()
 
@@ -640,9 +662,8 @@ def main():
         work.step()
     torch.cuda.synchronize()
 
-    # timed region: events on the launching stream, per-layer events for the decode call
+    # timed region: events on the launching stream, per-layer events for the layer call
     layer_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(spec.layers)]
-    layer_ms = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
@@ -650,7 +671,7 @@ def main():
     with ClockSampler(local) as clocks:
         clocks.mark_start()
         start.record()
-        for s in range(args.steps):
+        for _ in range(args.steps):
             work.step(layer_events)
         end.record()
         torch.cuda.synchronize()
@@ -665,7 +686,6 @@ def main():
     value = job_throughput(work.step_bytes, world, ms_per_step, scale)
 
     # the same step captured once in a CUDA graph and replayed (launch overhead removed)
-    graph_info = None
     try:
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
@@ -684,7 +704,7 @@ def main():
         g1.record()
         torch.cuda.synchronize()
         g_ms = max_over_ranks(dist, g0.elapsed_time(g1) / args.steps, dev)
-        graph_info = {"ms_per_step": round(g_ms, 4), "value": round(job_throughput(work.step_bytes, world, g_ms, getattr(work, "scale", 1e9)), 1)}
+        graph_info = {"ms_per_step": round(g_ms, 4), "value": round(job_throughput(work.step_bytes, world, g_ms, scale), 1)}
         del graph
     except Exception as exc:  # reported, never silently replaced
         graph_info = {"error": str(exc)[:200]}
@@ -706,19 +726,19 @@ def main():
 
     avg_layer_ms = float(np.mean(layer_ms)) if layer_ms else ms_per_step / spec.layers
     achieved = work.layer_bytes / (avg_layer_ms * 1e-3) / scale
-    kernel_src = KERNEL_SOURCES.get(args.workload, KERNEL_SOURCES["decode_llama3_8b"])
-    traffic = recorded_traffic(args.workload, source_hash(*kernel_src))
+    kernel_src = KERNEL_SOURCES.get(name, KERNEL_SOURCES["decode_llama3_8b"])
+    traffic = recorded_traffic(name, source_hash(*kernel_src))
     unit = getattr(work, "unit", "GB/s")
-    if unit == "TFLOP/s" and args.workload == "sage_extend_prefix":
+    if unit == "TFLOP/s" and name == "sage_extend_prefix":
         # int8 and e4m3 contractions: the 8-bit dense peak, 2x the measured bf16 one (the nominal ratio)
-        bound, peak, peak_note = "tensor", round(2.0 * bf16_sus, 1), peak_src + (
-            " sustained bf16 dense x 2 (8-bit dense = 2x bf16 nominal), kernel timed inside a long step")
+        bound, peak, peak_note = "tensor", round(2.0 * bf16_peak, 1), peak_src + (
+            " burst bf16 dense x 2 (8-bit dense = 2x bf16 nominal): the kernel runs in a sub-second region")
     elif unit == "TFLOP/s":
-        bound, peak, peak_note = "tensor", bf16_sus, peak_src + " (sustained bf16 dense, kernel timed inside a long step)"
+        bound, peak, peak_note = "tensor", bf16_peak, peak_src + " burst bf16 dense (the kernel runs in a sub-second region)"
     else:
         bound, peak, peak_note = "hbm", hbm_peak, peak_src
 
-    line = {
+    out = {
         "metric": METRIC,
         "value": round(value, 1),
         "unit": unit,
@@ -729,35 +749,21 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
-                  "sage_sparse_decode": "int8/e4m3 in, fp32 math, bf16 out",
-                  "sage_extend_prefix": "int8 x int8 -> int32 (QK) and e4m3 x e4m3 -> fp32 (PV) tensor-core math, bf16 out",
-                  "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}.get(
-                      args.workload, "bf16"),
+        "dtype": DTYPES.get(name, "bf16"),
         "data": "synthetic",
         "config": {
-            "workload": args.workload,
+            "workload": name,
             "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
             "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
             "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
-            "step": "attn_plan + %d x %s" % (spec.layers, {"sage_decode": "attn_decode_paged_sage",
-                                                            "sage_sparse_decode": "attn_decode_paged_sage (block-sparse plan)",
-                                                            "sage_extend_prefix": "attn_extend_paged_sage",
-                                                            "extend_prefix": "attn_extend_paged",
-                                                            "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}.get(
-                                                               args.workload, "attn_decode_paged")),
-            "l2": "inputs larger than L2 (each layer reads its own >1 GB pool)",
+            "step": "attn_plan + %d x %s" % (spec.layers, STEP_CALLS.get(name, "attn_decode_paged")),
+            "l2": "inputs larger than L2 (the step's layers read their own pools, far more than L2)",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
             "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": {"sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
-                       "sage_sparse_decode": "attn_decode_paged_sage call, block-sparse plan (score + value + merge kernels)",
-                       "sage_extend_prefix": "sage_extend_kernel (one launch per attn_extend_paged_sage call; 3 contractions per tile pair, 2 counted)",
-                       "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
-                       "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}.get(
-                           args.workload, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
+            "kernel": ROOFLINE_KERNELS.get(name, "attn_decode_paged call (decode_splitkv_kernel + merge_kernel)")
                       + ", per-layer CUDA events",
             "peak_source": peak_note,
         },
@@ -767,10 +773,71 @@ def main():
         "graph": graph_info,
         "clocks": clocks.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if spec.mode == "extend":
+        out["config"]["new_lens"] = f"U[{spec.new_lo},{spec.new_hi}]"
+    if cpu_baseline and rank == 0 and world == 1:
         nbytes, secs, sample = work.oracle_sample()
-        line["cpu_baseline"] = {"value": round(nbytes / secs / scale, 6), "unit": unit, "cores": blas_threads(),
-                                "kind": "oracle", "sample": sample}
+        out["cpu_baseline"] = {"value": round(nbytes / secs / scale, 6), "unit": unit, "cores": blas_threads(),
+                               "kind": "oracle", "sample": sample}
+    del work
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_llama3_8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload only: skip the extend and Sage decode objects")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: fewer layer calls per step than the workload defines")
+    ap.add_argument("--distinct-pools", type=int, default=0,
+                    help="profiling only: allocate fewer pools (layers rotate over them)")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = init_ranks(world, local, "gloo" if args.impl == "reference" else "nccl")
+
+    def spec_for(name):
+        spec = wl.SPECS[name]
+        if args.layers:
+            spec = spec.scaled(layers=args.layers)
+        if args.distinct_pools:
+            spec = spec.scaled(distinct_pools=args.distinct_pools)
+        return spec
+
+    spec = spec_for(args.workload)
+    peaks = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            if dist is not None:
+                dist.destroy_process_group()
+            return
+        run_reference(args, spec, WORKLOADS[args.workload])
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    torch.cuda.set_device(f"cuda:{local}")
+    line = measure(args.workload, spec, args, dist, world, local, rank, peaks, not args.no_cpu_baseline)
+    # the default run also measures the extend half of the metric and the 8-bit Sage decode, each
+    # in its own timed region with its own clocks (the decode's pools are freed first)
+    if args.workload == "decode_llama3_8b" and not args.no_extras:
+        for name in DEFAULT_EXTRAS:
+            key = "extend" if name == "extend_prefix" else name
+            line[key] = measure(name, spec_for(name), args, dist, world, local, rank, peaks,
+                                not args.no_cpu_baseline)
+            for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):
+                line[key].pop(k, None)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -336,15 +336,28 @@ pa_status attn_extend_paged_sage(const pa_plan_params* params, const void* d_ws,
  * the array's device address (once per device, with that device current); make
  * that first call before any stream capture.  All calls share the array and it
  * keeps the last call's contents: calls that overlap on the GPU (other streams
- * or host threads) race and must be ordered by the caller.  Device-side errors
- * are recorded in the array's header and are not readable through
- * pa_read_device_error, which needs a workspace pointer.
+ * or host threads) race and must be ordered by the caller.  The device address
+ * is kept for the life of the process: after cudaDeviceReset (or anything else
+ * that destroys the device's primary context) this entry point must not be
+ * called again in that process.  Device-side errors (an out-of-range page id, a
+ * length beyond max_kv_len) are recorded in the array's header: read and clear
+ * them with pa_noalloc_read_device_error.
  */
 pa_status attn_decode_paged_noalloc(const pa_plan_params* params, const int32_t* d_seq_lens,
                                     const uint16_t* d_q, const uint16_t* d_k_pool,
                                     const uint16_t* d_v_pool, int64_t num_slots,
                                     const int32_t* d_page_table, int64_t pt_pitch, float sm_scale,
                                     uint16_t* d_out, float* d_lse_out, pa_stream_t stream);
+
+/*
+ * pa_noalloc_read_device_error - pa_read_device_error for attn_decode_paged_noalloc:
+ * synchronise `stream`, read the device error word of the library's fixed
+ * workspace array on the current device and clear it.  Returns PA_OK if clean,
+ * PA_ERR_DEVICE_INDEX if the last calls met an out-of-range slot or page id or
+ * length, PA_ERR_WORKSPACE if no no-allocation plan has been made on this device,
+ * PA_ERR_CUDA on a CUDA error.  Allocates nothing.  (No counterpart on the pages.)
+ */
+pa_status pa_noalloc_read_device_error(pa_stream_t stream);
 
 /*
  * attn_kv_store - write the K and V rows of new tokens into their pool slots: the cache

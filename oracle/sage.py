@@ -54,19 +54,36 @@ def sage_scores_f32(q8_row: np.ndarray, k8_rows: np.ndarray, sf_q: float, sf_k_r
     return (scale * dot.astype(np.float32)).astype(np.float32)        # fp32 product, rounded
 
 
-def sage_row(q8_row, k8_rows, v8_rows, sf_q, sf_k_rows, sf_v, v_mean, quantize_p: bool = True):
+def sage_scores_f64(q8_row: np.ndarray, k8_rows: np.ndarray, sf_q: float, sf_k_rows: np.ndarray) -> np.ndarray:
+    """S for one query row over keys with every step in float64: sfQ * sfK * (exact int dot).
+
+    The literal formula without the float32 reading; used to show that the precision in
+    which S is formed does not move the result beyond rounding.  Returns float64 [N].
+    """
+    dot = k8_rows.astype(np.int64) @ q8_row.astype(np.int64)
+    return np.float64(sf_q) * sf_k_rows.astype(np.float64) * dot.astype(np.float64)
+
+
+def sage_row(q8_row, k8_rows, v8_rows, sf_q, sf_k_rows, sf_v, v_mean, quantize_p: bool = True,
+             score_f64: bool = False):
     """The Sage formula for one query row; returns O [D] float64.
 
     v8_rows [N, D] uint8 E4M3 codes, sf_v and v_mean [D].  ``quantize_p=False``
     replaces the E4M3 step on 448 * p by the identity (a switch used to tie
-    this function to plain softmax attention in the tests).
+    this function to plain softmax attention in the tests).  ``score_f64=True``
+    forms S and its row max in float64 instead of the kernel's float32 (the
+    reading above), to measure what that reading moves.
     """
     D = v8_rows.shape[1] if v8_rows.ndim == 2 else len(sf_v)
     vm = np.zeros(D) if v_mean is None else np.asarray(v_mean, dtype=np.float64)
     if k8_rows.shape[0] == 0:
         return vm.copy()
-    S = sage_scores_f32(q8_row, k8_rows, sf_q, sf_k_rows)             # step 1: scores
-    m = np.float32(S.max())                                           # step 2: row max (fp32)
+    if score_f64:
+        S = sage_scores_f64(q8_row, k8_rows, sf_q, sf_k_rows)         # step 1: scores (fp64)
+        m = S.max()                                                   # step 2: row max (fp64)
+    else:
+        S = sage_scores_f32(q8_row, k8_rows, sf_q, sf_k_rows)         # step 1: scores
+        m = np.float32(S.max())                                       # step 2: row max (fp32)
     p = np.exp(S.astype(np.float64) - np.float64(m))                  # step 3: exp(S - m) in (0, 1]
     l = p.sum()                                                       # unquantised row sum
     if quantize_p:
@@ -93,7 +110,8 @@ def selected_positions(seq_len: int, mask_row, k_block: int = 64) -> np.ndarray:
 
 
 def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_lens,
-                page_size: int, k_block: int = 64, quantize_p: bool = True, block_mask=None) -> np.ndarray:
+                page_size: int, k_block: int = 64, quantize_p: bool = True, block_mask=None,
+                score_f64: bool = False) -> np.ndarray:
     """Sage DECODE over the paged cache; returns O [B, Hq, D] float64.
 
     Keys are gathered through the page table exactly as in the bf16 path
@@ -102,6 +120,7 @@ def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_
     With ``block_mask`` [B][n_blocks] (block-sparse mode), row r attends only to the keys
     of its selected blocks (``selected_positions``): the Sage formula, row max and row
     sum included, over that subset; a row with no selected key gives v_mean.
+    ``score_f64`` as for ``sage_row``.
     """
     B, Hq, D = q8.shape
     Hkv = k8_pool.shape[1]
@@ -119,7 +138,7 @@ def sage_decode(q8, sf_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_
             sfk = sf_k[blocks, hk]
             vm = None if v_mean is None else v_mean[hk]
             for h in range(hk * G, (hk + 1) * G):
-                out[r, h] = sage_row(q8[r, h], k8, v8, sf_q[r, h], sfk, sf_v[hk], vm, quantize_p)
+                out[r, h] = sage_row(q8[r, h], k8, v8, sf_q[r, h], sfk, sf_v[hk], vm, quantize_p, score_f64)
     return out
 
 
@@ -149,7 +168,7 @@ def kv_store_sage(k8_pool, v8_pool, sf_k, out_cache_loc, k8_new, v8_new, sf_k_ne
 
 
 def sage_extend(q8, sf_q, cu_seqlens_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, page_table, seq_lens,
-                page_size: int, k_block: int = 64) -> np.ndarray:
+                page_size: int, k_block: int = 64, heads=None) -> np.ndarray:
     """Sage EXTEND (prefill over a cached prefix); returns O [T, Hq, D] float64.
 
     The Sage formula of ``sage_row`` for every new token: row i of request r (Q8 row
@@ -158,24 +177,42 @@ def sage_extend(q8, sf_q, cu_seqlens_q, k8_pool, v8_pool, sf_k, sf_v, v_mean, pa
     of ``oracle.attention.extend``); its row max and row sum run over those keys.  This
     is the variant the pages measure at S = 10800 ("FlashInfer PrimTS, Sage Attention ...",
     performance item 2); the kernel for it runs on the prefill path.
+
+    The rows of one request and head are taken together as an [n, L] block with a
+    visibility mask, each element through the same steps as ``sage_row`` (exact integer
+    dot, float32 S and row max, float64 exp, E4M3(448 p), the unquantised row sum, the
+    epilogue); only the order in which the float64 sums add their terms differs.  The
+    integer dots run as float64 products, which are exact (every partial sum is an
+    integer below 2**22).  ``heads`` restricts the query heads computed (the others are 0).
     """
     T, Hq, D = q8.shape
     Hkv = k8_pool.shape[1]
     G = Hq // Hkv
     out = np.zeros((T, Hq, D))
+    heads = range(Hq) if heads is None else heads
     for r in range(len(seq_lens)):
         q0, q1 = int(cu_seqlens_q[r]), int(cu_seqlens_q[r + 1])
+        n = q1 - q0
+        if n == 0:
+            continue
         L = int(seq_lens[r])
-        p = L - (q1 - q0)
+        p = L - n
         slots = gather_slots(page_table, L, page_size, r)
         blocks = slots // k_block
-        for hk in range(Hkv):
-            vm = None if v_mean is None else v_mean[hk]
-            for i in range(q1 - q0):
-                vis = slots[: p + i + 1]
-                k8 = k8_pool[vis, hk, :]
-                v8 = v8_pool[vis, hk, :]
-                sfk = sf_k[blocks[: p + i + 1], hk]
-                for h in range(hk * G, (hk + 1) * G):
-                    out[q0 + i, h] = sage_row(q8[q0 + i, h], k8, v8, sf_q[q0 + i, h], sfk, sf_v[hk], vm)
+        visible = np.arange(L)[None, :] <= (p + np.arange(n))[:, None]      # [n, L]
+        for h in heads:
+            hk = h // G
+            k8 = k8_pool[slots, hk, :].astype(np.float64)                    # [L, D]
+            V = e4m3_to_f64(v8_pool[slots, hk, :])                           # [L, D]
+            dot = q8[q0:q1, h, :].astype(np.float64) @ k8.T                  # exact integers [n, L]
+            scale = sf_q[q0:q1, h].astype(np.float32)[:, None] * sf_k[blocks, hk].astype(np.float32)[None, :]
+            S = (scale * dot.astype(np.float32)).astype(np.float32)          # step 1 (fp32 products)
+            S = np.where(visible, S, np.float32(-np.inf))
+            m = S.max(axis=1)                                                # step 2: fp32 row max
+            pr = np.where(visible, np.exp(S.astype(np.float64) - m.astype(np.float64)[:, None]), 0.0)
+            l = pr.sum(axis=1)                                               # step 3: unquantised l
+            P = e4m3_to_f64(f64_to_e4m3(448.0 * pr))                         # step 4: E4M3(448 p)
+            acc = P @ V                                                      # step 5
+            vm = np.zeros(D) if v_mean is None else np.asarray(v_mean[hk], dtype=np.float64)
+            out[q0:q1, h] = np.asarray(sf_v[hk], dtype=np.float64) * acc / (448.0 * l[:, None]) + vm   # step 6
     return out

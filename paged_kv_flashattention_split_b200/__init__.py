@@ -34,6 +34,7 @@ from ._binding import (  # noqa: F401
     lib,
     make_params,
     pa_plan_params,
+    pa_noalloc_read_device_error,
     pa_plan_workspace_size,
     pa_read_device_error,
     pa_version,

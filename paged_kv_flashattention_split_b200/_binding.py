@@ -22,7 +22,8 @@ PA_MODE_DECODE, PA_MODE_EXTEND, PA_MODE_SAGE_DECODE, PA_MODE_SAGE_SPARSE = 0, 1,
 EXPORTED = ("pa_plan_workspace_size", "attn_plan", "attn_decode_paged", "attn_extend_paged",
             "attn_decode_paged_sage", "attn_debug_gather", "pa_read_device_error",
             "pa_status_string", "pa_version", "attn_decode_paged_noalloc", "attn_kv_store",
-            "attn_kv_store_sage", "attn_decode_paged_fp8", "attn_plan_sage_sparse", "attn_extend_paged_sage")
+            "attn_kv_store_sage", "attn_decode_paged_fp8", "attn_plan_sage_sparse", "attn_extend_paged_sage",
+            "pa_noalloc_read_device_error")
 
 
 class pa_plan_params(ctypes.Structure):
@@ -66,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "attn_debug_gather": (_I32, [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _I64, _P, _I64,
                                          _P, _P, _P]),
             "pa_read_device_error": (_I32, [_P, _P]),
+            "pa_noalloc_read_device_error": (_I32, [_P]),
             "attn_kv_store": (_I32, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I64, _P, _P]),
             "attn_kv_store_sage": (_I32, [_P, _P, _P, _P, _I64, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
             "attn_decode_paged_noalloc": (_I32, [PP, _P, _P, _P, _P, _I64, _P, _I64, _F32, _P, _P, _P]),
@@ -241,6 +243,11 @@ def attn_kv_store_sage(k8_new, v8_new, sf_k_new, out_cache_loc, k8_pool, v8_pool
 
 def pa_read_device_error(ws, stream=None) -> int:
     return lib().pa_read_device_error(_ptr(ws), _stream(stream))
+
+
+def pa_noalloc_read_device_error(stream=None) -> int:
+    """Read and clear the device error word of attn_decode_paged_noalloc's fixed array."""
+    return lib().pa_noalloc_read_device_error(_stream(stream))
 
 
 def pa_version() -> int:

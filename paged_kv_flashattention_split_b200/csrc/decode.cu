@@ -343,17 +343,11 @@ __global__ void debug_gather_kernel(GatherLaunch a) {
 
 template <int HG, int G>
 cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<HG, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kDecodeSmem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> smem_set[kMaxDevices];
+  cudaError_t e = raise_smem_limit(decode_splitkv_kernel<HG, G>, kDecodeSmem, smem_set);
+  if (e != cudaSuccess) return e;
   decode_splitkv_kernel<HG, G><<<a.slots * (a.hkv / HG), kThreads, kDecodeSmem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_merge(a, s);
 }

@@ -319,16 +319,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fp8_kernel(Fp8DecodeLaunch
 
 template <int HG, int G>
 cudaError_t launch_fp8_hg(const Fp8DecodeLaunch& a, cudaStream_t s) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_fp8_kernel<HG, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> smem_set[kMaxDevices];
+  cudaError_t e = raise_smem_limit(decode_fp8_kernel<HG, G>, kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   decode_fp8_kernel<HG, G><<<a.slots * (a.hkv / HG), kThreads, kSmem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecodeLaunch m{};
   m.ws = a.ws;

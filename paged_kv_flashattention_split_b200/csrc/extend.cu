@@ -804,14 +804,7 @@ bool encode_rows(CUtensorMap* tm, const void* ptr, int64_t rows, int heads, int 
 }  // namespace
 
 cudaError_t launch_extend(const ExtendArgs& in, cudaStream_t s) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> single_set[kMaxDevices], pair_set[kMaxDevices];
   ExtendLaunch a;
   const int box_rows = in.page_size < kTileKeys ? in.page_size : kTileKeys;
   if (!encode_rows(&a.tm_q, in.q, in.q_rows, in.hq, 128) ||
@@ -833,15 +826,12 @@ cudaError_t launch_extend(const ExtendArgs& in, cudaStream_t s) {
   a.max_items = in.max_items;
   a.q_rows = in.q_rows;
   if ((in.hq / in.hkv) % 2 == 0) {   // two heads of one KV group per CTA
-    static bool pair_attr[64] = {};
-    if (dev < 64 && !pair_attr[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(extend_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kPairSmemBytes);
-      if (e != cudaSuccess) return e;
-      pair_attr[dev] = true;
-    }
+    cudaError_t e = raise_smem_limit(extend_pair_kernel, kPairSmemBytes, pair_set);
+    if (e != cudaSuccess) return e;
     extend_pair_kernel<<<in.max_items * (in.hq / 2), kPairThreads, kPairSmemBytes, s>>>(a);
   } else {
+    cudaError_t e = raise_smem_limit(extend_kernel, kSmemBytes, single_set);
+    if (e != cudaSuccess) return e;
     extend_kernel<<<in.max_items * in.hq, kThreads, kSmemBytes, s>>>(a);
   }
   return cudaGetLastError();

@@ -1,9 +1,28 @@
 // kernels.h - host-side launchers implemented by the .cu files (internal).
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace pa {
+
+constexpr int kMaxDevices = 64;
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device.  Host threads may launch at the same time: the per-device flags are atomic, and
+// setting the attribute twice is harmless.  Devices beyond kMaxDevices set it on every call.
+template <typename K>
+cudaError_t raise_smem_limit(K kernel, int bytes, std::atomic<bool>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 struct PlanLaunch {
   WsView ws;

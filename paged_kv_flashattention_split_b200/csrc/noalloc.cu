@@ -67,3 +67,12 @@ extern "C" pa_status attn_decode_paged_noalloc(const pa_plan_params* params, con
   return attn_decode_paged(params, ws, kNoAllocBytes, d_q, d_k_pool, d_v_pool, num_slots, d_page_table,
                            pt_pitch, sm_scale, d_out, d_lse_out, stream);
 }
+
+// The error word of the fixed array's plan header: the no-allocation decode's own
+// pa_read_device_error (the caller has no workspace pointer to pass to that one).
+extern "C" pa_status pa_noalloc_read_device_error(pa_stream_t stream) {
+  void* ws = nullptr;
+  pa_status st = noalloc_workspace(&ws);
+  if (st != PA_OK) return st;
+  return pa_read_device_error(ws, stream);
+}

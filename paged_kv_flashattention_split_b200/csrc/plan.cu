@@ -285,15 +285,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
 
 cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s) {
   const size_t smem = sizeof(unsigned long long) * (size_t)a.sort_n;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(sizeof(unsigned long long) * kMaxSortItems));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> smem_set[kMaxDevices];
+  cudaError_t e = raise_smem_limit(plan_kernel, (int)(sizeof(unsigned long long) * kMaxSortItems), smem_set);
+  if (e != cudaSuccess) return e;
   plan_kernel<<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -755,17 +755,10 @@ template <int HG, int G>
 cudaError_t launch_sage_hg(SageLaunch& a, const int8_t* k8, const uint8_t* v8, int slots, cudaStream_t s) {
   using LS = SageSmem<HG, G, false>;
   using LV = SageSmem<HG, G, true>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sage_score_kernel<HG, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         LS::BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(sage_value_kernel<HG, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, LV::BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> score_set[kMaxDevices], value_set[kMaxDevices];
+  cudaError_t e0 = raise_smem_limit(sage_score_kernel<HG, G>, LS::BYTES, score_set);
+  if (e0 == cudaSuccess) e0 = raise_smem_limit(sage_value_kernel<HG, G>, LV::BYTES, value_set);
+  if (e0 != cudaSuccess) return e0;
   const dim3 grid(slots * (a.hkv / HG));
   if (!encode_scores(&a.tm_s, a.ws.scores, a.ws.score_pitch, (int64_t)a.batch * a.hq, HG * G) ||
       !encode_pool(&a.tm_kv, k8, a.num_slots, a.hkv, HG) ||

@@ -526,17 +526,10 @@ bool encode_rows8(CUtensorMap* tm, const void* ptr, int64_t rows, int heads, int
 }  // namespace
 
 cudaError_t launch_sage_extend(const SageExtendArgs& in, cudaStream_t s) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sage_extend_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<1>::kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(sage_extend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<2>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> one_set[kMaxDevices], two_set[kMaxDevices];
+  cudaError_t e0 = raise_smem_limit(sage_extend_kernel<1>, Cfg<1>::kSmemBytes, one_set);
+  if (e0 == cudaSuccess) e0 = raise_smem_limit(sage_extend_kernel<2>, Cfg<2>::kSmemBytes, two_set);
+  if (e0 != cudaSuccess) return e0;
   SageExtendLaunch a;
   if (!encode_rows8(&a.tm_q8, in.q8, in.q_rows, in.hq, 128) ||
       !encode_rows8(&a.tm_k8, in.k8, in.num_slots, in.hkv, kSageBlock) ||

@@ -43,8 +43,9 @@ __global__ void __launch_bounds__(256) kv_store_kernel(StoreLaunch a) {
 cudaError_t launch_kv_store(const StoreLaunch& a, cudaStream_t s) {
   const int64_t total = a.n_tokens * a.hkv * kHeadDim * a.elem_bytes / 16;
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   const int64_t want = (total + 255) / 256;
   const int blocks = (int)(want < (int64_t)sms * 8 ? (want > 0 ? want : 1) : (int64_t)sms * 8);
   kv_store_kernel<<<blocks, 256, 0, s>>>(a);

@@ -47,16 +47,16 @@ def oracle_fp8(spec, batch, q, k8, v8, ks=wl.FP8_SCALE, vs=wl.FP8_SCALE):
                          batch.seq_lens.cpu().numpy(), spec.page_size, spec.sm_scale)
 
 
-def case(spec, peaked=False):
+def case(spec, peaked=False, layer=0):
     batch = wl.make_batch(spec, DEV)
-    k8, v8 = wl.make_fp8_pools(spec, batch, 0, DEV)
+    k8, v8 = wl.make_fp8_pools(spec, batch, layer, DEV)
     if peaked:   # 2% of the (slot, head) K rows scaled by 8 (still within E4M3's range: clamp)
         g = torch.Generator(device=DEV).manual_seed(44)
         sel = torch.rand(k8.shape[:2], generator=g, device=DEV) < 0.02
         kf = k8.view(torch.float8_e4m3fn).float()
         kf = torch.where(sel[..., None], (kf * 8).clamp(-448, 448), kf)
         k8 = torch.where(sel[..., None], kf.to(torch.float8_e4m3fn).view(torch.uint8), k8)
-    q = wl.make_bf16_queries(spec, spec.batch, 0, DEV)
+    q = wl.make_bf16_queries(spec, spec.batch, layer, DEV)
     return batch, q, k8, v8
 
 
@@ -69,9 +69,11 @@ def check(spec, batch, q, k8, v8, what, **kw):
     assert np.all(np.isneginf(g[~fin])) and np.max(np.abs(g[fin] - ref_lse[fin]), initial=0.0) <= LSE_ABS
 
 
-def test_fp8_decode_full_workload():
+@pytest.mark.parametrize("layer", [0, 31])
+def test_fp8_decode_full_workload(layer):
+    """Every output element of the first and the last layer of the FP8-KV decode workload."""
     spec = wl.SPECS["decode_fp8_llama3_8b"]
-    batch, q, k8, v8 = case(spec)
+    batch, q, k8, v8 = case(spec, layer=layer)
     check(spec, batch, q, k8, v8, "fp8 full")
 
 

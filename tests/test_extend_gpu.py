@@ -56,23 +56,8 @@ def run_extend(spec, batch, q, k, v):
     return out, lse
 
 
-def oracle_extend(spec, batch, q, k, v, heads=None):
-    qb, kb, vb = bits16(q), bits16(k), bits16(v)
-    if heads is not None:                       # the oracle on a subset of query heads (with their KV heads)
-        G = spec.hq // spec.hkv
-        hk = sorted({h // G for h in heads})
-        qsel = np.stack([qb[:, h] for h in heads], axis=1)
-        kmap = [hk.index(h // G) for h in heads]
-        o, l = [], []
-        for i, h in enumerate(heads):
-            oi, li = oa.extend(qsel[:, i:i + 1], batch.cu_seqlens_q.cpu().numpy(), kb[:, h // G:h // G + 1],
-                               vb[:, h // G:h // G + 1], batch.page_table.cpu().numpy(),
-                               batch.seq_lens.cpu().numpy(), spec.page_size, spec.sm_scale)
-            o.append(oi[:, 0])
-            l.append(li[:, 0])
-        del kmap
-        return np.stack(o, axis=1), np.stack(l, axis=1)
-    return oa.extend(qb, batch.cu_seqlens_q.cpu().numpy(), kb, vb, batch.page_table.cpu().numpy(),
+def oracle_extend(spec, batch, q, k, v):
+    return oa.extend(bits16(q), batch.cu_seqlens_q.cpu().numpy(), bits16(k), bits16(v), batch.page_table.cpu().numpy(),
                      batch.seq_lens.cpu().numpy(), spec.page_size, spec.sm_scale)
 
 
@@ -137,11 +122,16 @@ def test_extend_with_one_new_token_equals_decode():
     assert_bf16_close(out, bf16_bits_to_f64(bits16(dout)), "extend n=1 vs decode")
 
 
-def test_extend_full_workload_sampled_heads():
+@pytest.mark.parametrize("layer", [0, 31])
+def test_extend_full_workload(layer):
+    """Every output element and LSE, all 32 query heads, of the first and the last layer of the
+    extend workload (the oracle's heads spread over a process pool)."""
+    from tests import oracle_jobs
     spec = wl.SPECS["extend_prefix"]
-    batch, q, k, v = extend_case(spec)
+    batch, q, k, v = extend_case(spec, layer=layer)
     out, lse = run_extend(spec, batch, q, k, v)
-    heads = [0, 13, 31]
-    ref, ref_lse = oracle_extend(spec, batch, q, k, v, heads=heads)
-    assert_bf16_close(out[:, heads], ref, "extend full (sampled heads)")
-    check_lse(lse[:, heads], ref_lse)
+    ref, ref_lse = oracle_jobs.extend_all_heads(bits16(q), batch.cu_seqlens_q.cpu().numpy(), bits16(k), bits16(v),
+                                                batch.page_table.cpu().numpy(), batch.seq_lens.cpu().numpy(),
+                                                spec.page_size, spec.sm_scale)
+    assert_bf16_close(out, ref, f"extend full layer {layer}")
+    check_lse(lse, ref_lse)

@@ -69,20 +69,21 @@ def test_clock_summary_keeps_the_timed_region():
     """The clocks reported beside a number are the samples taken while it was timed."""
     sys.path.insert(0, ROOT)
     import bench
-    idle = "0, 1000, 1965, 100, 0x0, Not Active, Not Active, Not Active, Not Active"
-    busy = "0, 1965, 1965, 900, 0x4, Not Active, Not Active, Not Active, Active"
-    hot = "0, 1500, 1965, 950, 0x8, Not Active, Not Active, Active, Not Active"
+    idle = (1000.0, 1965.0, set())
+    busy = (1965.0, 1965.0, {"sw_power_cap"})
+    hot = (1500.0, 1965.0, {"sw_thermal_slowdown"})
     c = bench.ClockSampler(0)
-    c.lines = [(0.9, idle), (1.1, busy), (1.3, hot), (1.5, busy), (1.9, idle)]
+    c.samples = [(t,) + x for t, x in [(0.9, idle), (1.1, busy), (1.3, hot), (1.5, busy), (1.9, idle)]]
     c.t0, c.t1 = 1.0, 1.6
     got = c.summary()
     assert got["samples"] == 3 and got["sm_mhz"] == 1965.0 and got["sm_max_mhz"] == 1965.0
-    assert got["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
-    # shorter than the sampling period: the first sample after the start stands for it
+    assert got["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"] and got["window"] == "in_region"
+    # no sample inside the region: the first one after its start stands for it, marked as such
     c.t0, c.t1 = 1.12, 1.2
     got = c.summary()
     assert got["samples"] == 1 and got["sm_mhz"] == 1500.0 and got["reasons"] == ["sw_thermal_slowdown"]
-    c.lines = []
+    assert got["window"] == "post_region"
+    c.samples = []
     assert c.summary()["reasons"] == ["unsampled"]
 
 

@@ -4,7 +4,7 @@ The bar is the Sage decode's: max over output rows (token, head) of
 ||O_gpu - O_ref||_inf / max(||O_ref||_inf, 1e-6) <= 3e-2; on small cases that span several
 query and key tiles with ragged tails, head groups 1-8, no prefix, one new token per
 request (which equals the Sage decode of the same row), without v_mean, and on the full
-Sage extend workload (sampled heads).
+Sage extend workload (every head of the first and last layer).
 """
 import os
 
@@ -30,10 +30,10 @@ def _lib():
     pa.lib()
 
 
-def case(spec):
+def case(spec, layer=0):
     batch = wl.make_batch(spec, DEV)
     T = int(batch.cu_seqlens_q[-1])
-    lay = wl.make_sage_layer(spec, batch, 0, DEV, q_rows=T)
+    lay = wl.make_sage_layer(spec, batch, layer, DEV, q_rows=T)
     return batch, lay, T
 
 
@@ -50,22 +50,13 @@ def run(spec, batch, lay, T, use_v_mean=True):
     return out
 
 
-def oracle(spec, batch, lay, heads=None, use_v_mean=True):
+def oracle(spec, batch, lay, use_v_mean=True):
     cu = batch.cu_seqlens_q.cpu().numpy()
     table, lens = batch.page_table.cpu().numpy(), batch.seq_lens.cpu().numpy()
     q8, sfq = lay.q8.cpu().numpy(), lay.sf_q.cpu().numpy()
     k8, v8, sfk = lay.k8.cpu().numpy(), lay.v8.cpu().numpy(), lay.sf_k.cpu().numpy()
     sfv, vm = lay.sf_v.cpu().numpy(), lay.v_mean.cpu().numpy() if use_v_mean else None
-    if heads is None:
-        return osg.sage_extend(q8, sfq, cu, k8, v8, sfk, sfv, vm, table, lens, 64)
-    G = spec.hq // spec.hkv
-    cols = []
-    for h in heads:
-        hk = h // G
-        o = osg.sage_extend(q8[:, h:h + 1], sfq[:, h:h + 1], cu, k8[:, hk:hk + 1], v8[:, hk:hk + 1],
-                            sfk[:, hk:hk + 1], sfv[hk:hk + 1], None if vm is None else vm[hk:hk + 1], table, lens, 64)
-        cols.append(o[:, 0])
-    return np.stack(cols, axis=1)
+    return osg.sage_extend(q8, sfq, cu, k8, v8, sfk, sfv, vm, table, lens, 64)
 
 
 def small(**kw):
@@ -105,9 +96,16 @@ def test_sage_extend_one_new_token_matches_sage_decode_and_no_v_mean():
     assert sage_row_rel_error(out, ref) <= SAGE_REL
 
 
-def test_sage_extend_full_workload_sampled_heads():
+@pytest.mark.parametrize("layer", [0, 31])
+def test_sage_extend_full_workload(layer):
+    """Every output row, all 32 query heads, of the first and the last layer of the Sage extend
+    workload (the oracle's heads spread over a process pool)."""
+    from tests import oracle_jobs
     spec = wl.SPECS["sage_extend_prefix"]
-    batch, lay, T = case(spec)
+    batch, lay, T = case(spec, layer)
     out = run(spec, batch, lay, T)
-    heads = [0, 13, 31]
-    assert sage_row_rel_error(out[:, heads], oracle(spec, batch, lay, heads=heads)) <= SAGE_REL
+    h = {k: getattr(lay, k).cpu().numpy() for k in ("q8", "sf_q", "k8", "v8", "sf_k", "sf_v", "v_mean")}
+    ref = oracle_jobs.sage_extend_all_heads(h["q8"], h["sf_q"], batch.cu_seqlens_q.cpu().numpy(), h["k8"], h["v8"],
+                                            h["sf_k"], h["sf_v"], h["v_mean"], batch.page_table.cpu().numpy(),
+                                            batch.seq_lens.cpu().numpy())
+    assert sage_row_rel_error(out, ref) <= SAGE_REL

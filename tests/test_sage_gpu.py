@@ -54,10 +54,12 @@ def oracle_sage(spec, batch, lay, use_v_mean=True):
                            batch.page_table.cpu().numpy(), batch.seq_lens.cpu().numpy(), 64)
 
 
-def test_sage_full_workload():
+@pytest.mark.parametrize("layer", [0, 31])
+def test_sage_full_workload(layer):
+    """Every output row of the first and the last layer of the Sage decode workload."""
     spec = wl.SPECS["sage_decode"]
     batch = wl.make_batch(spec, DEV)
-    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    lay = wl.make_sage_layer(spec, batch, layer, DEV)
     out = run_sage(spec, batch, lay)
     ref = oracle_sage(spec, batch, lay)
     err = sage_row_rel_error(out, ref)

@@ -88,10 +88,13 @@ def test_sparse_plan_bit_exact():
         assert raw[off:off + 4 * nsel].view(np.int32).tolist() == o["sel_block"]
 
 
-def test_sparse_full_workload_density_0125():
+@pytest.mark.parametrize("layer", [0, 31])
+def test_sparse_full_workload_density_0125(layer):
+    """Every output row of the first and the last layer (32 layers rotate over 8 pools, so
+    the last layer reads pool 7, as in the bench)."""
     spec = wl.SPECS["sage_sparse_decode"]
     batch = wl.make_batch(spec, DEV)
-    lay = wl.make_sage_layer(spec, batch, 0, DEV)
+    lay = wl.make_sage_layer(spec, batch, layer % spec.distinct_pools, DEV)
     mask = wl.make_block_mask(spec, batch, DEV)
     out, _, _ = run(spec, batch, lay, mask)
     assert sage_row_rel_error(out, oracle(spec, batch, lay, mask)) <= SAGE_REL

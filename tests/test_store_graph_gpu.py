@@ -195,3 +195,53 @@ def test_sage_store_then_decode_matches_the_oracle():
                           lay.v_mean.cpu().numpy(), table.cpu().numpy(), lens.cpu().numpy(), 64)
     from tests.helpers import SAGE_REL, sage_row_rel_error
     assert sage_row_rel_error(out, ref) <= SAGE_REL
+
+
+def test_graph_captured_at_one_batch_size_serves_new_lengths_at_that_size():
+    """A captured plan + decode step serves one batch size: its launch geometry depends only on
+    the plan parameters (batch, heads, max_kv_len), never on device data, so after the caller
+    writes new sequence lengths and page-table rows into the same device buffers (same B, lengths
+    within max_kv_len) a replay re-plans from them and matches the oracle on the new lengths."""
+    spec = wl.SPECS["decode_llama3_8b"].scaled(batch=8, pool_slots=60_000, len_lo=100, len_hi=3000)
+    batch = wl.make_batch(spec, DEV)
+    k, v = wl.make_bf16_pools(spec, batch, 0, DEV)
+    q = wl.make_bf16_queries(spec, spec.batch, 0, DEV)
+    max_len = batch.page_table.shape[1]
+    params = pa.make_params(pa.PA_MODE_DECODE, spec.batch, spec.hq, spec.hkv, 128, 1, max_kv_len=max_len)
+    ws = alloc_ws(params)
+    lens, table = batch.seq_lens.clone(), batch.page_table.clone()
+    out = torch.zeros_like(q)
+
+    def step():
+        pa.attn_plan(params, lens, None, ws)
+        pa.attn_decode_paged(params, ws, q, k, v, table, spec.sm_scale, out)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            step()
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(77)
+    for trial in range(3):
+        # new lengths for the same requests (shorter prefixes of their rows, one request empty on
+        # the last trial): the table rows still hold the same slots, so every length stays valid
+        new = torch.randint(0, 1 << 30, (spec.batch,), generator=g) % (batch.seq_lens.cpu() + 1)
+        if trial == 2:
+            new[3] = 0
+        lens.copy_(new.to(torch.int32))
+        # and a reversed row order, so the table contents change too
+        perm = torch.arange(spec.batch - 1, -1, -1)
+        table.copy_(batch.page_table[perm.to(DEV)])
+        lens.copy_(new[perm].to(torch.int32))
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert pa.pa_read_device_error(ws) == pa.PA_OK
+        ref, _ = oa.decode(bits16(q), bits16(k), bits16(v), table.cpu().numpy(), lens.cpu().numpy(), 1,
+                           spec.sm_scale)
+        assert_bf16_close(out, ref, f"graph replay with new lengths, trial {trial}")
+    del graph

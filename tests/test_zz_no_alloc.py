@@ -6,8 +6,11 @@ host process's memory pool, or a call site where allocating would synchronise
 the device.  For them the library keeps the plan and the split partials in a
 fixed 16 MiB device array.  This file checks, through the C ABI, that the
 no-allocation call decodes exactly like attn_decode_paged with a caller
-workspace on two calls in a row (the second finds the first one's leftovers in
-the shared array), and that a plan too large for the array is refused.
+workspace, and within the bf16 bar of the fp64 oracle, on two calls in a row
+(the second finds the first one's leftovers in the shared array); that repeated
+calls leave the device's free memory and torch's reserved memory unchanged;
+that an out-of-range page id is reported by pa_noalloc_read_device_error; and
+that a plan too large for the array is refused.
 
 It is named to be collected last, so that a run stopping at the first failure
 has run every other test before it; it also passes alone in a fresh process.
@@ -20,6 +23,7 @@ import torch
 
 import paged_kv_flashattention_split_b200 as pa
 import workloads as wl
+from oracle import attention as oa
 from oracle.codecs import bf16_bits_to_f64
 from tests.helpers import LSE_ABS, alloc_ws, assert_bf16_close, bits16
 
@@ -62,8 +66,36 @@ def test_noalloc_matches_the_workspace_entry_point_on_consecutive_calls():
         lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device=DEV)
         pa.attn_decode_paged_noalloc(params, batch.seq_lens, q, k, v, batch.page_table, spec.sm_scale, out, lse)
         torch.cuda.synchronize()
+        assert pa.pa_noalloc_read_device_error() == pa.PA_OK
         assert_bf16_close(out, bf16_bits_to_f64(bits16(ref)), f"noalloc layer {layer}")
         assert np.max(np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy())) <= LSE_ABS
+        o_ref, l_ref = oa.decode(bits16(q), bits16(k), bits16(v), batch.page_table.cpu().numpy(),
+                                 batch.seq_lens.cpu().numpy(), spec.page_size, spec.sm_scale)
+        assert_bf16_close(out, o_ref, f"noalloc vs oracle, layer {layer}")
+        assert np.max(np.abs(lse.cpu().numpy() - l_ref)) <= LSE_ABS
+
+
+def test_noalloc_calls_leave_device_memory_unchanged_and_report_bad_page_ids():
+    spec = wl.SPECS["decode_tiny"]
+    batch = wl.make_batch(spec, DEV)
+    params = _params(spec, batch)
+    k, v = wl.make_bf16_pools(spec, batch, 0, DEV)
+    q = wl.make_bf16_queries(spec, spec.batch, 0, DEV)
+    out = torch.empty_like(q)
+    pa.attn_decode_paged_noalloc(params, batch.seq_lens, q, k, v, batch.page_table, spec.sm_scale, out)
+    torch.cuda.synchronize()
+    free0, reserved0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_reserved()
+    for _ in range(5):
+        pa.attn_decode_paged_noalloc(params, batch.seq_lens, q, k, v, batch.page_table, spec.sm_scale, out)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0 and torch.cuda.memory_reserved() == reserved0
+    assert pa.pa_noalloc_read_device_error() == pa.PA_OK
+    # one page id past the pool: the kernels skip that key (it reads as zero) and record the error
+    bad = batch.page_table.clone()
+    bad[1, 0] = batch.num_slots + 5
+    pa.attn_decode_paged_noalloc(params, batch.seq_lens, q, k, v, bad, spec.sm_scale, out)
+    assert pa.pa_noalloc_read_device_error() == pa.PA_ERR_DEVICE_INDEX
+    assert pa.pa_noalloc_read_device_error() == pa.PA_OK        # reading clears the word
 
 
 def test_noalloc_refuses_plans_larger_than_its_array():
