@@ -62,7 +62,7 @@ typedef enum {
                                an input the mode does not use passed non-NULL, bad plan mode */
   PA_ERR_UNSUPPORTED = 2,   /* head_dim != 128, page size not a power of two <= 256,
                                Hq / Hkv not in {1,2,4,8}, Sage shared-memory budget exceeded,
-                               EXTEND page size < 8 */
+                               Sage page size other than 64 */
   PA_ERR_ARCH = 3,          /* the current device is not sm_100 (B200) */
   PA_ERR_WORKSPACE = 4,     /* workspace too small, or a run call's mode differs from the plan's */
   PA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
@@ -88,7 +88,7 @@ typedef struct {
   int32_t hq;            /* query heads */
   int32_t hkv;           /* KV heads; hq % hkv == 0 and hq / hkv in {1, 2, 4, 8} */
   int32_t head_dim;      /* D, must be 128 */
-  int32_t page_size;     /* P: power of two, 1 .. 256 (EXTEND: 8 .. 256; SAGE: == sage_k_block) */
+  int32_t page_size;     /* P: power of two, 1 .. 256 (SAGE: == sage_k_block) */
   int32_t max_kv_len;    /* upper bound on every seq_lens[r]; longer lengths are clamped and flagged */
   int32_t max_q_tokens;  /* EXTEND: upper bound on sum of new tokens (sizes the grid); else 0 */
   int32_t num_sms;       /* SMs the plan schedules for; 0 = query the current device */
@@ -244,11 +244,15 @@ pa_status attn_decode_paged_fp8(const pa_plan_params* params, const void* d_ws, 
  * request r (row cu_seqlens_q[r] + i of Q) sits at absolute position p_r + i
  * and attends to keys j <= p_r + i, whose K/V (prefix and new tokens alike)
  * are already in the pool.  O = softmax(sm_scale Q K^T + mask) V.
- * Query tiles of 128 rows per head; key pages arrive by TMA; QK^T and PV run on
- * tcgen05 tensor cores with TMEM accumulators; key tiles above the diagonal
- * are skipped.
+ * Query tiles of 128 rows per head; QK^T and PV run on the tcgen05 tensor
+ * cores with TMEM accumulators; key tiles above the diagonal are skipped.
+ * Key pages of 8 or more slots arrive by TMA (one box per page); smaller pages,
+ * down to the slot-granular page size 1 where the table is req_to_token itself,
+ * are gathered slot by slot with 16-byte copies.  With 4 or 8 query heads per KV
+ * head, a pair of CTAs serves four heads and the tensor cores' two-SM form
+ * shares every K/V tile between them (each SM loads half of it).
  *
- * params, d_ws    the plan (mode PA_MODE_EXTEND); page_size must be >= 8.
+ * params, d_ws    the plan (mode PA_MODE_EXTEND); any page size 1 .. 256.
  * d_q, d_out      bf16 [sum n][Hq][D];  d_lse_out fp32 [sum n][Hq] or NULL.
  * Pools and table as for attn_decode_paged; num_slots < 2^31.
  */

@@ -79,7 +79,6 @@ pa_status derive(const pa_plan_params* p, Derived* d) {
       break;
     case PA_MODE_EXTEND:
       if (p->sage_k_block != 0 || p->max_splits > 1) return PA_ERR_INVALID;
-      if (P < 8) return PA_ERR_UNSUPPORTED;
       d->max_splits = 1;
       d->tile = kExtendKvTile;
       break;

@@ -31,6 +31,7 @@
 // Every wait on an mbarrier is bounded: on timeout the CTA records
 // PA_ERR_DEVICE_INDEX in the workspace, every role stops, the MMA issuer
 // drains its tensor-core work, and TMEM is freed before the CTA exits.
+#include "gather.cuh"
 #include "kernels.h"
 #include "tma.cuh"
 
@@ -57,6 +58,9 @@ constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers, TMEM address, fla
 
 struct ExtendLaunch {
   CUtensorMap tm_q, tm_k, tm_v;   // 64-byte aligned kernel parameters
+  const uint16_t* k_pool;         // for the slot-by-slot gather (page sizes below 8)
+  const uint16_t* v_pool;
+  int gather;                     // 1: K/V tiles by 16-byte cp.async gathers, 0: one TMA box per page
   WsView ws;
   const int32_t* page_table;
   int64_t pt_pitch;
@@ -158,6 +162,55 @@ enum Bar {
 };
 static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
 
+// Producer warp, page sizes below 8: K and V tiles of 128 keys gathered slot by slot with
+// cp.async into the same [2 chunks][128 rows][128 B] layout the TMA boxes produce.  Tile j's
+// copies are issued, then tile j - 1's are waited for, fenced for the tensor cores (async
+// proxy) and announced on its FULL barriers, so one tile is always in flight.  Rows past the
+// request's end (up to the 16-key step the MMAs read) are zero-filled.
+template <typename WaitFn>
+__device__ __forceinline__ int produce_gathered(const ExtendLaunch& a, const int32_t* table, int L, int n_kv,
+                                                int h_kv, uint32_t k_base, uint32_t v_base, uint32_t bar_kfull,
+                                                uint32_t bar_vfull, uint32_t bar_kempty, uint32_t bar_vempty,
+                                                int lane, WaitFn&& wait) {
+  constexpr int kTileBytes = 2 * 128 * 128;
+  int issued = 0;
+  for (int j = 0; j < n_kv; ++j) {
+    const int s = j & 1;
+    const uint32_t par = ((uint32_t)(j >> 1) & 1u) ^ 1u;
+    const int nk = min(128, L - j * 128);
+    const int pad = (nk + 15) & ~15;
+    bool ok = true;
+    if (lane == 0) ok = j < 2 || wait(bar_kempty + 8u * s, par);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    gather_rows<2>(k_base + s * kTileBytes, 128 * 128, 0, a.k_pool, table, j * 128, nk, pad, a.page_shift,
+                   a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
+    cp_async_commit();
+    if (lane == 0) ok = j < 2 || wait(bar_vempty + 8u * s, par);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    gather_rows<2>(v_base + s * kTileBytes, 128 * 128, 0, a.v_pool, table, j * 128, nk, pad, a.page_shift,
+                   a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
+    cp_async_commit();
+    issued = j + 1;
+    if (j > 0) {                                  // tile j - 1 has landed: announce it
+      cp_async_wait<2>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_kfull + 8u * ((j - 1) & 1));
+        mbar_arrive(bar_vfull + 8u * ((j - 1) & 1));
+      }
+    }
+  }
+  cp_async_wait<0>();
+  fence_proxy_async();
+  __syncwarp();
+  if (lane == 0 && issued > 0) {
+    mbar_arrive(bar_kfull + 8u * ((issued - 1) & 1));
+    mbar_arrive(bar_vfull + 8u * ((issued - 1) & 1));
+  }
+  return issued;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_constant__ ExtendLaunch a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -236,9 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       }
       return (int)slot;
     };
-    int next_slot = box_slot(0);
     int issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
+    if (a.gather) {
+      produce_gathered(a, table, L, n_kv, h_kv, base + kOffK, base + kOffV, bar(B_K_FULL), bar(B_V_FULL),
+                       bar(B_K_EMPTY), bar(B_V_EMPTY), lane, wait);
+    }
+    int next_slot = a.gather ? 0 : box_slot(0);
+    for (int j = 0; !a.gather && j < n_kv; ++j) {
       const int s = j & 1;
       const int slot = next_slot;
       const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
@@ -269,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_consta
       if (j + 1 < n_kv) next_slot = box_slot(j + 1);
     }
     // copies still in flight when the CTA gives up: wait (bounded) until they land
-    if (lane == 0 && *abort_flag) {
+    if (lane == 0 && *abort_flag && !a.gather) {
       for (int j = max(0, issued - kNumStages); j < issued; ++j) {
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_K_FULL + (j & 1)), ring_parity(j)); ++i) {}
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_V_FULL + (j & 1)), ring_parity(j)); ++i) {}
@@ -571,9 +628,13 @@ __global__ void __launch_bounds__(kPairThreads, 1) extend_pair_kernel(const __gr
       }
       return (int)slot;
     };
-    int next_slot = box_slot(0);
     int issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
+    if (a.gather) {
+      produce_gathered(a, table, L, n_kv, h_kv, base + kPairOffK, base + kPairOffV, bar(PB_K_FULL), bar(PB_V_FULL),
+                       bar(PB_K_EMPTY), bar(PB_V_EMPTY), lane, wait);
+    }
+    int next_slot = a.gather ? 0 : box_slot(0);
+    for (int j = 0; !a.gather && j < n_kv; ++j) {
       const int s = j & 1;
       const int slot = next_slot;
       const int n_ops = (tile_keys(j) + a.box_rows - 1) / a.box_rows;
@@ -601,7 +662,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) extend_pair_kernel(const __gr
       issued = j + 1;
       if (j + 1 < n_kv) next_slot = box_slot(j + 1);
     }
-    if (lane == 0 && *abort_flag) {
+    if (lane == 0 && *abort_flag && !a.gather) {
       for (int j = max(0, issued - kNumStages); j < issued; ++j) {
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(PB_K_FULL + (j & 1)), ring_parity(j)); ++i) {}
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(PB_V_FULL + (j & 1)), ring_parity(j)); ++i) {}
@@ -804,12 +865,17 @@ bool encode_rows(CUtensorMap* tm, const void* ptr, int64_t rows, int heads, int 
 }  // namespace
 
 cudaError_t launch_extend(const ExtendArgs& in, cudaStream_t s) {
+  // four heads of one KV group over a pair of CTAs sharing every K/V tile (extend_duo.cu)
+  if ((in.hq / in.hkv) % 4 == 0) return launch_extend_duo(in, s);
   static std::atomic<bool> single_set[kMaxDevices], pair_set[kMaxDevices];
   ExtendLaunch a;
+  a.gather = in.page_size < 8 ? 1 : 0;
+  a.k_pool = in.k_pool;
+  a.v_pool = in.v_pool;
   const int box_rows = in.page_size < kTileKeys ? in.page_size : kTileKeys;
   if (!encode_rows(&a.tm_q, in.q, in.q_rows, in.hq, 128) ||
-      !encode_rows(&a.tm_k, in.k_pool, in.num_slots, in.hkv, box_rows) ||
-      !encode_rows(&a.tm_v, in.v_pool, in.num_slots, in.hkv, box_rows))
+      (!a.gather && (!encode_rows(&a.tm_k, in.k_pool, in.num_slots, in.hkv, box_rows) ||
+                     !encode_rows(&a.tm_v, in.v_pool, in.num_slots, in.hkv, box_rows))))
     return cudaErrorInvalidValue;
   a.ws = in.ws;
   a.page_table = in.page_table;

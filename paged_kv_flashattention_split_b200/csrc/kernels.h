@@ -102,6 +102,7 @@ struct ExtendArgs {
   int hq, hkv, page_size, page_shift, max_items;
 };
 cudaError_t launch_extend(const ExtendArgs& a, cudaStream_t s);
+cudaError_t launch_extend_duo(const ExtendArgs& a, cudaStream_t s);   // head groups of 4 or 8, a CTA pair per quad
 
 struct SageExtendArgs {
   WsView ws;

@@ -51,26 +51,42 @@ __device__ void flat_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
   const int U = a.mode == PA_MODE_DECODE ? a.tile : kSageUnit;   // keys per unit
   // 1. lengths (clamped and flagged when out of range); the units of each request
   //    (req_prefix holds them during the plan), and its selected block count (SAGE_SPARSE)
-  for (int r = tid; r < B; r += nt) {
-    int L = a.seq_lens[r];
-    if (L < 0 || L > a.max_kv_len) {
-      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-      L = max(0, min(L, a.max_kv_len));
+  const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
+  if (!sparse) {
+    for (int r = tid; r < B; r += nt) {
+      int L = a.seq_lens[r];
+      if (L < 0 || L > a.max_kv_len) {
+        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+        L = max(0, min(L, a.max_kv_len));
+      }
+      ws.req_len[r] = L;
+      ws.req_prefix[r] = (int)cdiv_ll(L, U);
+      ws.req_splits[r] = 0;
     }
-    ws.req_len[r] = L;
-    int units = (int)cdiv_ll(L, U), nsel = 0;
-    if (sparse) {
+  } else {
+    // one warp per request scans its block mask 32 blocks at a time (coalesced byte loads, ballots)
+    for (int r = warp; r < B; r += nwarps) {
+      int L = a.seq_lens[r];
+      if (L < 0 || L > a.max_kv_len) {
+        if (lane == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+        L = max(0, min(L, a.max_kv_len));
+      }
       const int nb = (int)cdiv_ll(L, kSageBlock);
       const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
-      units = 0;
-      for (int b = 0; b < nb; ++b)
-        if (m[b]) {
-          ++nsel;
-          units += L - kSageBlock * b <= kSageUnit ? 1 : 2;
-        }
+      int units = 0, nsel = 0;
+      for (int b0 = 0; b0 < nb; b0 += 32) {
+        const int b = b0 + lane;
+        const bool sel = b < nb && m[b] != 0;
+        nsel += __popc(__ballot_sync(0xffffffffu, sel));
+        if (sel) units += L - kSageBlock * b <= kSageUnit ? 1 : 2;   // a last block of <= 32 keys is one unit
+      }
+      for (int o = 16; o > 0; o >>= 1) units += __shfl_xor_sync(0xffffffffu, units, o);
+      if (lane == 0) {
+        ws.req_len[r] = L;
+        ws.req_prefix[r] = units;
+        ws.req_splits[r] = nsel;   // scratch until step 3
+      }
     }
-    ws.req_prefix[r] = units;
-    ws.req_splits[r] = nsel;   // scratch until step 3
   }
   __syncthreads();
   const int per_t = (B + nt - 1) / nt;
@@ -87,12 +103,17 @@ __device__ void flat_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
     }
     if (tid == 0) ws.sel_base[B] = total_b;
     __syncthreads();
-    for (int r = tid; r < B; r += nt) {
+    for (int r = warp; r < B; r += nwarps) {    // the selected blocks in ascending order, a warp per request
       const int L = ws.req_len[r], nb = (int)cdiv_ll(L, kSageBlock);
       const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
       int k = ws.sel_base[r];
-      for (int b = 0; b < nb; ++b)
-        if (m[b]) ws.sel_block[k++] = b;
+      for (int b0 = 0; b0 < nb; b0 += 32) {
+        const int b = b0 + lane;
+        const bool sel = b < nb && m[b] != 0;
+        const unsigned ballot = __ballot_sync(0xffffffffu, sel);
+        if (sel) ws.sel_block[k + __popc(ballot & ((1u << lane) - 1u))] = b;
+        k += __popc(ballot);
+      }
     }
   }
   // 2. g_r = exclusive prefix sum of the units (kept in req_aux), total

@@ -50,7 +50,6 @@ constexpr int kTile8 = 128 * 128;                  // 128 rows x 128 bytes of 8-
 constexpr int kStg = 8;                            // ring stages
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLog2_448 = 8.8073549220576041f;   // log2(448): 448 e^x = 2^(x log2(e) + log2(448))
 // int32 -> fp32 without the conversion unit: for |v| < 2^22 the bits 0x4B400000 + v are the
 // float 1.5 * 2^23 + v exactly, and subtracting 1.5 * 2^23 leaves fp32(v) exactly (the
 // dots here are at most 128 * 128 * 128 = 2^21 in magnitude)
@@ -411,10 +410,14 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
       if (mx[1] != INT_MIN) m = fmaxf(m, s1 * (float)(s1 >= 0.f ? mx[1] : mn[1]));
     }
     const float m_use = m == NEG_INF ? 0.f : m;
-    // exponent of 448 e^(S - m) as one fused multiply-add of the exact fp32 dot:
-    // x (sc log2 e) + (log2 448 - m log2 e)
-    const float c2 = kLog2_448 - m_use * kLog2e;
-    float2 l2 = make_float2(0.f, 0.f);   // l scaled by 448
+    // P8 = E4M3(448 exp(S - m)) with S = fp32(sc * dot) formed exactly as the row max was, so
+    // S - m is exact for every key near the max (Sterbenz) and the code each key gets is the
+    // one its float32 score decides: 448 p carries only the rounding of (S - m) log2 e, of
+    // ex2 and of the product by 448 (well under 1e-6 relative), not the error of a score
+    // folded into one fused multiply-add (about 1e-5 near the max at these magnitudes)
+    const float2 neg_m2 = make_float2(-m_use, -m_use), log2e2 = make_float2(kLog2e, kLog2e);
+    const float2 k448 = make_float2(448.f, 448.f);
+    float2 l2 = make_float2(0.f, 0.f);   // l, the sum of the unquantised p
     // pass 2: P8 = E4M3(448 exp(S - m)) into a shared-memory P tile; l of the unquantised p
     for (int j = 0; j < n && ok; ++j) {
       float s0, s1;
@@ -428,28 +431,30 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
       const bool full = __all_sync(0xffffffffu, key0 + kTileRows - 1 <= limit);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        const float a = (cc < 2 ? s0 : s1) * kLog2e;
-        const float2 a2 = make_float2(a, a), c22 = make_float2(c2, c2), nb = make_float2(-kCvtBias, -kCvtBias);
+        const float sc = cc < 2 ? s0 : s1;
+        const float2 sc2 = make_float2(sc, sc), nb = make_float2(-kCvtBias, -kCvtBias);
         uint32_t pw[8];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          float p[4];
+          float q[4];
 #pragma unroll
           for (int u = 0; u < 4; u += 2) {
             float2 x = make_float2(__int_as_float((int)sv[cc][e + u] + kCvtBiasBits),
                                    __int_as_float((int)sv[cc][e + u + 1] + kCvtBiasBits));
-            x = __fadd2_rn(x, nb);                    // the exact fp32 dots
-            const float2 t = __ffma2_rn(x, a2, c22);
-            p[u] = ex2(t.x);
-            p[u + 1] = ex2(t.y);
+            x = __fadd2_rn(x, nb);                                        // the exact fp32 dots
+            const float2 t = __fmul2_rn(__fadd2_rn(__fmul2_rn(x, sc2), neg_m2), log2e2);   // (S - m) log2 e
+            float2 p = make_float2(ex2(t.x), ex2(t.y));
             if (!full) {
               const int k = key0 + 32 * cc + e + u;
-              if (k > limit) p[u] = 0.f;
-              if (k + 1 > limit) p[u + 1] = 0.f;
+              if (k > limit) p.x = 0.f;
+              if (k + 1 > limit) p.y = 0.f;
             }
-            l2 = __fadd2_rn(l2, make_float2(p[u], p[u + 1]));
+            l2 = __fadd2_rn(l2, p);
+            const float2 p448 = __fmul2_rn(p, k448);
+            q[u] = p448.x;
+            q[u + 1] = p448.y;
           }
-          pw[e >> 2] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+          pw[e >> 2] = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
         }
         // keys 32 cc .. 32 cc + 31 are the 16-byte chunks 2 cc and 2 cc + 1 of the row
         *reinterpret_cast<uint4*>(prow + (((2 * cc) ^ sw) << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
@@ -474,7 +479,7 @@ __global__ void __launch_bounds__(Cfg<NH>::kThreads, 1) sage_extend_kernel(const
     if (ok) ok = wwait(bar(B_O_DONE), 0);
     if (ok) {
       tc_fence_after();
-      const float l448 = l2.x + l2.y;
+      const float l448 = 448.f * (l2.x + l2.y);
       const float inv = l448 > 0.f ? 1.f / l448 : 0.f;
       uint16_t* orow = a.out + ((size_t)(q_start + q_local) * a.hq + h) * kHeadDim;
       const float* sfv = a.sf_v + (size_t)h_kv * kHeadDim;

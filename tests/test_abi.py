@@ -63,7 +63,7 @@ def P(**kw):
     (dict(max_q_tokens=5), pa.PA_ERR_INVALID),          # decode plan given an extend-only input
     (dict(sage_k_block=64), pa.PA_ERR_INVALID),
     (dict(max_splits=4), pa.PA_ERR_INVALID),             # no split cap in DECODE (flat partition)
-    (dict(mode=1, page_size=4, max_q_tokens=100), pa.PA_ERR_UNSUPPORTED),
+    (dict(mode=1, page_size=3, max_q_tokens=100), pa.PA_ERR_UNSUPPORTED),
     (dict(mode=2, page_size=64, sage_k_block=16), pa.PA_ERR_UNSUPPORTED),
     (dict(mode=2, page_size=64, sage_k_block=64, max_q_tokens=8), pa.PA_ERR_INVALID),
     (dict(mode=2, page_size=64, sage_k_block=64, max_splits=4), pa.PA_ERR_INVALID),   # no split cap in SAGE
@@ -73,6 +73,12 @@ def P(**kw):
 ])
 def test_parameter_validation(lib, kw, status):
     assert pa.pa_plan_workspace_size(P(**kw), raise_on_error=False) == status
+
+
+@pytest.mark.parametrize("page_size", [1, 2, 4, 8, 256])
+def test_extend_accepts_every_page_size(lib, page_size):
+    """EXTEND plans for any power-of-two page size (below 8 the kernels gather slot by slot)."""
+    assert pa.pa_plan_workspace_size(P(mode=1, page_size=page_size, max_q_tokens=100)) > 64
 
 
 def test_workspace_size_matches_documented_layout(lib):

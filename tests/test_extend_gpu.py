@@ -89,6 +89,12 @@ def test_extend_small_first():
     (64, 8, 1000, 3000, 1, 1),     # single new token per request (decode through extend)
     (128, 2, 0, 700, 200, 600),
     (256, 4, 300, 900, 1, 400),
+    (1, 1, 0, 500, 1, 300),        # page size 1: the table is req_to_token (slot-by-slot gathers)
+    (1, 4, 100, 700, 100, 400),
+    (2, 8, 0, 300, 50, 200),
+    (4, 4, 60, 70, 120, 140),      # a CTA pair whose second K half is empty on the last tile
+    (2, 2, 10, 900, 1, 260),
+    (4, 1, 129, 129, 127, 127),
 ])
 def test_extend_page_sizes_groups_and_ragged_tiles(P, G, lo, hi, nlo, nhi):
     spec = small_spec(page_size=P, hq=2 * G, hkv=2, len_lo=lo, len_hi=hi, new_lo=nlo, new_hi=nhi, batch=4)
@@ -135,3 +141,27 @@ def test_extend_full_workload(layer):
                                                 spec.page_size, spec.sm_scale)
     assert_bf16_close(out, ref, f"extend full layer {layer}")
     check_lse(lse, ref_lse)
+
+
+def test_extend_page_size_one_at_the_extend_workload_lengths():
+    """The extend workload's lengths and heads over a slot-granular cache (page size 1, the
+    table being req_to_token itself), on a sample of query heads of every KV head."""
+    spec = wl.SPECS["extend_prefix"].scaled(page_size=1, spare_pages=0.0, pool_slots=0, layers=1)
+    batch, q, k, v = extend_case(spec)
+    out, lse = run_extend(spec, batch, q, k, v)
+    heads = [0, 5, 10, 15, 16, 21, 26, 31]                      # two of each KV head's four query heads
+    G = spec.hq // spec.hkv
+    qb = bits16(q)[:, heads]
+    kv = sorted({h // G for h in heads})
+    kb, vb = bits16(k)[:, kv], bits16(v)[:, kv]
+    # the oracle over the sampled heads: query head i of the sample reads sampled KV head kv.index(h // G)
+    qs = np.stack([qb[:, i] for i in range(len(heads))], axis=1)
+    ref = np.zeros(qs.shape)
+    ref_lse = np.zeros(qs.shape[:2])
+    for i, h in enumerate(heads):
+        hk = kv.index(h // G)
+        o, l = oa.extend(qs[:, i:i + 1], batch.cu_seqlens_q.cpu().numpy(), kb[:, hk:hk + 1], vb[:, hk:hk + 1],
+                         batch.page_table.cpu().numpy(), batch.seq_lens.cpu().numpy(), 1, spec.sm_scale)
+        ref[:, i], ref_lse[:, i] = o[:, 0], l[:, 0]
+    assert_bf16_close(out[:, heads], ref, "extend P=1 at the extend workload lengths")
+    check_lse(lse[:, heads], ref_lse)
