@@ -163,16 +163,25 @@ enum Bar {
 static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
 
 // Producer warp, page sizes below 8: K and V tiles of 128 keys gathered slot by slot with
-// cp.async into the same [2 chunks][128 rows][128 B] layout the TMA boxes produce.  Tile j's
-// copies are issued, then tile j - 1's are waited for, fenced for the tensor cores (async
-// proxy) and announced on its FULL barriers, so one tile is always in flight.  Rows past the
-// request's end (up to the 16-key step the MMAs read) are zero-filled.
+// cp.async into the same [2 chunks][128 rows][128 B] layout the TMA boxes produce.  The
+// copies complete on no barrier, so the warp announces them itself: once K(j) is issued it
+// waits for K(j - 1)'s copies, fences them for the tensor cores (async proxy) and arrives on
+// K_FULL(j - 1); the same for V after V(j) is issued.  K's announcement never waits for a V
+// stage (the MMA issuer needs K(j) before it can finish with V(j - 1)).  Rows past the
+// request's end, up to the 16-key step the MMAs read, are zero-filled.
 template <typename WaitFn>
-__device__ __forceinline__ int produce_gathered(const ExtendLaunch& a, const int32_t* table, int L, int n_kv,
-                                                int h_kv, uint32_t k_base, uint32_t v_base, uint32_t bar_kfull,
-                                                uint32_t bar_vfull, uint32_t bar_kempty, uint32_t bar_vempty,
-                                                int lane, WaitFn&& wait) {
+__device__ __forceinline__ void produce_gathered(const ExtendLaunch& a, const int32_t* table, int L, int n_kv,
+                                                 int h_kv, uint32_t k_base, uint32_t v_base, uint32_t bar_kfull,
+                                                 uint32_t bar_vfull, uint32_t bar_kempty, uint32_t bar_vempty,
+                                                 int lane, WaitFn&& wait) {
   constexpr int kTileBytes = 2 * 128 * 128;
+  // copy groups are committed in the order K(0), V(0), K(1), V(1), ...
+  auto announce = [&](uint32_t full_bar, int tile) {
+    cp_async_wait<2>();                           // all but the two newest groups have landed
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full_bar + 8u * (tile & 1));
+  };
   int issued = 0;
   for (int j = 0; j < n_kv; ++j) {
     const int s = j & 1;
@@ -185,21 +194,14 @@ __device__ __forceinline__ int produce_gathered(const ExtendLaunch& a, const int
     gather_rows<2>(k_base + s * kTileBytes, 128 * 128, 0, a.k_pool, table, j * 128, nk, pad, a.page_shift,
                    a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
     cp_async_commit();
+    if (j > 0) announce(bar_kfull, j - 1);        // groups after K(j - 1): V(j - 1), K(j)
     if (lane == 0) ok = j < 2 || wait(bar_vempty + 8u * s, par);
     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     gather_rows<2>(v_base + s * kTileBytes, 128 * 128, 0, a.v_pool, table, j * 128, nk, pad, a.page_shift,
                    a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
     cp_async_commit();
+    if (j > 0) announce(bar_vfull, j - 1);        // groups after V(j - 1): K(j), V(j)
     issued = j + 1;
-    if (j > 0) {                                  // tile j - 1 has landed: announce it
-      cp_async_wait<2>();
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar_kfull + 8u * ((j - 1) & 1));
-        mbar_arrive(bar_vfull + 8u * ((j - 1) & 1));
-      }
-    }
   }
   cp_async_wait<0>();
   fence_proxy_async();
@@ -208,7 +210,6 @@ __device__ __forceinline__ int produce_gathered(const ExtendLaunch& a, const int
     mbar_arrive(bar_kfull + 8u * ((issued - 1) & 1));
     mbar_arrive(bar_vfull + 8u * ((issued - 1) & 1));
   }
-  return issued;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) extend_kernel(const __grid_constant__ ExtendLaunch a) {

@@ -112,11 +112,13 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
-// Arrive on an mbarrier of either CTA of the cluster (release at cluster scope).
+// Arrive on an mbarrier of either CTA of the cluster (`cluster_addr` in the shared::cluster
+// window; the default release semantics, as for a local arrive).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
-// Try-wait that acquires at cluster scope (arrivals may come from the peer CTA).
+// Try-wait that acquires at cluster scope: the MMA issuer's barriers that count the peer
+// CTA's arrivals and copies.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -125,6 +127,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
+}
+// Non-blocking test of a phase, acquiring at cluster scope (the issuer polls several barriers).
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 // 4-D tiled load into this CTA's shared memory completing on an mbarrier of either CTA of
 // the pair (`bar` in the shared::cluster window).  No multicast.
@@ -235,15 +252,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+  // bounded waits: `wait` for barriers completed by this CTA's own copies and arrivals or by the
+  // issuer's commits, `wait_cl` (cluster-scope acquire) for the issuer's barriers that count the
+  // peer CTA's copies and arrivals
+  auto wait_impl = [&](uint32_t b, uint32_t parity, bool cluster) -> bool {
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
-      if (mbar_try_wait_cluster(b, parity)) return true;
+      if (cluster ? mbar_try_wait_cluster(b, parity) : mbar_try_wait(b, parity)) return true;
       if (*abort_flag) return false;
     }
     *abort_flag = 1;
     set_device_error(hdr, PA_ERR_DEVICE_INDEX);
     return false;
   };
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool { return wait_impl(b, parity, false); };
+  auto wait_cl = [&](uint32_t b, uint32_t parity) -> bool { return wait_impl(b, parity, true); };
   auto stage_parity = [](int j) -> uint32_t { return (uint32_t)(j / kStages) & 1u; };
   // keys of tile j: [128 j, 128 j + 128) clipped to L; this CTA's K half starts 64 rank further
   auto tile_keys = [&](int j) { return min(kTileKeys, L - j * kTileKeys); };
@@ -273,8 +295,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     int issued = 0;
     if (a.gather) {
-      // tile j's copies are issued, then tile j - 1's are waited for, fenced for the tensor cores
-      // (async proxy) and announced: K to the rank-0 CTA, V to this CTA's softmax warps
+      // the copies complete on no barrier, so the warp announces them: once K(j) is issued it
+      // waits for K(j - 1)'s copies, fences them for the tensor cores (async proxy) and arrives
+      // on the rank-0 CTA's KFULL; the same for V (this CTA's VLAND) after V(j) is issued.
+      // Copy groups are committed K(0), V(0), K(1), V(1), ...: two newer groups each time.
+      auto announce = [&](uint32_t full_bar_cluster) {
+        cp_async_wait<2>();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(full_bar_cluster);
+      };
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
         const int nk = half_keys(j, (int)rank), nv = tile_keys(j);
@@ -284,21 +314,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         gather_rows<2>(base + kOffK + s * kKStage, kKChunk, 0, a.k_pool, table, j * kTileKeys + 64 * (int)rank, nk,
                        (nk + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
         cp_async_commit();
+        if (j > 0) announce(map_to_rank(bar(B_KFULL + (j - 1) % kStages), 0));
         if (lane == 0) ok = j < kStages || wait(bar(B_VEMPTY + s), stage_parity(j) ^ 1u);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         gather_rows<1>(base + kOffV + s * kVStage, kVStage, (int)rank, a.v_pool, table, j * kTileKeys, nv,
                        (nv + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
         cp_async_commit();
+        if (j > 0) announce(map_to_rank(bar(B_VLAND + (j - 1) % kStages), rank));
         issued = j + 1;
-        if (j > 0) {
-          cp_async_wait<2>();
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_cluster(map_to_rank(bar(B_KFULL + (j - 1) % kStages), 0));
-            mbar_arrive(bar(B_VLAND + (j - 1) % kStages));
-          }
-        }
       }
       cp_async_wait<0>();
       fence_proxy_async();
@@ -347,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int j = max(0, issued - kStages); j < issued; ++j) {
         if (leader)
           for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait_cluster(bar(B_KFULL + j % kStages), stage_parity(j)); ++i) {}
-        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait_cluster(bar(B_VLAND + j % kStages), stage_parity(j)); ++i) {}
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_VLAND + j % kStages), stage_parity(j)); ++i) {}
       }
     }
   } else if (warp == 1) {
@@ -372,36 +395,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       smem_desc(vb + kk * 16 * 128, kVStage), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit_pair(bar(B_PVDONE + t));
       };
-      bool ok = wait(bar(B_Q), 0) && wait(bar(B_KFULL), 0);
+      bool ok = wait_cl(bar(B_Q), 0) && wait_cl(bar(B_KFULL), 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
         tc_commit_pair(bar(B_KEMPTY));
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          const int s1 = (j + 1) % kStages;
-          if (!(ok = wait(bar(B_KFULL + s1), stage_parity(j + 1)))) break;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!(ok = wait(bar(B_SFREE + t), (uint32_t)j & 1u))) break;   // both CTAs read S_t(j)
+      // Event-driven issue: each head's next S (needs its K tile and both CTAs' softmax to have
+      // read the previous S) and next PV (needs both CTAs' P) go to the tensor cores as soon as
+      // they are ready, so one head's softmax never holds up the other head's MMAs.  A K stage
+      // is released once both heads' S of that tile are issued, a V stage once both PVs are.
+      int ns[2] = {1, 1}, npv[2] = {0, 0}, k_rel = 1, v_rel = 0;
+      uint32_t idle = 0;
+      while (ok && (npv[0] < n_kv || npv[1] < n_kv)) {
+        bool progress = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (npv[t] < n_kv && mbar_test_wait_cluster(bar(B_PFULL + t), (uint32_t)npv[t] & 1u)) {
             tc_fence_after();
-            issue_s(t, j + 1);
+            issue_pv(t, npv[t]++);
+            progress = true;
           }
-          if (!ok) break;
-          tc_commit_pair(bar(B_KEMPTY + s1));
+          if (ns[t] < n_kv && mbar_test_wait_cluster(bar(B_SFREE + t), (uint32_t)(ns[t] - 1) & 1u) &&
+              mbar_test_wait_cluster(bar(B_KFULL + ns[t] % kStages), stage_parity(ns[t]))) {
+            tc_fence_after();
+            issue_s(t, ns[t]++);
+            progress = true;
+          }
         }
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = wait(bar(B_PFULL + t), (uint32_t)j & 1u))) break;     // both CTAs wrote P_t(j)
-          tc_fence_after();
-          issue_pv(t, j);
+        while (k_rel < n_kv && ns[0] > k_rel && ns[1] > k_rel) tc_commit_pair(bar(B_KEMPTY + (k_rel++) % kStages));
+        while (v_rel < n_kv && npv[0] > v_rel && npv[1] > v_rel) tc_commit_pair(bar(B_VEMPTY + (v_rel++) % kStages));
+        if (progress) {
+          idle = 0;
+        } else if (++idle > 4 * kWaitLimit || *abort_flag) {
+          if (!*abort_flag) {
+            *abort_flag = 1;
+            set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+          }
+          ok = false;
+        } else {
+          __nanosleep(32);
         }
-        if (!ok) break;
-        tc_commit_pair(bar(B_VEMPTY + j % kStages));
       }
       // all issued tensor-core work has finished before TMEM is released
       tc_commit_pair(bar(B_DRAIN));
-      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait_cluster(bar(B_DRAIN), 0); ++i) {}
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++i) {}
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -442,15 +481,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e)
             if (key0 + 32 * cc + e > limit) sv[cc][e] = __float_as_uint(NEG_INF);
       }
-      float mxp[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mxp[i] = NEG_INF;
+      // row max over four independent 3-input chains
+      float mxp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(sv[cc][e]));
-      float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        for (int e = 0; e < 32; e += 2)
+          mxp[cc] = max3(mxp[cc], __uint_as_float(sv[cc][e]), __uint_as_float(sv[cc][e + 1]));
+      float mx = max3(mxp[0], mxp[1], fmaxf(mxp[2], mxp[3]));
       mx *= c;                                                  // log2 units
       float alpha = 1.f;
       if (m_used == NEG_INF) {
@@ -459,21 +497,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         alpha = ex2(m_used - mx);
         m_used = mx;
       }
-      // P = 2^(c s - m) as bf16 pairs (in the low half of each 32-register row), row sum of the rounded values
+      // P = 2^(c s - m) packed to bf16 pairs (in the low half of each 32-register row); the row sum
+      // adds the same bf16-rounded values the PV MMA multiplies, so O is a convex combination of V
+      // rows whatever the rounding of P
       const float neg_m = m_used == NEG_INF ? 0.f : -m_used;
-      float ltp[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ltp[i] = 0.f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+      float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint32_t w = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[cc][e]), c, neg_m)),
-                                         ex2(fmaf(__uint_as_float(sv[cc][e + 1]), c, neg_m)));
-          ltp[(e >> 1) & 7] += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[cc][e]), __uint_as_float(sv[cc][e + 1])), c2, nm2);
+          const uint32_t w = pack_bf16x2(ex2(x.x), ex2(x.y));
+          lsum[(e >> 1) & 3] = __fadd2_rn(lsum[(e >> 1) & 3], make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w)));
           sv[cc][e >> 1] = w;
         }
-      const float lt = ((ltp[0] + ltp[1]) + (ltp[2] + ltp[3])) + ((ltp[4] + ltp[5]) + (ltp[6] + ltp[7]));
+      const float2 ls = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+      const float lt = ls.x + ls.y;
       // PV_t(j-1) done: the P_t buffer is free and O_t holds every earlier tile
       if (j > 0 && !(ok = wwait(bar(B_PVDONE + t), (uint32_t)(j - 1) & 1u))) break;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {              // rescale rows of O_t in TMEM
@@ -500,10 +540,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(prow_base + chunk * kPChunk + row * 128 + ((unit ^ (row & 7)) << 4)) =
             make_uint4(w0, w1, w2, w3);
       }
-      // this CTA's V half of tile j has landed; rows past L inside the last 16-key step must read as zero
+      // this CTA's V half of tile j has landed; rows past L inside the last 16-key step must read
+      // as zero.  Either head's PV(j) may run first, so the first warp of each warpgroup writes the
+      // same zeros before its own P_FULL arrival.
       if (!(ok = wwait(bar(B_VLAND + j % kStages), stage_parity(j)))) break;
       const int nk = tile_keys(j);
-      if (t == 0 && warp == 2 && nk < kTileKeys && (nk & 15)) {
+      if ((warp & 3) == 2 && nk < kTileKeys && (nk & 15)) {
         uint8_t* vt = base_ptr + kOffV + (j % kStages) * kVStage;
         const int z0 = nk, z1 = (nk + 15) & ~15;
         for (int idx = lane; idx < (z1 - z0) * 8; idx += 32) {   // 16-byte units of rows z0 .. z1 - 1
