@@ -173,7 +173,8 @@ KERNEL_SOURCES = {
     "decode_long_llama3_70b": ("decode.cu", "common.cuh"),
     "decode_tiny": ("decode.cu", "common.cuh"),
     "decode_fp8_llama3_8b": ("decode_fp8.cu", "decode.cu", "common.cuh"),
-    "extend_prefix": ("extend.cu", "common.cuh", "tma.cuh"),
+    "extend_prefix": ("extend_duo.cu", "gather.cuh", "kernels.h", "common.cuh", "tma.cuh"),
+    "extend_prefix_page1": ("extend_duo.cu", "gather.cuh", "kernels.h", "common.cuh", "tma.cuh"),
     "sage_decode": ("sage.cu", "common.cuh", "tma.cuh"),
     "sage_sparse_decode": ("sage.cu", "common.cuh", "tma.cuh"),
     "sage_extend_prefix": ("sage_extend.cu", "common.cuh", "tma.cuh"),
@@ -619,6 +620,7 @@ class Fp8DecodeWorkload(DecodeWorkload):
 
 WORKLOADS = {   # workload name (workloads.SPECS) -> the step it runs
     "extend_prefix": ExtendWorkload,
+    "extend_prefix_page1": ExtendWorkload,
     "decode_fp8_llama3_8b": Fp8DecodeWorkload,
     "sage_sparse_decode": SageSparseWorkload,
     "sage_extend_prefix": SageExtendWorkload,
@@ -637,12 +639,14 @@ DTYPES = {"sage_decode": "int8/e4m3 in, fp32 math, bf16 out",
           "decode_fp8_llama3_8b": "e4m3 KV, bf16 Q/O, f16 tensor-core math, fp32 accumulation"}
 STEP_CALLS = {"sage_decode": "attn_decode_paged_sage", "sage_sparse_decode": "attn_decode_paged_sage (block-sparse plan)",
               "sage_extend_prefix": "attn_extend_paged_sage", "extend_prefix": "attn_extend_paged",
+              "extend_prefix_page1": "attn_extend_paged",
               "decode_fp8_llama3_8b": "attn_decode_paged_fp8"}
 ROOFLINE_KERNELS = {
     "sage_decode": "attn_decode_paged_sage call (sage_score_kernel + sage_value_kernel + sage_merge_kernel)",
     "sage_sparse_decode": "attn_decode_paged_sage call, block-sparse plan (score + value + merge kernels)",
     "sage_extend_prefix": "sage_extend_kernel (one launch per attn_extend_paged_sage call; 3 contractions per tile pair, 2 counted)",
-    "extend_prefix": "extend_pair_kernel (one launch per attn_extend_paged call)",
+    "extend_prefix": "extend_duo_kernel (a pair of CTAs per query tile and 4 heads; one launch per attn_extend_paged call)",
+    "extend_prefix_page1": "extend_duo_kernel with slot-by-slot cp.async gathers (page size 1; one launch per call)",
     "decode_fp8_llama3_8b": "attn_decode_paged_fp8 call (decode_fp8_kernel + merge_kernel)"}
 # workloads measured beside the default decode in the default run (the other halves of the metric)
 DEFAULT_EXTRAS = ("extend_prefix", "sage_decode")

@@ -191,13 +191,13 @@ __device__ __forceinline__ void produce_gathered(const ExtendLaunch& a, const in
     bool ok = true;
     if (lane == 0) ok = j < 2 || wait(bar_kempty + 8u * s, par);
     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-    gather_rows<2>(k_base + s * kTileBytes, 128 * 128, 0, a.k_pool, table, j * 128, nk, pad, a.page_shift,
+    gather_rows<2, 128>(k_base + s * kTileBytes, 128 * 128, 0, a.k_pool, table, j * 128, nk, pad, a.page_shift,
                    a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
     cp_async_commit();
     if (j > 0) announce(bar_kfull, j - 1);        // groups after K(j - 1): V(j - 1), K(j)
     if (lane == 0) ok = j < 2 || wait(bar_vempty + 8u * s, par);
     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-    gather_rows<2>(v_base + s * kTileBytes, 128 * 128, 0, a.v_pool, table, j * 128, nk, pad, a.page_shift,
+    gather_rows<2, 128>(v_base + s * kTileBytes, 128 * 128, 0, a.v_pool, table, j * 128, nk, pad, a.page_shift,
                    a.page_size, a.hkv, h_kv, a.num_slots, a.ws.hdr, lane);
     cp_async_commit();
     if (j > 0) announce(bar_vfull, j - 1);        // groups after V(j - 1): K(j), V(j)

@@ -201,6 +201,9 @@ constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3
 constexpr uint32_t kIdescS = kIdescBase;                 // A (Q) and B (K) K-major
 constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);   // A (P) K-major, B (V) MN-major: d contiguous
 
+// GATHER: the page-size-below-8 path (cp.async gathers); a separate instantiation, so the TMA
+// path's register allocation carries none of the gather code.
+template <bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     extend_duo_kernel(const __grid_constant__ DuoLaunch a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -236,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       const bool warp_arrivals = (i >= B_SFREE && i < B_SFREE + 2) || (i >= B_PFULL && i < B_PFULL + 2);
-      const bool gathered_k = a.gather && i >= B_KFULL && i < B_KFULL + kStages;
+      const bool gathered_k = GATHER && i >= B_KFULL && i < B_KFULL + kStages;
       mbar_init(bar(i), warp_arrivals ? 8u : gathered_k ? 2u : 1u);
     }
     *abort_flag = 0;
@@ -294,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       return (int)slot;
     };
     int issued = 0;
-    if (a.gather) {
+    if (GATHER) {
       // the copies complete on no barrier, so the warp announces them: once K(j) is issued it
       // waits for K(j - 1)'s copies, fences them for the tensor cores (async proxy) and arrives
       // on the rank-0 CTA's KFULL; the same for V (this CTA's VLAND) after V(j) is issued.
@@ -311,13 +314,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
         if (lane == 0) ok = j < kStages || wait(bar(B_KEMPTY + s), stage_parity(j) ^ 1u);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        gather_rows<2>(base + kOffK + s * kKStage, kKChunk, 0, a.k_pool, table, j * kTileKeys + 64 * (int)rank, nk,
+        gather_rows<2, 64>(base + kOffK + s * kKStage, kKChunk, 0, a.k_pool, table, j * kTileKeys + 64 * (int)rank, nk,
                        (nk + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
         cp_async_commit();
         if (j > 0) announce(map_to_rank(bar(B_KFULL + (j - 1) % kStages), 0));
         if (lane == 0) ok = j < kStages || wait(bar(B_VEMPTY + s), stage_parity(j) ^ 1u);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        gather_rows<1>(base + kOffV + s * kVStage, kVStage, (int)rank, a.v_pool, table, j * kTileKeys, nv,
+        gather_rows<1, 128>(base + kOffV + s * kVStage, kVStage, (int)rank, a.v_pool, table, j * kTileKeys, nv,
                        (nv + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
         cp_async_commit();
         if (j > 0) announce(map_to_rank(bar(B_VLAND + (j - 1) % kStages), rank));
@@ -332,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       issued = 0;                                                // nothing left in flight
     }
-    for (int j = 0; !a.gather && j < n_kv; ++j) {
+    for (int j = 0; !GATHER && j < n_kv; ++j) {
       const int s = j % kStages;
       // K: this CTA's 64-key half, one box per page (box_k rows), both d chunks
       const int kk0 = j * kTileKeys + 64 * (int)rank;
@@ -610,8 +613,9 @@ bool encode_rows(CUtensorMap* tm, const void* ptr, int64_t rows, int heads, int 
 }  // namespace
 
 cudaError_t launch_extend_duo(const ExtendArgs& in, cudaStream_t s) {
-  static std::atomic<bool> smem_set[kMaxDevices];
-  cudaError_t e = raise_smem_limit(extend_duo_kernel, kSmemBytes, smem_set);
+  static std::atomic<bool> smem_set[kMaxDevices], smem_set_g[kMaxDevices];
+  cudaError_t e = in.page_size < 8 ? raise_smem_limit(extend_duo_kernel<true>, kSmemBytes, smem_set_g)
+                                   : raise_smem_limit(extend_duo_kernel<false>, kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   DuoLaunch a;
   a.gather = in.page_size < 8 ? 1 : 0;
@@ -637,7 +641,10 @@ cudaError_t launch_extend_duo(const ExtendArgs& in, cudaStream_t s) {
   a.page_shift = in.page_shift;
   a.box_k = box_k;
   a.box_v = box_v;
-  extend_duo_kernel<<<in.max_items * (in.hq / 4) * 2, kThreads, kSmemBytes, s>>>(a);
+  if (a.gather)
+    extend_duo_kernel<true><<<in.max_items * (in.hq / 4) * 2, kThreads, kSmemBytes, s>>>(a);
+  else
+    extend_duo_kernel<false><<<in.max_items * (in.hq / 4) * 2, kThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 

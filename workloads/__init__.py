@@ -90,6 +90,8 @@ CONFIGS = {
             page_size=64, spare_pages=0.05, layers=32, distinct_pools=8, density=0.125),
     8: Spec("sage_extend_prefix", 8, "extend", batch=8, len_lo=0, len_hi=4096, hq=32, hkv=8,
             page_size=64, spare_pages=0.10, new_lo=128, new_hi=2048, layers=32),
+    9: Spec("extend_prefix_page1", 9, "extend", batch=8, len_lo=0, len_hi=4096, hq=32, hkv=8,
+            page_size=1, new_lo=128, new_hi=2048, layers=32),
 }
 
 # the workloads by name (the number of each is its seed id)
