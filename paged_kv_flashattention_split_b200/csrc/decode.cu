@@ -58,6 +58,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
   // the merge kernel (launched as a programmatic dependent) may be scheduled now; it
   // waits for this whole grid to finish before it reads anything
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // this grid is itself a programmatic dependent of whatever precedes it on the stream (the
+  // previous layer's merge lets it start early): nothing is read before that grid is done
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   int32_t* sbuf = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes);   // [2][TK]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -281,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
 // and keeps up to 8 splits' loads in flight.
 __global__ void __launch_bounds__(256) merge_kernel(DecodeLaunch a) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the decode grid has completed and its writes are visible
+  // the next layer's decode grid (a programmatic dependent) may be scheduled: it waits for this one
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   PlanHeader* hdr = a.ws.hdr;
   if (!workspace_ok(hdr, PA_MODE_DECODE)) return;
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -346,8 +351,7 @@ cudaError_t launch_decode_hg(const DecodeLaunch& a, cudaStream_t s) {
   static std::atomic<bool> smem_set[kMaxDevices];
   cudaError_t e = raise_smem_limit(decode_splitkv_kernel<HG, G>, kDecodeSmem, smem_set);
   if (e != cudaSuccess) return e;
-  decode_splitkv_kernel<HG, G><<<a.slots * (a.hkv / HG), kThreads, kDecodeSmem, s>>>(a);
-  e = cudaGetLastError();
+  e = launch_programmatic(decode_splitkv_kernel<HG, G>, dim3(a.slots * (a.hkv / HG)), dim3(kThreads), kDecodeSmem, a, s);
   if (e != cudaSuccess) return e;
   return launch_decode_merge(a, s);
 }

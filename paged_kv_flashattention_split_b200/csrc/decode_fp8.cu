@@ -79,6 +79,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fp8_kernel(Fp8DecodeLaunch
   extern __shared__ __align__(128) uint8_t smem[];
   // the merge (a programmatic dependent) may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // a programmatic dependent of whatever precedes it on the stream: nothing is read before
+  // that grid is done
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   int32_t* sbuf = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes);   // [2][TK]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -322,8 +325,7 @@ cudaError_t launch_fp8_hg(const Fp8DecodeLaunch& a, cudaStream_t s) {
   static std::atomic<bool> smem_set[kMaxDevices];
   cudaError_t e = raise_smem_limit(decode_fp8_kernel<HG, G>, kSmem, smem_set);
   if (e != cudaSuccess) return e;
-  decode_fp8_kernel<HG, G><<<a.slots * (a.hkv / HG), kThreads, kSmem, s>>>(a);
-  e = cudaGetLastError();
+  e = launch_programmatic(decode_fp8_kernel<HG, G>, dim3(a.slots * (a.hkv / HG)), dim3(kThreads), kSmem, a, s);
   if (e != cudaSuccess) return e;
   DecodeLaunch m{};
   m.ws = a.ws;

@@ -9,6 +9,24 @@ namespace pa {
 
 constexpr int kMaxDevices = 64;
 
+// Launches `kernel` as a programmatic dependent of the grid before it on `s`: it may start
+// once that grid executes griddepcontrol.launch_dependents (or exits), and must itself
+// execute griddepcontrol.wait before it reads anything that grid (or any earlier work) wrote.
+template <typename K, typename A>
+cudaError_t launch_programmatic(K kernel, dim3 grid, dim3 block, size_t smem, const A& args, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device, once per
 // device.  Host threads may launch at the same time: the per-device flags are atomic, and
 // setting the attribute twice is harmless.  Devices beyond kMaxDevices set it on every call.

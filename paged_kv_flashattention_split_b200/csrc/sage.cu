@@ -379,6 +379,9 @@ __global__ void __launch_bounds__(kThreads, 2) sage_score_kernel(const __grid_co
   // the value pass (a programmatic dependent) may be scheduled now; it waits for this
   // whole grid to finish before it reads the scores
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // this grid is itself a programmatic dependent of whatever precedes it on the stream (the
+  // previous layer's merge lets it start early): nothing is read before that grid is done
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3, mat = lane >> 3;
   PlanHeader* hdr = a.ws.hdr;
@@ -654,6 +657,8 @@ __global__ void __launch_bounds__(kThreads, 2 * SageSmem<HG, G, true>::BYTES <= 
 // issues the loads of 8 items before it adds them (in item order).
 __global__ void __launch_bounds__(256) sage_merge_kernel(const __grid_constant__ SageLaunch a) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the value pass has completed
+  // the next layer's score pass (a programmatic dependent) may be scheduled: it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   PlanHeader* hdr = a.ws.hdr;
   if (!sage_ws_ok(hdr)) return;
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -764,8 +769,7 @@ cudaError_t launch_sage_hg(SageLaunch& a, const int8_t* k8, const uint8_t* v8, i
       !encode_pool(&a.tm_kv, k8, a.num_slots, a.hkv, HG) ||
       (HG >= 4 && !encode_sfk(&a.tm_sfk, a.sf_k, a.num_slots / kSageBlock, a.hkv, HG)))
     return cudaErrorInvalidValue;
-  sage_score_kernel<HG, G><<<grid, kThreads, LS::BYTES, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(sage_score_kernel<HG, G>, grid, dim3(kThreads), LS::BYTES, a, s);
   if (e != cudaSuccess) return e;
   if (!encode_pool(&a.tm_kv, v8, a.num_slots, a.hkv, HG)) return cudaErrorInvalidValue;
   e = launch_pdl(sage_value_kernel<HG, G>, grid, dim3(kThreads), LV::BYTES, a, s);
