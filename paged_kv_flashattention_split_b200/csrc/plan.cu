@@ -6,6 +6,8 @@
 // 도입", 코드 분석 items 1-3, 왜 이게 좋은가 item 1).  The algorithm is the one
 // stated at attn_plan in pagedattn.h; every step is integer so the result is
 // exact and identical on recomputation.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace pa {
@@ -15,21 +17,46 @@ constexpr int kPlanThreads = 1024;
 
 __device__ __forceinline__ long long cdiv_ll(long long a, long long b) { return (a + b - 1) / b; }
 
-// Block-wide exclusive scan of one int per thread; returns this thread's prefix.
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, at most 1024);
+// returns this thread's prefix.  Warps scan by shuffles, one warp scans the warp totals:
+// two barriers (and one more before `scratch`, 33 ints, may be reused).
 __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
-  const int tid = threadIdx.x;
-  scratch[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < blockDim.x; off <<= 1) {
-    int add = tid >= off ? scratch[tid - off] : 0;
-    __syncthreads();
-    scratch[tid] += add;
-    __syncthreads();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  int incl = scratch[tid];
-  *total = scratch[blockDim.x - 1];
+  if (lane == 31) scratch[warp] = x;
   __syncthreads();
-  return incl - v;
+  if (warp == 0) {
+    int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    scratch[lane] = w;                            // inclusive over warps 0 .. lane
+    if (lane == 31) scratch[32] = w;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? scratch[warp - 1] : 0;
+  *total = scratch[32];
+  __syncthreads();
+  return before + x - v;
+}
+
+// The block mask of one request, 512 blocks per warp-wide step: lane l holds blocks
+// b0 + 16 l .. b0 + 16 l + 15 as bits 0..15 (16 independent byte loads, so one load latency).
+__device__ __forceinline__ uint32_t mask_bits(const uint8_t* m, int b0, int nb, int lane) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int b = b0 + 16 * lane + i;
+    if (b < nb && __ldg(m + b) != 0) bits |= 1u << i;
+  }
+  return bits;
 }
 
 // EXTEND: work of query tile s (key tiles it needs) for the sort key; items run longest first.
@@ -41,132 +68,164 @@ __device__ __forceinline__ int item_work(int s, int prefix, int n) {
 // DECODE, SAGE_DECODE, SAGE_SPARSE: the flat partition of the requests' units (T-key tiles
 // for DECODE, 32-key units for Sage, of the selected 64-key blocks only for SAGE_SPARSE)
 // over CTA slots (the algorithm at attn_plan).  Items come out r-major, which is also slot
-// order, so no sort.
-__device__ void flat_plan(const PlanLaunch& a, int* item_slot, int* scan, int* chunk_out, int* n_out) {
+// order, so no sort.  Each thread owns the requests [r0, r1) through every step; the
+// per-request values live in shared memory (`sm`, 3 B + max_items ints), so the only global
+// reads are the lengths and the masks, issued together, and the workspace is written once.
+__device__ void flat_plan(const PlanLaunch& a, int* sm, int* scan, int* chunk_out, int* n_out) {
   const int tid = threadIdx.x, nt = blockDim.x;
   WsView ws = a.ws;
   PlanHeader* hdr = ws.hdr;
   const int B = a.batch;
   const bool sparse = a.mode == PA_MODE_SAGE_SPARSE;
   const int U = a.mode == PA_MODE_DECODE ? a.tile : kSageUnit;   // keys per unit
-  // 1. lengths (clamped and flagged when out of range); the units of each request
-  //    (req_prefix holds them during the plan), and its selected block count (SAGE_SPARSE)
+  int* s_len = sm;               // L_r
+  int* s_units = sm + B;         // units of request r
+  int* s_sel = sm + 2 * B;       // SAGE_SPARSE: selected blocks of r, then sel_base[r]
+  int* item_slot = sm + 3 * B;   // [max_items]
   const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
+  const int per_t = (B + nt - 1) / nt;
+  const int r0 = min(B, tid * per_t), r1 = min(B, r0 + per_t);
+  auto clamp_len = [&](int L) {
+    if (L < 0 || L > a.max_kv_len) {
+      set_device_error(hdr, PA_ERR_DEVICE_INDEX);
+      L = max(0, min(L, a.max_kv_len));
+    }
+    return L;
+  };
+  // 1. lengths (clamped and flagged when out of range), the units of each request, and its
+  //    selected block count (SAGE_SPARSE)
+  uint32_t kept_bits = 0;        // SAGE_SPARSE: this lane's mask bits of the warp's one request
+  const bool keep = sparse && B <= nwarps;
   if (!sparse) {
-    for (int r = tid; r < B; r += nt) {
-      int L = a.seq_lens[r];
-      if (L < 0 || L > a.max_kv_len) {
-        set_device_error(hdr, PA_ERR_DEVICE_INDEX);
-        L = max(0, min(L, a.max_kv_len));
-      }
+    for (int r = r0; r < r1; ++r) {
+      const int L = clamp_len(a.seq_lens[r]);
+      s_len[r] = L;
+      s_units[r] = (int)cdiv_ll(L, U);
       ws.req_len[r] = L;
-      ws.req_prefix[r] = (int)cdiv_ll(L, U);
-      ws.req_splits[r] = 0;
+      ws.req_prefix[r] = 0;
     }
   } else {
-    // one warp per request scans its block mask 32 blocks at a time (coalesced byte loads, ballots)
+    // one warp per request; the first 512 mask bytes are read together with the length (the
+    // row holds mask_pitch >= ceil(max_kv_len / 64) bytes) and cut to ceil(L / 64) blocks
+    const int first_chunk = (int)min(a.mask_pitch, (int64_t)512);
     for (int r = warp; r < B; r += nwarps) {
-      int L = a.seq_lens[r];
+      const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
+      const int L_raw = a.seq_lens[r];
+      uint32_t bits = mask_bits(m, 0, first_chunk, lane);
+      int L = L_raw;
       if (L < 0 || L > a.max_kv_len) {
         if (lane == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
         L = max(0, min(L, a.max_kv_len));
       }
       const int nb = (int)cdiv_ll(L, kSageBlock);
-      const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
-      int units = 0, nsel = 0;
-      for (int b0 = 0; b0 < nb; b0 += 32) {
-        const int b = b0 + lane;
-        const bool sel = b < nb && m[b] != 0;
-        nsel += __popc(__ballot_sync(0xffffffffu, sel));
-        if (sel) units += L - kSageBlock * b <= kSageUnit ? 1 : 2;   // a last block of <= 32 keys is one unit
+      const int live = nb - 16 * lane;                   // blocks of this lane's 16 inside the row
+      bits &= live >= 16 ? 0xFFFFu : live > 0 ? (1u << live) - 1u : 0u;
+      int nsel = __popc(bits);
+      bool last_sel = live >= 1 && live <= 16 && ((bits >> (live - 1)) & 1u);
+      if (keep) kept_bits = bits;
+      for (int b0 = 512; b0 < nb; b0 += 512) {           // rows of more than 512 blocks
+        const uint32_t more = mask_bits(m, b0, nb, lane);
+        nsel += __popc(more);
+        const int i_last = nb - 1 - b0 - 16 * lane;
+        if (i_last >= 0 && i_last < 16) last_sel = (more >> i_last) & 1u;
       }
-      for (int o = 16; o > 0; o >>= 1) units += __shfl_xor_sync(0xffffffffu, units, o);
+      for (int o = 16; o > 0; o >>= 1) nsel += __shfl_xor_sync(0xffffffffu, nsel, o);
+      // two 32-key units per selected block; a last block of <= 32 keys is one unit
+      const bool short_last = __any_sync(0xffffffffu, last_sel) && L - kSageBlock * (nb - 1) <= kSageUnit;
       if (lane == 0) {
+        s_len[r] = L;
+        s_units[r] = 2 * nsel - (short_last ? 1 : 0);
+        s_sel[r] = nsel;
         ws.req_len[r] = L;
-        ws.req_prefix[r] = units;
-        ws.req_splits[r] = nsel;   // scratch until step 3
+        ws.req_prefix[r] = 0;
       }
     }
   }
   __syncthreads();
-  const int per_t = (B + nt - 1) / nt;
-  const int r0 = min(B, tid * per_t), r1 = min(B, r0 + per_t);
   if (sparse) {
-    // sel_base = exclusive prefix sum of the selected block counts; the block lists
+    // sel_base = exclusive prefix sum of the selected block counts; then the block lists
     int local_b = 0;
-    for (int r = r0; r < r1; ++r) local_b += ws.req_splits[r];
+    for (int r = r0; r < r1; ++r) local_b += s_sel[r];
     int total_b = 0;
     int run_b = block_exclusive_scan(local_b, scan, &total_b);
     for (int r = r0; r < r1; ++r) {
+      const int n = s_sel[r];
+      s_sel[r] = run_b;
       ws.sel_base[r] = run_b;
-      run_b += ws.req_splits[r];
+      run_b += n;
     }
     if (tid == 0) ws.sel_base[B] = total_b;
     __syncthreads();
     for (int r = warp; r < B; r += nwarps) {    // the selected blocks in ascending order, a warp per request
-      const int L = ws.req_len[r], nb = (int)cdiv_ll(L, kSageBlock);
+      const int nb = (int)cdiv_ll(s_len[r], kSageBlock);
       const uint8_t* m = a.block_mask + (size_t)r * a.mask_pitch;
-      int k = ws.sel_base[r];
-      for (int b0 = 0; b0 < nb; b0 += 32) {
-        const int b = b0 + lane;
-        const bool sel = b < nb && m[b] != 0;
-        const unsigned ballot = __ballot_sync(0xffffffffu, sel);
-        if (sel) ws.sel_block[k + __popc(ballot & ((1u << lane) - 1u))] = b;
-        k += __popc(ballot);
+      int k = s_sel[r];
+      for (int b0 = 0; b0 < nb; b0 += 512) {
+        uint32_t bits = keep && b0 == 0 ? kept_bits : mask_bits(m, b0, nb, lane);
+        const int cnt = __popc(bits);
+        int incl = cnt;                                     // lanes before this one hold lower blocks
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int at = k + incl - cnt;
+        while (bits) {
+          const int i = __ffs(bits) - 1;
+          ws.sel_block[at++] = b0 + 16 * lane + i;
+          bits &= bits - 1;
+        }
+        k += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
   }
-  // 2. g_r = exclusive prefix sum of the units (kept in req_aux), total
-  long long local = 0;
-  for (int r = r0; r < r1; ++r) local += ws.req_prefix[r];
+  // 2. g_r = exclusive prefix sum of the units (written to req_aux), total
+  int local = 0;
+  for (int r = r0; r < r1; ++r) local += s_units[r];
   int total = 0;
-  int run = block_exclusive_scan((int)local, scan, &total);
-  for (int r = r0; r < r1; ++r) {
-    ws.req_aux[r] = run;
-    run += ws.req_prefix[r];
-  }
+  const int run_u = block_exclusive_scan(local, scan, &total);
   const int per = (int)max(1LL, cdiv_ll(total, a.slots));
   const int used = (int)cdiv_ll(total, per);
-  __syncthreads();
   // 3. pieces per request, then req_base
-  for (int r = tid; r < B; r += nt) {
-    const int u = ws.req_prefix[r], g = ws.req_aux[r];
-    ws.req_splits[r] = u > 0 ? (g + u - 1) / per - g / per + 1 : 1;
-  }
-  __syncthreads();
+  auto pieces = [&](int u, int g) { return u > 0 ? (g + u - 1) / per - g / per + 1 : 1; };
   int local_s = 0;
-  for (int r = r0; r < r1; ++r) local_s += ws.req_splits[r];
-  int n_items = 0;
-  int run_s = block_exclusive_scan(local_s, scan, &n_items);
-  for (int r = r0; r < r1; ++r) {
-    ws.req_base[r] = run_s;
-    run_s += ws.req_splits[r];
+  for (int r = r0, g = run_u; r < r1; ++r) {
+    const int u = s_units[r];
+    const int sp = pieces(u, g);
+    ws.req_aux[r] = g;
+    ws.req_splits[r] = sp;
+    local_s += sp;
+    g += u;
   }
+  int n_items = 0;
+  const int run_s = block_exclusive_scan(local_s, scan, &n_items);
   if (tid == 0) ws.req_base[B] = n_items;
   if (n_items > a.max_items) {  // cannot happen (bound slots + B); keep the grid safe
     if (tid == 0) set_device_error(hdr, PA_ERR_DEVICE_INDEX);
     n_items = a.max_items;
   }
-  __syncthreads();
   // 4. the items (key ranges; SAGE_SPARSE: unit ranges) and the slot of each
-  for (int r = tid; r < B; r += nt) {
-    const int L = ws.req_len[r], u = ws.req_prefix[r], g = ws.req_aux[r], base = ws.req_base[r];
+  for (int r = r0, g = run_u, base = run_s; r < r1; ++r) {
+    const int L = s_len[r], u = s_units[r];
+    ws.req_base[r] = base;
     if (u == 0) {
       if (base < n_items) {
         ws.items[base] = make_int4(r, 0, 0, 0);
         item_slot[base] = min(g / per, max(used - 1, 0));
       }
-      continue;
+    } else {
+      const int c_first = g / per, c_last = (g + u - 1) / per;
+      for (int c = c_first; c <= c_last; ++c) {
+        const int i = base + (c - c_first);
+        if (i >= n_items) break;
+        const int u0 = max(g, c * per) - g, u1 = min(g + u, (c + 1) * per) - g;
+        ws.items[i] = sparse ? make_int4(r, c - c_first, u0, u1)
+                             : make_int4(r, c - c_first, u0 * U, (int)min((long long)u1 * U, (long long)L));
+        item_slot[i] = c;
+      }
     }
-    const int c_first = g / per, c_last = (g + u - 1) / per;
-    for (int c = c_first; c <= c_last; ++c) {
-      const int i = base + (c - c_first);
-      if (i >= n_items) break;
-      const int u0 = max(g, c * per) - g, u1 = min(g + u, (c + 1) * per) - g;
-      ws.items[i] = sparse ? make_int4(r, c - c_first, u0, u1)
-                           : make_int4(r, c - c_first, u0 * U, (int)min((long long)u1 * U, (long long)L));
-      item_slot[i] = c;
-    }
+    base += pieces(u, g);
+    g += u;
   }
   for (int c = tid; c <= a.slots; c += nt) ws.slot_first[c] = n_items;
   __syncthreads();
@@ -175,8 +234,6 @@ __device__ void flat_plan(const PlanLaunch& a, int* item_slot, int* scan, int* c
     const int c_prev = i > 0 ? item_slot[i - 1] : -1;
     for (int c = c_prev + 1; c <= item_slot[i]; ++c) ws.slot_first[c] = i;
   }
-  __syncthreads();
-  for (int r = tid; r < B; r += nt) ws.req_prefix[r] = 0;
   *chunk_out = per;
   *n_out = n_items;
 }
@@ -305,9 +362,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanLaunch a) {
 }  // namespace
 
 cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s) {
-  const size_t smem = sizeof(unsigned long long) * (size_t)a.sort_n;
+  // EXTEND: the sort keys; flat modes: 3 ints per request and one per item
+  size_t smem = sizeof(unsigned long long) * (size_t)a.sort_n;
+  if (flat_mode(a.mode)) smem = std::max(smem, sizeof(int) * (3 * (size_t)a.batch + (size_t)a.max_items));
+  constexpr int kSmemMax = (int)std::max(sizeof(unsigned long long) * kMaxSortItems,
+                                         sizeof(int) * (3 * (size_t)kMaxBatch + kMaxSortItems));
   static std::atomic<bool> smem_set[kMaxDevices];
-  cudaError_t e = raise_smem_limit(plan_kernel, (int)(sizeof(unsigned long long) * kMaxSortItems), smem_set);
+  cudaError_t e = raise_smem_limit(plan_kernel, kSmemMax, smem_set);
   if (e != cudaSuccess) return e;
   plan_kernel<<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();

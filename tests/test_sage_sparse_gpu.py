@@ -60,9 +60,11 @@ def oracle(spec, batch, lay, mask):
 
 def test_sparse_plan_bit_exact():
     rng = np.random.default_rng(71)
-    for _ in range(12):
-        B = int(rng.integers(1, 40))
-        spec = wl.Spec("sp_plan", 71, "sage", batch=B, len_lo=0, len_hi=int(rng.integers(1, 9000)), hq=32,
+    # (batch, longest length): rows within one 512-block mask step, and rows of 2-3 steps with
+    # more requests than the plan has warps
+    shapes = [(int(rng.integers(1, 40)), int(rng.integers(1, 9000))) for _ in range(12)] + [(50, 70000), (7, 40000)]
+    for B, len_hi in shapes:
+        spec = wl.Spec("sp_plan", 71, "sage", batch=B, len_lo=0, len_hi=len_hi, hq=32,
                        hkv=int(rng.choice([2, 8, 16])), page_size=64, spare_pages=0.1,
                        density=float(rng.choice([0.0, 0.1, 0.5, 1.0])))
         spec = spec.scaled(hq=spec.hkv * 2)
