@@ -160,6 +160,20 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int s
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
+// An L2 cache policy that marks the lines an access brings in as the first to evict: for data
+// streamed through once (KV tiles), so it does not push out what is read again (partials,
+// score rows, page tables).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+// The same with an L2 cache policy (createpolicy) for the line it reads.
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, int src_bytes, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes), "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

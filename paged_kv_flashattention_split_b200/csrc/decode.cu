@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
     const size_t slot_stride = (size_t)a.hkv * kHeadDim;
     const size_t grp_off = (size_t)grp * HG * kHeadDim + (size_t)ld_c * 8;
     const uint32_t smem_base = smem_u32(smem);
+    const uint64_t policy = l2_evict_first();   // KV rows stream through once
     auto issue = [&](int tile) {
       const uint32_t kst = smem_base + (tile % kStages) * kStageBytes;
       const int32_t* sl = sbuf + (tile & 1) * TK;
@@ -123,8 +124,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitkv_kernel(DecodeLaunc
         const size_t off = slot >= 0 ? (size_t)slot * slot_stride + grp_off : 0;
         const int bytes = slot >= 0 ? 16 : 0;      // rows past the split (or bad ids) are zero-filled
         const uint32_t dst = kst + key * ROW + ((ld_c ^ (key & 7)) << 4);
-        cp_async_16(dst, a.k_pool + off, bytes);
-        cp_async_16(dst + kHalfStage, a.v_pool + off, bytes);
+        cp_async_16_hint(dst, a.k_pool + off, bytes, policy);
+        cp_async_16_hint(dst + kHalfStage, a.v_pool + off, bytes, policy);
       }
     };
 

@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fp8_kernel(Fp8DecodeLaunch
     const size_t slot_stride = (size_t)a.hkv * kHeadDim;
     const size_t grp_off = (size_t)grp * HG * kHeadDim + (size_t)ld_c * 16;
     const uint32_t smem_base = smem_u32(smem);
+    const uint64_t policy = l2_evict_first();   // KV rows stream through once
     auto issue = [&](int tile) {
       const uint32_t kst = smem_base + (tile % kStages) * kStageBytes;
       const int32_t* sl = sbuf + (tile & 1) * TK;
@@ -143,8 +144,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fp8_kernel(Fp8DecodeLaunch
         const size_t off = slot >= 0 ? (size_t)slot * slot_stride + grp_off : 0;
         const int bytes = slot >= 0 ? 16 : 0;      // rows past the split (or bad ids) are zero-filled
         const uint32_t dst = kst + key * ROW + ((ld_c ^ (key & 7)) << 4);
-        cp_async_16(dst, a.k8_pool + off, bytes);
-        cp_async_16(dst + kHalfStage, a.v8_pool + off, bytes);
+        cp_async_16_hint(dst, a.k8_pool + off, bytes, policy);
+        cp_async_16_hint(dst + kHalfStage, a.v8_pool + off, bytes, policy);
       }
     };
 

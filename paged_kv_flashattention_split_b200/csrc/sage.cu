@@ -344,7 +344,9 @@ __device__ __forceinline__ void produce(const SageLaunch& a, const Ring<HG, G, V
           }
           const bool sfk_box = !VPASS && !kSfkLanes && p >= 0;
           mbar_expect_tx(rg.full(s), (p >= 0 ? L::KV : 0) + L::SB + (sfk_box ? HG * 4 : 0));
-          if (p >= 0) tma_load_3d(rg.stage(s), &a.tm_kv, 0, p * kSageBlock + (ks & (kSageBlock - 1)), grp * HG, rg.full(s));
+          if (p >= 0)   // K8 / V8 stream through once: first out of L2, ahead of the score rows
+            tma_load_3d_hint(rg.stage(s), &a.tm_kv, 0, p * kSageBlock + (ks & (kSageBlock - 1)), grp * HG, rg.full(s),
+                             l2_evict_first());
           if (sfk_box) tma_load_2d(smem_u32(rg.sfk(s)), &a.tm_sfk, grp * HG, p, rg.full(s));
           if (VPASS) {
             if (waited) {
