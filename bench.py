@@ -652,6 +652,22 @@ ROOFLINE_KERNELS = {
 DEFAULT_EXTRAS = ("extend_prefix", "sage_decode")
 
 
+def workload_config(name, spec, num_slots, world):
+    """The `config` object of a JSON line: the workload itself, the same for both arms."""
+    cfg = {
+        "workload": name,
+        "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
+        "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
+        "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": num_slots,
+        "step": "attn_plan + %d x %s" % (spec.layers, STEP_CALLS.get(name, "attn_decode_paged")),
+        "l2": "inputs larger than L2 (the step's layers read their own pools, far more than L2)",
+        "parallelism": f"replicas x{world}",
+    }
+    if spec.mode == "extend":
+        cfg["new_lens"] = f"U[{spec.new_lo},{spec.new_hi}]"
+    return cfg
+
+
 def measure(name, spec, args, dist, world, local, rank, peaks, cpu_baseline=True):
     """Run one workload: warm-up, the timed steps (CUDA events, max over ranks), the CUDA-graph replay,
     the end-to-end run through host buffers, and (rank 0, one GPU) the oracle on a bounded sample.
@@ -762,15 +778,7 @@ def measure(name, spec, args, dist, world, local, rank, peaks, cpu_baseline=True
         "vs_baseline": None,
         "dtype": DTYPES.get(name, "bf16"),
         "data": "synthetic",
-        "config": {
-            "workload": name,
-            "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]", "hq": spec.hq, "hkv": spec.hkv,
-            "head_dim": spec.head_dim, "page_size": spec.page_size, "layers": spec.layers,
-            "distinct_pools": spec.distinct_pools or spec.layers, "pool_slots": work.batch.num_slots,
-            "step": "attn_plan + %d x %s" % (spec.layers, STEP_CALLS.get(name, "attn_decode_paged")),
-            "l2": "inputs larger than L2 (the step's layers read their own pools, far more than L2)",
-            "parallelism": f"replicas x{world}",
-        },
+        "config": workload_config(name, spec, work.batch.num_slots, world),
         "roofline": {
             "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -786,8 +794,6 @@ def measure(name, spec, args, dist, world, local, rank, peaks, cpu_baseline=True
     }
     if sustained is not None:
         out["roofline"]["sustained"] = sustained
-    if spec.mode == "extend":
-        out["config"]["new_lens"] = f"U[{spec.new_lo},{spec.new_hi}]"
     if cpu_baseline and rank == 0 and world == 1:
         nbytes, secs, sample = work.oracle_sample()
         out["cpu_baseline"] = {"value": round(nbytes / secs / scale, 6), "unit": unit, "cores": blas_threads(),
@@ -951,9 +957,7 @@ def run_reference(args, spec, cls):
         "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": 0, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * total / max(1, args.steps), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": args.workload, "batch": spec.batch, "seq_lens": f"U[{spec.len_lo},{spec.len_hi}]",
-                   "hq": spec.hq, "hkv": spec.hkv, "head_dim": spec.head_dim, "page_size": spec.page_size,
-                   "layers": spec.layers},
+        "config": workload_config(args.workload, spec, batch.num_slots, 1),
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{per_step} {what} of layer 0 per step, the fp64 oracle (oracle/)"},
         "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
