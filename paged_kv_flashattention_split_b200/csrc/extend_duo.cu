@@ -16,8 +16,10 @@
 // serving two heads alone would load.  Per CTA (10 warps):
 //   warp 0      producer: Q once, then K/V key tiles into 3-stage rings, one TMA box
 //               per page (K boxes complete on the rank-0 CTA's barrier, V boxes on this
-//               CTA's own), or, for pages below 8 slots, 16-byte cp.async gathers that the
-//               warp announces itself once they have landed;
+//               CTA's own), or, for pages below 8 slots, 16-byte cp.async gathers of K that
+//               the warp announces itself once they have landed (V is then gathered by an
+//               eleventh warp, warp 10, the same way: one warp's gathers alone held the
+//               slot-granular cache at half the rate);
 //   warp 1      TMEM (512 columns: S_0, S_1, O_0, O_1) and, in the rank-0 CTA, the MMA
 //               issuer;
 //   warps 2-9   one softmax warpgroup per head: thread i owns query row i, reads S_t from
@@ -40,6 +42,7 @@ namespace pa {
 namespace {
 
 constexpr int kThreads = 320;
+constexpr int kThreadsGather = 352;               // + one warp that gathers V (page sizes below 8)
 constexpr int kTileKeys = 128;
 constexpr int kStages = 3;
 constexpr int kQTile = 128 * 256;                    // 128 rows x 128 d bf16 = 32 KB (2 chunks of 64 d)
@@ -204,7 +207,7 @@ constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);   // A (P) K-major, B (V)
 // GATHER: the page-size-below-8 path (cp.async gathers); a separate instantiation, so the TMA
 // path's register allocation carries none of the gather code.
 template <bool GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GATHER ? kThreadsGather : kThreads, 1)
     extend_duo_kernel(const __grid_constant__ DuoLaunch a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -300,39 +303,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (GATHER) {
       // the copies complete on no barrier, so the warp announces them: once K(j) is issued it
       // waits for K(j - 1)'s copies, fences them for the tensor cores (async proxy) and arrives
-      // on the rank-0 CTA's KFULL; the same for V (this CTA's VLAND) after V(j) is issued.
-      // Copy groups are committed K(0), V(0), K(1), V(1), ...: two newer groups each time.
-      auto announce = [&](uint32_t full_bar_cluster) {
-        cp_async_wait<2>();
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(full_bar_cluster);
-      };
+      // on the rank-0 CTA's KFULL (V is gathered the same way by warp 10, on this CTA's VLAND).
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
-        const int nk = half_keys(j, (int)rank), nv = tile_keys(j);
+        const int nk = half_keys(j, (int)rank);
         bool ok = true;
         if (lane == 0) ok = j < kStages || wait(bar(B_KEMPTY + s), stage_parity(j) ^ 1u);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         gather_rows<2, 64>(base + kOffK + s * kKStage, kKChunk, 0, a.k_pool, table, j * kTileKeys + 64 * (int)rank, nk,
                        (nk + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
         cp_async_commit();
-        if (j > 0) announce(map_to_rank(bar(B_KFULL + (j - 1) % kStages), 0));
-        if (lane == 0) ok = j < kStages || wait(bar(B_VEMPTY + s), stage_parity(j) ^ 1u);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        gather_rows<1, 128>(base + kOffV + s * kVStage, kVStage, (int)rank, a.v_pool, table, j * kTileKeys, nv,
-                       (nv + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
-        cp_async_commit();
-        if (j > 0) announce(map_to_rank(bar(B_VLAND + (j - 1) % kStages), rank));
+        if (j > 0) {
+          cp_async_wait<1>();
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_to_rank(bar(B_KFULL + (j - 1) % kStages), 0));
+        }
         issued = j + 1;
       }
       cp_async_wait<0>();
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0 && issued > 0) {
-        mbar_arrive_cluster(map_to_rank(bar(B_KFULL + (issued - 1) % kStages), 0));
-        mbar_arrive(bar(B_VLAND + (issued - 1) % kStages));
-      }
+      if (lane == 0 && issued > 0) mbar_arrive_cluster(map_to_rank(bar(B_KFULL + (issued - 1) % kStages), 0));
       issued = 0;                                                // nothing left in flight
     }
     for (int j = 0; !GATHER && j < n_kv; ++j) {
@@ -376,6 +368,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar(B_VLAND + j % kStages), stage_parity(j)); ++i) {}
       }
     }
+  } else if (GATHER && warp == 10) {
+    // ------------------------------------------------------------ V gathers (page sizes below 8)
+    const int32_t* table = a.page_table + (size_t)r * a.pt_pitch;
+    int vissued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j % kStages;
+      const int nv = tile_keys(j);
+      bool ok = true;
+      if (lane == 0) ok = j < kStages || wait(bar(B_VEMPTY + s), stage_parity(j) ^ 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      gather_rows<1, 128>(base + kOffV + s * kVStage, kVStage, (int)rank, a.v_pool, table, j * kTileKeys, nv,
+                          (nv + 15) & ~15, a.page_shift, a.page_size, a.hkv, h_kv, a.num_slots, hdr, lane);
+      cp_async_commit();
+      if (j > 0) {
+        cp_async_wait<1>();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_VLAND + (j - 1) % kStages));
+      }
+      vissued = j + 1;
+    }
+    cp_async_wait<0>();
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0 && vissued > 0) mbar_arrive(bar(B_VLAND + (vissued - 1) % kStages));
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (rank 0 only)
     if (leader && lane == 0) {
@@ -642,7 +659,7 @@ cudaError_t launch_extend_duo(const ExtendArgs& in, cudaStream_t s) {
   a.box_k = box_k;
   a.box_v = box_v;
   if (a.gather)
-    extend_duo_kernel<true><<<in.max_items * (in.hq / 4) * 2, kThreads, kSmemBytes, s>>>(a);
+    extend_duo_kernel<true><<<in.max_items * (in.hq / 4) * 2, kThreadsGather, kSmemBytes, s>>>(a);
   else
     extend_duo_kernel<false><<<in.max_items * (in.hq / 4) * 2, kThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();
