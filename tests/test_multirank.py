@@ -63,6 +63,12 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload object as this arm's line (one rank per GPU: parallelism replicas x1)
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    spec = wl.SPECS["decode_tiny"]
+    assert d["config"] == bench.workload_config("decode_tiny", spec, wl.make_batch(spec, "cpu").num_slots, 1)
 
 
 def test_clock_summary_keeps_the_timed_region():
